@@ -1,0 +1,262 @@
+"""CPU oracle for Reduced Matrix Multiplication (RMM) -- TEST INFRASTRUCTURE ONLY.
+
+Only the test-suite, the package's smoke check and the benchmark's CPU-baseline
+leg may import or run this module.  The product path (the CUDA library and its
+Python binding) never calls it and shares no code with it.
+
+It restates, plainly and slowly in float64 with numpy, what RMM computes.  Every
+function cites the page passage it follows.  Pages (by title):
+
+  [DD]   "Algorithm Deep-Dive: RMM -- TopK Column-Norm Slicing: Formulas, 1B-70B
+          Results, and the Attention/MLP Asymmetry" (hackcv.com)
+  [KB]   "RMM：把 Transformer 矩阵乘法切到刚好够用" (kaelemshawn.blog)
+  [GS]   "Reduced Matrix Multiplication: Input-Adaptive Matrix-Product Reduction
+          for LLM Inference", Technical Summary (gist.science)
+
+Readings where the pages are silent (each is also pinned by a test):
+  * k = ceil(rho*d), computed as ceil(x - 1e-9*x) with x = rho*d so that a
+    product such as 0.1*30 = 3.0000000000000004 still gives 3; clamped to [1, d].
+  * Ties in the column norm: the lower index wins.  The index set is returned
+    in ascending order.
+  * Retained energy = sum_{j in I} s_j^2 / sum_j s_j^2.
+  * Causal attention (QK^T and PV) is bottom-right aligned: key j is visible to
+    query i iff j <= i + (nk - nq).  Masked scores are -inf; masked entries of
+    P are treated as zero (they are neither read for the norms nor multiplied).
+  * GQA: query head h reads key/value head h // (Hq // Hkv).
+
+Parity: every function here is pinned by tests/test_oracle.py against
+hand-derived fixtures, closed forms, brute force or invariants; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "retention_count", "column_sq_norms", "column_norms", "topk_ascending",
+    "retained_energy", "select", "reduced_product", "error_bound", "rmm_linear",
+    "rmm_linear_rows", "kv_head", "rmm_qk", "rmm_qk_rows", "rmm_pv", "rmm_pv_rows",
+    "near_tie_band",
+]
+
+
+def retention_count(rho: float, d: int) -> int:
+    """k = ceil(rho * d), the number of contraction indices kept.
+
+    [DD] "The retention-ratio (rho) Knob": rho in (0, 1] keeps ceil(rho d) dims;
+    [KB] "先把...想清楚": |I| = ceil(rho d); [GS] Methodology, Selection Strategy.
+    """
+    rho = float(rho)
+    d = int(d)
+    if not (rho > 0.0 and rho <= 1.0) or d < 1:
+        raise ValueError(f"rho must lie in (0, 1] and d >= 1 (rho={rho}, d={d})")
+    x = rho * d
+    k = math.ceil(x - 1e-9 * x)
+    return max(1, min(d, k))
+
+
+def _visible_cols(i: int, nq: int, nk: int) -> int:
+    """Number of key positions visible to query row i under bottom-right causal alignment."""
+    return max(0, min(nk, i + (nk - nq) + 1))
+
+
+def column_sq_norms(A: np.ndarray, causal: bool = False) -> np.ndarray:
+    """q_j = sum_i A[i, j]^2 in float64, summed in row order.
+
+    The importance score is the activation column L2 norm s_j = ||A[:, j]||_2
+    ([DD] "Contraction-Dimension TopK Selection"; [GS] Selection Strategy); this
+    returns its square.  With ``causal`` the entries above the bottom-right
+    aligned diagonal are treated as zero (attention probabilities P).
+    """
+    A = np.asarray(A, dtype=np.float64)
+    n, d = A.shape
+    q = np.zeros(d, dtype=np.float64)
+    for i in range(n):
+        lim = _visible_cols(i, n, d) if causal else d
+        if lim > 0:
+            row = A[i, :lim]
+            q[:lim] += row * row
+    return q
+
+
+def column_norms(A: np.ndarray, causal: bool = False) -> np.ndarray:
+    """s_j = ||A[:, j]||_2 ([DD] "Contraction-Dimension TopK Selection")."""
+    return np.sqrt(column_sq_norms(A, causal))
+
+
+def topk_ascending(s: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest scores, ties to the lower index, returned ascending.
+
+    [DD] "take TopK-largest ceil(rho d)"; [GS] "The top-k indices with the
+    highest scores are retained".  Order: by score descending, then index
+    ascending; keep the first k; sort the kept indices ascending.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    d = s.shape[0]
+    if not (1 <= k <= d):
+        raise ValueError("k out of range")
+    order = np.lexsort((np.arange(d), -s))
+    return np.sort(order[:k]).astype(np.int64)
+
+
+def retained_energy(q: np.ndarray, I: np.ndarray) -> float:
+    """sum_{j in I} s_j^2 / sum_j s_j^2 (reading of the pages' "retained activation
+    energy", [DD] "Attention vs MLP: structural asymmetry", supplementary note)."""
+    total = float(np.sum(q))
+    return float(np.sum(q[I])) / total if total > 0 else 1.0
+
+
+def near_tie_band(s: np.ndarray, k: int, rel: float = 1e-5) -> np.ndarray:
+    """Indices j whose norm lies within ``rel`` (relative) of the k-th largest norm.
+
+    Selections that differ only inside this band are all correct up to rounding
+    of the scores; parity tests accept (and log) differences there."""
+    s = np.asarray(s, dtype=np.float64)
+    kth = np.sort(s)[::-1][k - 1]
+    return np.nonzero(np.abs(s - kth) <= rel * abs(kth))[0]
+
+
+def select(A: np.ndarray, rho: float, causal: bool = False):
+    """Score, count and TopK: returns (I, q, retained) for one activation matrix.
+
+    [DD] "Core Approach (Formula Level)"; [GS] Methodology items 1-2.
+    """
+    A = np.asarray(A, dtype=np.float64)
+    d = A.shape[1]
+    k = retention_count(rho, d)
+    q = column_sq_norms(A, causal)
+    I = topk_ascending(np.sqrt(q), k)
+    return I, q, retained_energy(q, I)
+
+
+def reduced_product(A: np.ndarray, B: np.ndarray, I: np.ndarray) -> np.ndarray:
+    """RMM_rho(A, B) = A[:, I] . B[I, :] in float64.
+
+    [DD] "Contraction-Dimension TopK Selection"; [KB] "RMMρ(A, B) = A[:, I] B[I, :]";
+    [GS] Core Mechanism.  Weights are not modified; rows of B outside I are skipped.
+    """
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    return A[:, I] @ B[I, :]
+
+
+def error_bound(A: np.ndarray, B: np.ndarray, I: np.ndarray) -> float:
+    """sum_{j not in I} ||A[:, j]||_2 * ||B[j, :]||_2 ([DD] "Properties", error bound)."""
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    keep = np.zeros(A.shape[1], dtype=bool)
+    keep[I] = True
+    s = column_norms(A)
+    b = np.sqrt(np.sum(B * B, axis=1))
+    return float(np.sum(s[~keep] * b[~keep]))
+
+
+def rmm_linear(A: np.ndarray, B: np.ndarray, rho: float):
+    """Reduced linear projection Y = X[:, I] W[I, :] with I chosen on X.
+
+    [DD] "Component mapping": MLP/linear projections select along the activation
+    hidden dim; [KB] "在线性投影和 MLP 里"; [GS] Application Scope (XW).
+    Returns dict(Y, I, q, retained).
+    """
+    I, q, ret = select(A, rho)
+    return {"Y": reduced_product(A, B, I), "I": I, "q": q, "retained": ret}
+
+
+def rmm_linear_rows(A: np.ndarray, B: np.ndarray, I: np.ndarray, rows) -> np.ndarray:
+    """Rows ``rows`` of A[:, I] . B[I, :] (for sampled checks of large products)."""
+    A = np.asarray(A, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    rows = np.asarray(rows)
+    return A[rows][:, I] @ B[I, :]
+
+
+def kv_head(h: int, hq: int, hkv: int) -> int:
+    """Key/value head read by query head h under GQA: h // (Hq // Hkv)."""
+    if hq % hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return h // (hq // hkv)
+
+
+def _qk_head(Qh, Kg, rho, causal, scale, rows=None):
+    nq, dh = Qh.shape
+    nk = Kg.shape[0]
+    k = retention_count(rho, dh)
+    q = column_sq_norms(Qh)
+    I = topk_ascending(np.sqrt(q), k)
+    r = np.arange(nq) if rows is None else np.asarray(rows)
+    S = scale * (Qh[r][:, I] @ Kg[:, I].T)
+    if causal:
+        vis = np.array([_visible_cols(i, nq, nk) for i in r])
+        S[np.arange(nk)[None, :] >= vis[:, None]] = -np.inf
+    return S, I
+
+
+def rmm_qk(Q: np.ndarray, K: np.ndarray, rho: float, causal: bool = True, scale: float = 1.0):
+    """Reduced attention scores S_h = scale * Q_h[:, I_h] K_g(h)[:, I_h]^T per query head.
+
+    [DD] "Component mapping": QK^T selects along the head feature dim with score =
+    Q column norm; under GQA the selection is made on Q per head and K gathers the
+    corresponding dims.  [KB] "计算 attention score 时"; [GS] Application Scope.
+    Q [B, Hq, nq, dh], K [B, Hkv, nk, dh] -> S [B, Hq, nq, nk] (float64, -inf where
+    masked), I [B, Hq, k].
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    Bsz, hq, nq, dh = Q.shape
+    hkv, nk = K.shape[1], K.shape[2]
+    k = retention_count(rho, dh)
+    S = np.empty((Bsz, hq, nq, nk))
+    I = np.empty((Bsz, hq, k), dtype=np.int64)
+    for b in range(Bsz):
+        for h in range(hq):
+            S[b, h], I[b, h] = _qk_head(Q[b, h], K[b, kv_head(h, hq, hkv)], rho, causal, scale)
+    return {"S": S, "I": I}
+
+
+def rmm_qk_rows(Qh: np.ndarray, Kg: np.ndarray, rho: float, rows, causal=True, scale=1.0):
+    """Rows ``rows`` of one head's reduced scores: Qh [nq, dh] (the query head),
+    Kg [nk, dh] (its GQA key head).  Returns (S_rows, I)."""
+    return _qk_head(np.asarray(Qh, dtype=np.float64), np.asarray(Kg, dtype=np.float64),
+                    rho, causal, scale, rows)
+
+
+def _pv_head(Ph, Vg, rho, causal, rows=None):
+    nq, nk = Ph.shape
+    k = retention_count(rho, nk)
+    q = column_sq_norms(Ph, causal)
+    I = topk_ascending(np.sqrt(q), k)
+    r = np.arange(nq) if rows is None else np.asarray(rows)
+    Pr = Ph[r][:, I].copy()
+    if causal:
+        vis = np.array([_visible_cols(i, nq, nk) for i in r])
+        Pr[I[None, :] >= vis[:, None]] = 0.0
+    return Pr @ Vg[I, :], I, q
+
+
+def rmm_pv(P: np.ndarray, V: np.ndarray, rho: float, causal: bool = True):
+    """Reduced attention output O_h = P_h[:, I_h] V_g(h)[I_h, :] per head.
+
+    [DD] "Component mapping": PV optionally selects along token positions;
+    [KB] "计算 attention output 时": P's norm over positions decides which V rows
+    take part; [GS] Application Scope.  The score of key position j is the norm of
+    column j of P over all query rows.  P [B, H, nq, nk], V [B, Hkv, nk, dh] ->
+    O [B, H, nq, dh], I [B, H, k].
+    """
+    P = np.asarray(P, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    Bsz, h_, nq, nk = P.shape
+    hkv, dh = V.shape[1], V.shape[3]
+    k = retention_count(rho, nk)
+    O = np.empty((Bsz, h_, nq, dh))
+    I = np.empty((Bsz, h_, k), dtype=np.int64)
+    for b in range(Bsz):
+        for h in range(h_):
+            O[b, h], I[b, h], _ = _pv_head(P[b, h], V[b, kv_head(h, h_, hkv)], rho, causal)
+    return {"O": O, "I": I}
+
+
+def rmm_pv_rows(Ph: np.ndarray, Vg: np.ndarray, rho: float, rows, causal=True):
+    """Rows ``rows`` of one head's reduced PV output.  Returns (O_rows, I, q)."""
+    return _pv_head(np.asarray(Ph, dtype=np.float64), np.asarray(Vg, dtype=np.float64), rho, causal, rows)

@@ -1,0 +1,263 @@
+"""Pins for the CPU oracle: it is checked against things other than itself.
+
+Hand-derived fixtures (tests/golden/*.json, each with its citation), closed
+forms, brute force over all subsets on tiny d, and invariants of the
+mathematics.  Each check is chosen so that a plausible slip in the oracle (row
+norms instead of column norms, the wrong tie rule, a dropped term, a transposed
+or mismatched operand, the wrong GQA head, a causal mask off by one) fails.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------- k = ceil(rho d)
+def test_retention_count_table():
+    fx = load("retention_count.json")
+    for rho, d, k in fx["cases"]:
+        assert oracle.retention_count(rho, d) == k, (rho, d)
+    for rho, d in fx["invalid"]:
+        rho = float(rho)
+        with pytest.raises(ValueError):
+            oracle.retention_count(rho, d)
+
+
+# ----------------------------------------------------------------- hand fixtures
+def test_linear_hand_fixture():
+    fx = load("linear_hand.json")
+    A = np.array(fx["A"], float)
+    B = np.array(fx["B"], float)
+    assert np.array_equal(oracle.column_sq_norms(A), np.array(fx["colsq"], float))
+    for case in fx["cases"]:
+        out = oracle.rmm_linear(A, B, case["rho"])
+        assert out["I"].tolist() == case["I"], case["rho"]
+        assert len(out["I"]) == case["k"]
+        assert out["retained"] == pytest.approx(case["retained_num"] / case["retained_den"], abs=1e-15)
+        if "Y" in case:
+            assert np.array_equal(out["Y"], np.array(case["Y"], float))
+        if "err_fro_sq" in case:
+            dense = np.array(fx["dense"], float)
+            err = np.sum((dense - out["Y"]) ** 2)
+            assert err == case["err_fro_sq"]
+            bound = case["bound_int"] + case["bound_sqrt5"] * math.sqrt(5)
+            assert oracle.error_bound(A, B, out["I"]) == pytest.approx(bound, rel=1e-14)
+
+
+def test_qk_hand_fixture_and_gqa():
+    fx = load("qk_hand.json")
+    Q = np.array(fx["Q"], float)
+    K = np.array(fx["K"], float)
+    exp_c = np.array([[[np.nan if v is None else v for v in row] for row in h] for h in fx["S_causal"][0]])
+    exp_f = np.array(fx["S_full"][0], float)
+    out = oracle.rmm_qk(Q, K, fx["rho"], causal=True)
+    assert out["I"].tolist() == fx["I"]
+    S = out["S"][0]
+    assert np.array_equal(np.isneginf(S), np.isnan(exp_c))
+    fin = ~np.isnan(exp_c)
+    assert np.array_equal(S[fin], exp_c[fin])
+    full = oracle.rmm_qk(Q, K, fx["rho"], causal=False, scale=0.5)
+    assert np.array_equal(full["S"][0], 0.5 * exp_f)
+    # GQA: Hq = 4, Hkv = 2; query heads 2,3 repeat 0,1 and must read key head 1 = 10 K.
+    f = fx["gqa_key_head1_factor"]
+    Q4 = np.concatenate([Q, Q], axis=1)
+    K2 = np.concatenate([K, f * K], axis=1)
+    g = oracle.rmm_qk(Q4, K2, fx["rho"], causal=False)
+    assert np.array_equal(g["S"][0, :2], exp_f)
+    assert np.array_equal(g["S"][0, 2:], f * exp_f)
+    assert [oracle.kv_head(h, 4, 2) for h in range(4)] == [0, 0, 1, 1]
+    assert [oracle.kv_head(h, 32, 8) for h in (0, 3, 4, 31)] == [0, 0, 1, 7]
+
+
+def test_pv_hand_fixture():
+    fx = load("pv_hand.json")
+    P = np.array(fx["P"], float)
+    V = np.array(fx["V"], float)
+    c = oracle.rmm_pv(P, V, fx["rho"], causal=True)
+    assert c["I"][0, 0].tolist() == fx["causal"]["I"]
+    assert np.array_equal(c["O"][0, 0], np.array(fx["causal"]["O"], float))
+    assert np.array_equal(oracle.column_sq_norms(P[0, 0], causal=True), np.array(fx["causal"]["colsq"], float))
+    nc = oracle.rmm_pv(P, V, fx["rho"], causal=False)
+    assert nc["I"][0, 0].tolist() == fx["noncausal"]["I"]
+    assert np.array_equal(nc["O"][0, 0], np.array(fx["noncausal"]["O"], float))
+
+
+# ----------------------------------------------------------------- brute force
+def _unit_columns(g, n, d):
+    U = g.standard_normal((n, d))
+    return U / np.sqrt(np.sum(U * U, axis=0))[None, :]
+
+
+def test_topk_maximises_retained_mass_bruteforce_known_norms():
+    """Theorem 1 in checkable form: over all |S| = k subsets, the chosen set has the
+    largest retained column-norm mass sum_{j in S} s_j (and energy sum s_j^2).  The
+    columns are built with known norms c_j (A[:, j] = c_j u_j, u_j unit), so the
+    test does not recompute norms from A."""
+    g = np.random.Generator(np.random.PCG64(7))
+    d, k, n = 12, 6, 16
+    subsets = np.array(list(itertools.combinations(range(d), k)))
+    for _ in range(100):
+        c = np.exp(g.standard_normal(d))
+        A = _unit_columns(g, n, d) * c[None, :]
+        I, _, _ = oracle.select(A, 0.5)
+        mass = c[subsets].sum(axis=1)
+        best = subsets[np.argmax(mass)]
+        assert I.tolist() == best.tolist()
+        assert c[I].sum() >= mass.max() * (1 - 1e-12)
+        assert (c[I] ** 2).sum() >= (c[subsets] ** 2).sum(axis=1).max() * (1 - 1e-12)
+
+
+def test_topk_bruteforce_with_ties_lexicographic():
+    """Equal norms: the lexicographically smallest maximiser is chosen."""
+    d, k = 12, 6
+    c = np.array([3, 1, 3, 2, 3, 1, 2, 3, 2, 1, 3, 2], float)
+    # exact column norms: column j is c_j times a basis vector (a permuted diagonal)
+    A = np.zeros((d, d))
+    A[(np.arange(d) * 5) % d, np.arange(d)] = c
+    I, _, _ = oracle.select(A, 0.5)
+    subsets = list(itertools.combinations(range(d), k))
+    mass = [sum(c[list(s)]) for s in subsets]
+    best = max(mass)
+    first = min(s for s, m in zip(subsets, mass) if m == best)
+    assert first == (0, 2, 3, 4, 7, 10)
+    assert tuple(I.tolist()) == first
+
+
+def test_row_norms_would_fail():
+    """Rows and columns carry different norms: selecting on row norms (a transposed
+    score) picks a different set than the known column norms."""
+    A = np.array([[10.0, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0], [0, 0, 0, 2], [0, 9, 0, 0]])
+    I, q, _ = oracle.select(A, 0.5)
+    assert q.tolist() == [100.0, 82.0, 1.0, 4.0]
+    assert I.tolist() == [0, 1]
+
+
+def test_all_equal_norms_pick_prefix_and_k1_argmax():
+    for d in (1, 5, 12, 64):
+        A = np.ones((3, d))
+        for rho in (0.25, 0.5, 1.0):
+            k = oracle.retention_count(rho, d)
+            I, _, _ = oracle.select(A, rho)
+            assert I.tolist() == list(range(k))
+    g = np.random.Generator(np.random.PCG64(11))
+    for _ in range(20):
+        A = g.standard_normal((5, 40))
+        norms2 = [sum(A[i, j] ** 2 for i in range(5)) for j in range(40)]
+        I, _, _ = oracle.select(A, 1e-6)
+        assert I.tolist() == [int(np.argmax(norms2))]
+
+
+def test_reduced_product_bruteforce_loops():
+    """A[:, I] B[I, :] against explicit Python loops on tiny random inputs."""
+    g = np.random.Generator(np.random.PCG64(5))
+    for _ in range(25):
+        n, d, m = g.integers(1, 6), g.integers(1, 9), g.integers(1, 6)
+        A = g.standard_normal((n, d))
+        B = g.standard_normal((d, m))
+        k = int(g.integers(1, d + 1))
+        I = np.sort(g.choice(d, size=k, replace=False))
+        Y = oracle.reduced_product(A, B, I)
+        for i in range(n):
+            for c in range(m):
+                ref = 0.0
+                for j in I:
+                    ref += A[i, j] * B[j, c]
+                assert Y[i, c] == pytest.approx(ref, rel=1e-12, abs=1e-12)
+
+
+def test_identity_weight_masks_columns():
+    g = np.random.Generator(np.random.PCG64(9))
+    A = g.standard_normal((7, 10)) * np.exp(g.standard_normal(10))[None, :]
+    out = oracle.rmm_linear(A, np.eye(10), 0.4)
+    expect = np.zeros_like(A)
+    expect[:, out["I"]] = A[:, out["I"]]
+    assert np.array_equal(out["Y"], expect)
+
+
+def test_rho_one_is_the_dense_product_bruteforce():
+    g = np.random.Generator(np.random.PCG64(13))
+    A = g.standard_normal((4, 6))
+    B = g.standard_normal((6, 3))
+    Y = oracle.rmm_linear(A, B, 1.0)["Y"]
+    for i in range(4):
+        for c in range(3):
+            assert Y[i, c] == pytest.approx(sum(A[i, j] * B[j, c] for j in range(6)), rel=1e-12)
+
+
+def test_error_bound_holds_on_tiny_draws():
+    for A, B in synthetic.tiny_bruteforce_set(draws=100):
+        out = oracle.rmm_linear(A, B, 0.5)
+        dense = np.array([[sum(A[i, j] * B[j, c] for j in range(A.shape[1])) for c in range(B.shape[1])]
+                          for i in range(A.shape[0])])
+        err = math.sqrt(float(np.sum((dense - out["Y"]) ** 2)))
+        assert err <= oracle.error_bound(A, B, out["I"]) * (1 + 1e-12) + 1e-300
+
+
+def test_nested_sets_monotone_energy_scale_invariance():
+    g = np.random.Generator(np.random.PCG64(17))
+    for _ in range(10):
+        A = g.standard_normal((9, 33)) * np.exp(1.5 * g.standard_normal(33))[None, :]
+        prev, prev_e = set(), 0.0
+        for rho in (0.1, 0.3, 0.5, 0.7, 0.9, 1.0):
+            I, _, e = oracle.select(A, rho)
+            assert prev <= set(I.tolist())
+            assert e >= prev_e - 1e-15
+            prev, prev_e = set(I.tolist()), e
+            I2, _, _ = oracle.select(A * 4.0, rho)
+            assert np.array_equal(I, I2)
+        assert prev_e == 1.0
+
+
+def test_permutation_equivariance():
+    g = np.random.Generator(np.random.PCG64(19))
+    A = g.standard_normal((6, 20)) * np.exp(g.standard_normal(20))[None, :]
+    B = g.standard_normal((20, 5))
+    perm = g.permutation(20)
+    a = oracle.rmm_linear(A, B, 0.5)
+    b = oracle.rmm_linear(A[:, perm], B[perm, :], 0.5)
+    assert sorted(perm[b["I"]].tolist()) == a["I"].tolist()
+    assert np.allclose(a["Y"], b["Y"], rtol=1e-12, atol=1e-12)
+
+
+def test_causal_alignment_bottom_right():
+    Q = np.ones((1, 1, 2, 4))
+    K = np.ones((1, 1, 5, 4))
+    S = oracle.rmm_qk(Q, K, 1.0, causal=True)["S"][0, 0]
+    # nq = 2, nk = 5: query i sees keys j <= i + 3
+    assert np.isfinite(S).tolist() == [[True] * 4 + [False], [True] * 5]
+    P = np.ones((1, 1, 2, 5))
+    V = np.arange(10, dtype=float).reshape(1, 1, 5, 2)
+    O = oracle.rmm_pv(P, V, 1.0, causal=True)["O"][0, 0]
+    assert O.tolist() == [[0 + 2 + 4 + 6, 1 + 3 + 5 + 7], [20, 25]]
+
+
+def test_near_tie_band():
+    s = np.array([1.0, 2.0, 2.0 * (1 + 5e-6), 3.0, 2.0 * (1 - 2e-5)])
+    band = oracle.near_tie_band(s, 3)
+    assert band.tolist() == [1, 2]
+
+
+def test_synthetic_generators_are_seeded_and_shaped():
+    A, B = synthetic.linear_small()
+    A2, _ = synthetic.linear_small()
+    assert tuple(A.shape) == (128, 1024) and tuple(B.shape) == (1024, 1024)
+    assert bool((A == A2).all())
+    Q, K = synthetic.qk_inputs(hq=4, hkv=2, n=64)
+    assert tuple(Q.shape) == (1, 4, 64, 128) and tuple(K.shape) == (1, 2, 64, 128)
+    P, V = synthetic.pv_inputs(heads=2, n=64)
+    Pw = synthetic.widen(P)
+    assert np.allclose(Pw.sum(axis=-1), 1.0, atol=2e-2)
+    assert np.all(np.triu(Pw[0, 0], 1) == 0)
