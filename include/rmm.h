@@ -1,0 +1,156 @@
+/*
+ * rmm.h -- C ABI of the B200 (sm_100a) Reduced Matrix Multiplication library.
+ *
+ * Reduced Matrix Multiplication (RMM) replaces a product Y = A.B, with A (n x d)
+ * the activations and B (d x m), by the reduced product over the contraction
+ * indices whose activation columns carry the most energy:
+ *
+ *     s_j = ||A[:, j]||_2,   I = TopK_{k}(s),   k = ceil(rho * d),
+ *     RMM_rho(A, B) = A[:, I] . B[I, :]
+ *
+ * Source: "Algorithm Deep-Dive: RMM -- TopK Column-Norm Slicing" (hackcv.com),
+ * section "Core Approach (Formula Level)"; the same statement appears in
+ * "RMM：把 Transformer 矩阵乘法切到刚好够用" (kaelemshawn.blog) and in the
+ * gist.science technical summary of "Reduced Matrix Multiplication:
+ * Input-Adaptive Matrix-Product Reduction for LLM Inference", Methodology.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Element types: activations, weights and products are bfloat16, passed as
+ *    raw 16-bit patterns (rmm_bf16).  Accumulation is fp32 on the tensor cores;
+ *    bf16 outputs are rounded to nearest even.  Column scores are fp64.
+ *  - Layouts are row-major.  Leading dimensions (lda, ldb, ldy) count elements.
+ *  - Index sets are int32, strictly ascending, of length k; ties in the column
+ *    norm go to the lower index.
+ *  - Ownership: the caller owns every buffer.  Device pointers must point to
+ *    memory of the current CUDA device.  The library allocates nothing,
+ *    keeps no state between calls and never synchronises: all work is enqueued
+ *    on `stream` (an opaque cudaStream_t; NULL is the legacy default stream).
+ *    Scratch memory is the caller's `ws` buffer of at least the size returned
+ *    by the matching *_workspace_bytes() query (0 bytes is valid when the
+ *    query returns 0).  Calls that share one workspace must be ordered.
+ *  - Alignment: device pointers must be 16-byte aligned and leading dimensions
+ *    multiples of 8 elements; otherwise RMM_ERR_UNSUPPORTED is returned.
+ *  - Errors: argument problems are detected on the host and returned before
+ *    anything is enqueued.  A failed launch returns RMM_ERR_CUDA.  Device-side
+ *    faults surface on the caller's next synchronisation.  A kernel that waits
+ *    on a barrier for about a second without progress gives up, records a code
+ *    read by rmm_device_error(), and returns.  rmm_last_error() describes the
+ *    most recent failure on the calling thread.
+ *  - There is no CPU fallback: every compute step runs in the library's CUDA
+ *    kernels (sm_100a only).
+ */
+#ifndef RMM_H_
+#define RMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t rmm_bf16; /* IEEE bfloat16 bit pattern */
+typedef void* rmm_stream;  /* cudaStream_t */
+
+typedef enum {
+  RMM_OK = 0,
+  RMM_ERR_INVALID_ARG = 1,    /* bad rho, negative or zero size, null pointer, Hq % Hkv != 0 ... */
+  RMM_ERR_UNSUPPORTED = 2,    /* misaligned pointer / leading dim, size beyond the documented limits */
+  RMM_ERR_WORKSPACE = 3,      /* ws_bytes smaller than the query's answer, or ws == NULL when needed */
+  RMM_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  RMM_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up on a bounded wait (see rmm_device_error) */
+} rmm_status;
+
+/* k = ceil(rho * d): the number of kept contraction indices.
+ * ("The retention-ratio (rho) Knob": rho in (0, 1] keeps ceil(rho d) dims.)
+ * Computed as ceil(x - 1e-9 x) with x = rho * d, so that products which land a
+ * rounding step above an integer (0.1 * 30 = 3.0000000000000004) give the
+ * intended value; clamped to [1, d].  Returns -1 if rho is not in (0, 1]
+ * (NaN included) or d < 1. */
+int64_t rmm_k(double rho, int64_t d);
+
+/* ---------------------------------------------------------------- selection
+ * rmm_select: column scores and TopK index set ("Core Approach": s_j =
+ * ||A[:, j]||_2, keep the TopK-largest ceil(rho d)).  Batched: item b's matrix
+ * starts at A + b * batch_stride (elements), n rows x d columns, leading
+ * dimension lda.
+ *   causal      0, or 1 to treat entries (i, j) with j > i + (d - n) as zero
+ *               (bottom-right aligned causal attention probabilities; they are
+ *               not read).
+ *   idx_out     device int32 [batch][k], k = rmm_k(rho, d); required.
+ *   colsq_out   device fp64 [batch][d] or NULL: q_j = sum_i A[i, j]^2.
+ *   retained_out device fp64 [batch] or NULL: sum_{j in I} q_j / sum_j q_j.
+ * Limits: d <= 32768, n < 2^31.  Workspace: rmm_select_workspace_bytes(). */
+size_t rmm_select_workspace_bytes(int64_t batch, int64_t n, int64_t d);
+rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, int64_t n, int64_t d, int64_t lda,
+                      int causal, double rho, int32_t* idx_out, double* colsq_out, double* retained_out, void* ws,
+                      size_t ws_bytes, rmm_stream stream);
+
+/* ---------------------------------------------------------------- linear
+ * rmm_linear: Y = A[:, I] . B[I, :] with I selected on A (linear and MLP
+ * projections X.W reduce the activation hidden dim: "Core Approach",
+ * component mapping).
+ *   A   device bf16 [n][lda], n x d activations.
+ *   B   device bf16 [d][ldb], d x m, the contraction index is the ROW (the
+ *       transpose of a torch nn.Linear weight, stored once; weights are not
+ *       modified, rows outside I are simply not read).
+ *   Y   device bf16 [n][ldy], n x m output.
+ *   idx_out  device int32 [k] or NULL: the index set used.
+ * rho == 1 runs the dense product A.B (no scores, no selection, no pack).
+ * n <= 32 runs the decode path (a gathered GEMV-shaped kernel that streams only
+ * the kept rows of B).  Limits: d <= 32768, n, m < 2^31. */
+size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho);
+rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const rmm_bf16* B, int64_t m,
+                      int64_t ldb, rmm_bf16* Y, int64_t ldy, double rho, int32_t* idx_out, void* ws, size_t ws_bytes,
+                      rmm_stream stream);
+
+/* ---------------------------------------------------------------- attention scores
+ * rmm_qk: per query head h, I_h = TopK of the column norms of Q_h over its nq
+ * rows (head-feature dims), then S_h = scale * Q_h[:, I_h] . K_g(h)[:, I_h]^T
+ * with g(h) = h / (Hq / Hkv) under GQA ("Core Approach", component mapping:
+ * QK^T selects along the head feature dim with score = Q column norm; under GQA
+ * the selection is made on Q per head and K gathers the corresponding dims).
+ *   Q  device bf16 [batch][Hq][nq][dh], contiguous.
+ *   K  device bf16 [batch][Hkv][nk][dh], contiguous.
+ *   S  device fp32 [batch][Hq][nq][nk], contiguous.  With causal = 1, entries
+ *      with key j > i + (nk - nq) are -inf (bottom-right alignment).
+ *   idx_out device int32 [batch][Hq][k] or NULL, k = rmm_k(rho, dh).
+ * Requires Hq % Hkv == 0, dh % 8 == 0, nk % 4 == 0, dh <= 32768. */
+size_t rmm_qk_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh,
+                              double rho);
+rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch, int64_t hq, int64_t hkv, int64_t nq,
+                  int64_t nk, int64_t dh, int causal, float scale, double rho, int32_t* idx_out, void* ws,
+                  size_t ws_bytes, rmm_stream stream);
+
+/* ---------------------------------------------------------------- attention output
+ * rmm_pv: per head h, I_h = TopK over key positions of the column norms of P_h
+ * taken over all query rows, then O_h = P_h[:, I_h] . V_g(h)[I_h, :]
+ * ("Core Approach", component mapping: PV selects along token positions).
+ *   P  device bf16 [batch][H][nq][nk], contiguous (attention probabilities).
+ *   V  device bf16 [batch][Hkv][nk][dh], contiguous.
+ *   O  device bf16 [batch][H][nq][dh], contiguous.
+ *   causal = 1 treats P[i, j] with j > i + (nk - nq) as zero: those entries are
+ *   neither read for the scores nor multiplied.
+ *   idx_out device int32 [batch][H][k] or NULL, k = rmm_k(rho, nk).
+ * Requires H % Hkv == 0, nk % 8 == 0, dh == 64 or 128, nk <= 32768. */
+size_t rmm_pv_workspace_bytes(int64_t batch, int64_t h, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, double rho);
+rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t batch, int64_t h, int64_t hkv,
+                  int64_t nq, int64_t nk, int64_t dh, int causal, double rho, int32_t* idx_out, void* ws,
+                  size_t ws_bytes, rmm_stream stream);
+
+/* ---------------------------------------------------------------- diagnostics */
+const char* rmm_status_string(rmm_status s);
+/* Message of the most recent failure on the calling thread ("" if none). */
+const char* rmm_last_error(void);
+/* Reads and clears the device-side error word of the current device (0 = no
+ * kernel gave up on a wait).  Synchronises the device.  Returns RMM_ERR_CUDA if
+ * the read itself fails, else RMM_OK. */
+rmm_status rmm_device_error(int32_t* code_out);
+/* Library version, e.g. "rmm-b200 0.1". */
+const char* rmm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RMM_H_ */

@@ -1,0 +1,226 @@
+"""B200-native Reduced Matrix Multiplication (RMM).
+
+Thin ctypes binding over the C ABI of ``librmm.so`` (declared in
+``include/rmm.h``).  This module only marshals arguments -- every step of the
+path (column scores, TopK selection, pack, tensor-core product) runs in the
+library's sm_100a CUDA kernels.  PyTorch provides device memory and streams.
+
+Importing this package does not load the library; the first call does, and
+raises if ``librmm.so`` has not been built (there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["lib", "rmm_k", "select", "linear", "qk", "pv", "RMMError", "device_error", "library_path"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "librmm.so")
+
+
+class RMMError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+_c_i64 = ctypes.c_int64
+_c_p = ctypes.c_void_p
+_c_dbl = ctypes.c_double
+_c_int = ctypes.c_int
+_c_size = ctypes.c_size_t
+_c_float = ctypes.c_float
+
+_SIGNATURES = {
+    "rmm_k": (_c_i64, [_c_dbl, _c_i64]),
+    "rmm_select_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64]),
+    "rmm_select": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_dbl, _c_p, _c_p, _c_p, _c_p,
+                            _c_size, _c_p]),
+    "rmm_linear_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_linear": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_dbl, _c_p, _c_p,
+                            _c_size, _c_p]),
+    "rmm_qk_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_qk": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_float, _c_dbl,
+                        _c_p, _c_p, _c_size, _c_p]),
+    "rmm_pv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_pv": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_dbl, _c_p, _c_p,
+                        _c_size, _c_p]),
+    "rmm_status_string": (ctypes.c_char_p, [_c_int]),
+    "rmm_last_error": (ctypes.c_char_p, []),
+    "rmm_device_error": (_c_int, [ctypes.POINTER(ctypes.c_int32)]),
+    "rmm_version": (ctypes.c_char_p, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load librmm.so (once) and declare the C signatures."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is not built; run `python -m input_adaptive_reduced_colnorm_b200.build`")
+        L = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        L = lib()
+        raise RMMError(status, f"{L.rmm_status_string(status).decode()}: {L.rmm_last_error().decode()}")
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream(device):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require(t, name, dtype, dim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions")
+
+
+def _workspace(nbytes: int, device, workspace=None):
+    import torch
+    if nbytes == 0:
+        return None
+    if workspace is not None and workspace.numel() * workspace.element_size() >= nbytes:
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def rmm_k(rho: float, d: int) -> int:
+    """k = ceil(rho * d) as the library computes it (-1 for invalid arguments)."""
+    return int(lib().rmm_k(float(rho), int(d)))
+
+
+def select(A, rho: float, *, causal: bool = False, colsq: bool = True, retained: bool = True, workspace=None):
+    """Column scores and TopK index set of A ([n, d] or [batch, n, d], bf16, CUDA).
+
+    Returns (idx int32 [batch?, k], colsq float64 [batch?, d] or None, retained float64 [batch?] or None)."""
+    import torch
+    _require(A, "A", torch.bfloat16)
+    squeeze = A.dim() == 2
+    A3 = A.unsqueeze(0) if squeeze else A
+    if A3.dim() != 3 or A3.stride(2) != 1:
+        raise ValueError("A must be [n, d] or [batch, n, d] with unit column stride")
+    batch, n, d = A3.shape
+    lda = A3.stride(1)
+    bstride = A3.stride(0) if batch > 1 else n * lda
+    k = rmm_k(rho, d)
+    if k < 0:
+        raise RMMError(1, f"invalid rho {rho}")
+    dev = A.device
+    idx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+    cs = torch.empty((batch, d), dtype=torch.float64, device=dev) if colsq else None
+    rt = torch.empty((batch,), dtype=torch.float64, device=dev) if retained else None
+    L = lib()
+    ws = None if colsq else _workspace(L.rmm_select_workspace_bytes(batch, n, d), dev, workspace)
+    _check(L.rmm_select(_ptr(A3), batch, bstride, n, d, lda, int(causal), float(rho), _ptr(idx), _ptr(cs), _ptr(rt),
+                        _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    if squeeze:
+        idx = idx[0]
+        cs = None if cs is None else cs[0]
+        rt = None if rt is None else rt[0]
+    return idx, cs, rt
+
+
+def linear(A, B, rho: float, *, out=None, return_idx: bool = False, workspace=None):
+    """Y = A[:, I] . B[I, :] with I the TopK column-norm set of A.
+
+    A [n, d] bf16 (row stride may exceed d), B [d, m] bf16 (contraction index on
+    rows), both CUDA.  Returns Y [n, m] bf16 (and idx int32 [k] if asked)."""
+    import torch
+    _require(A, "A", torch.bfloat16, 2)
+    _require(B, "B", torch.bfloat16, 2)
+    if A.stride(1) != 1 or B.stride(1) != 1:
+        raise ValueError("A and B need unit column stride")
+    n, d = A.shape
+    d2, m = B.shape
+    if d2 != d:
+        raise ValueError(f"contraction mismatch: A has {d} columns, B has {d2} rows")
+    dev = A.device
+    if out is None:
+        out = torch.empty((n, m), dtype=torch.bfloat16, device=dev)
+    _require(out, "out", torch.bfloat16, 2)
+    k = rmm_k(rho, d)
+    idx = torch.empty((max(k, 0),), dtype=torch.int32, device=dev) if return_idx else None
+    L = lib()
+    ws = _workspace(L.rmm_linear_workspace_bytes(n, d, m, float(rho)), dev, workspace)
+    _check(L.rmm_linear(_ptr(A), n, d, A.stride(0), _ptr(B), m, B.stride(0), _ptr(out), out.stride(0), float(rho),
+                        _ptr(idx), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def qk(Q, K, rho: float, *, causal: bool = True, scale: float = 1.0, out=None, return_idx: bool = False,
+       workspace=None):
+    """Reduced attention scores.  Q [B, Hq, nq, dh], K [B, Hkv, nk, dh] bf16 contiguous
+    -> S [B, Hq, nq, nk] float32 (-inf where causally masked)."""
+    import torch
+    _require(Q, "Q", torch.bfloat16, 4)
+    _require(K, "K", torch.bfloat16, 4)
+    if not (Q.is_contiguous() and K.is_contiguous()):
+        raise ValueError("Q and K must be contiguous")
+    b, hq, nq, dh = Q.shape
+    b2, hkv, nk, dh2 = K.shape
+    if b2 != b or dh2 != dh:
+        raise ValueError("Q / K shape mismatch")
+    dev = Q.device
+    if out is None:
+        out = torch.empty((b, hq, nq, nk), dtype=torch.float32, device=dev)
+    k = rmm_k(rho, dh)
+    idx = torch.empty((b, hq, max(k, 0)), dtype=torch.int32, device=dev) if return_idx else None
+    L = lib()
+    ws = _workspace(L.rmm_qk_workspace_bytes(b, hq, hkv, nq, nk, dh, float(rho)), dev, workspace)
+    _check(L.rmm_qk(_ptr(Q), _ptr(K), _ptr(out), b, hq, hkv, nq, nk, dh, int(causal), float(scale), float(rho),
+                    _ptr(idx), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def pv(P, V, rho: float, *, causal: bool = True, out=None, return_idx: bool = False, workspace=None):
+    """Reduced attention output.  P [B, H, nq, nk], V [B, Hkv, nk, dh] bf16 contiguous
+    -> O [B, H, nq, dh] bf16."""
+    import torch
+    _require(P, "P", torch.bfloat16, 4)
+    _require(V, "V", torch.bfloat16, 4)
+    if not (P.is_contiguous() and V.is_contiguous()):
+        raise ValueError("P and V must be contiguous")
+    b, h, nq, nk = P.shape
+    b2, hkv, nk2, dh = V.shape
+    if b2 != b or nk2 != nk:
+        raise ValueError("P / V shape mismatch")
+    dev = P.device
+    if out is None:
+        out = torch.empty((b, h, nq, dh), dtype=torch.bfloat16, device=dev)
+    k = rmm_k(rho, nk)
+    idx = torch.empty((b, h, max(k, 0)), dtype=torch.int32, device=dev) if return_idx else None
+    L = lib()
+    ws = _workspace(L.rmm_pv_workspace_bytes(b, h, hkv, nq, nk, dh, float(rho)), dev, workspace)
+    _check(L.rmm_pv(_ptr(P), _ptr(V), _ptr(out), b, h, hkv, nq, nk, dh, int(causal), float(rho), _ptr(idx),
+                    _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def device_error() -> int:
+    """Read and clear the device-side error word (synchronises the device)."""
+    v = ctypes.c_int32(0)
+    _check(lib().rmm_device_error(ctypes.byref(v)))
+    return int(v.value)

@@ -1,0 +1,354 @@
+// Reduced product on the 5th-generation tensor cores:
+//   Y[M x N] = A_I[M x k] . B[I, :][k x N]      ("Algorithm Deep-Dive: RMM",
+//   Core Approach: RMM_rho(A, B) = A[:, I] B[I, :]; the reduced product is still
+//   a dense contraction over the k kept indices).
+//
+// Persistent, warp-specialised tcgen05 kernel, one CTA per SM:
+//   warp 0      TMA producer: A tile (K-major, 128 x 64 bf16, 128-byte swizzle)
+//               and B tile, either gathered row by row from B[I, :] with
+//               tile::gather4 (four kept rows per copy), loaded as a plain
+//               MN-major tile (rho = 1 path, I = [0, d)), or loaded as a K-major
+//               tile (per-head Q K^T where K is packed like Q).
+//   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma (M=128,
+//               N=BN, K=16 per instruction) into a double-buffered fp32
+//               accumulator in TMEM and commits to mbarriers.
+//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> bf16/fp32 -> global.
+// Every wait is bounded (about one second); on a timeout the CTA records an
+// error code, drains its own copies in flight, frees its TMEM and returns.
+// There is no cluster multicast anywhere: each CTA fetches its own tiles and
+// L2 absorbs the reuse between CTAs.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace rmm {
+
+enum BMode : int { kBGather = 0, kBTileMN = 1, kBTileK = 2 };
+enum EpiMode : int { kEpiBf16 = 0, kEpiF32 = 1 };
+enum CausalMode : int { kCausalNone = 0, kCausalMaskScores = 1, kCausalLimitK = 2 };
+
+struct GemmParams {
+  int M, N;              // rows / columns of one batch item's output
+  int k;                 // kept contraction length (true k, not padded)
+  int num_kb;            // ceil(k / 64)
+  int batch;
+  int m_tiles, n_tiles;
+  int a_rows_per_batch;  // A tensor-map row of (b, m) = b * a_rows_per_batch + m
+  // B tensor-map row of batch item b: b_row_base(b) + I_b[t] (gather), + t (MN
+  // tile) or + n (K-major tile), b_row_base(b) = (b / b_g_outer) * b_s_outer +
+  // ((b % b_g_outer) / b_g_inner) * b_s_inner
+  const int32_t* idx;    // [batch][k] ascending kept indices, or null for I = [0, k)
+  int64_t idx_bstride;
+  int b_g_outer, b_g_inner;
+  int64_t b_s_outer, b_s_inner;
+  int b_oob_row;         // a row index outside the B tensor (reads zeros)
+  // output
+  void* out;
+  int64_t ldo;           // elements between output rows
+  int64_t out_bstride;   // elements between batch items
+  float scale;
+  int64_t causal_off;    // key/position j is visible to row i iff j <= i + causal_off
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ int64_t gemm_b_row_base(const GemmParams& p, int b) {
+  return static_cast<int64_t>(b / p.b_g_outer) * p.b_s_outer +
+         static_cast<int64_t>((b % p.b_g_outer) / p.b_g_inner) * p.b_s_inner;
+}
+
+// Number of 64-wide k-blocks a tile needs.
+template <int BN, int CAUSAL>
+__device__ __forceinline__ int gemm_tile_kb(const GemmParams& p, int b, int m0, int n0) {
+  if (CAUSAL == kCausalMaskScores) {
+    // a tile whose first key lies beyond every row's horizon is fully masked
+    if (static_cast<int64_t>(n0) > static_cast<int64_t>(m0) + 127 + p.causal_off) return 0;
+    return p.num_kb;
+  } else if (CAUSAL == kCausalLimitK) {
+    // kept positions I[t] <= last row + off contribute; I is ascending
+    const int64_t hz = static_cast<int64_t>(m0) + 127 + p.causal_off;
+    if (p.idx == nullptr) {  // identity index set
+      const int64_t lim = hz + 1 < 0 ? 0 : (hz + 1 > p.k ? p.k : hz + 1);
+      return static_cast<int>((lim + 63) >> 6);
+    }
+    const int32_t* I = p.idx + static_cast<int64_t>(b) * p.idx_bstride;
+    int lo = 0, hi = p.k;  // first t with I[t] > hz
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (static_cast<int64_t>(__ldg(I + mid)) <= hz) lo = mid + 1;
+      else hi = mid;
+    }
+    return (lo + 63) >> 6;
+  }
+  return p.num_kb;
+}
+
+// Tile order: batch item, then N tile, then M tile fastest, so CTAs running at
+// the same time share B column blocks in L2.
+__device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& b, int& m0, int& nt) {
+  const int per_b = p.m_tiles * p.n_tiles;
+  b = tile / per_b;
+  const int r = tile - b * per_b;
+  nt = r / p.m_tiles;
+  m0 = (r - nt * p.m_tiles) * 128;
+}
+
+template <int BN, int BMODE, int EPI, int CAUSAL>
+__global__ void __launch_bounds__(192, 1)
+    rmm_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmParams p) {
+  using C = GemmCfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr uint32_t IDESC = make_idesc_bf16(128, BN, 0, (BMODE == kBTileK) ? 0 : 1);
+
+  extern __shared__ uint8_t gemm_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = p.batch * p.m_tiles * p.n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      int b, m0, nt;
+      gemm_tile_coords(p, tile, b, m0, nt);
+      const int n0 = nt * BN;
+      const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, n0);
+      const int a_row = b * p.a_rows_per_batch + m0;
+      const int32_t* I = p.idx + static_cast<int64_t>(b) * p.idx_bstride;
+      const int64_t brow0 = gemm_b_row_base(p, b);
+      for (int kb = 0; kb < nkb; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
+          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * 64, a_row);
+        }
+        __syncwarp();
+        uint8_t* dstB = sB + stage * C::B_BYTES;
+        if (BMODE == kBGather) {
+          // 16 groups of 4 kept rows x (BN / 64) column chunks of 64
+          constexpr int OPS = 16 * (BN / 64);
+          for (int op = lane; op < OPS; op += 32) {
+            const int g = op & 15, c = op >> 4;
+            int32_t r[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int t = kb * 64 + g * 4 + q;
+              r[q] = (t < p.k) ? static_cast<int32_t>(brow0 + __ldg(I + t)) : p.b_oob_row;
+            }
+            tma_gather4(dstB + c * 8192 + g * 512, &tmB, &full[stage], n0 + c * 64, r[0], r[1], r[2], r[3]);
+          }
+        } else if (BMODE == kBTileMN) {
+          if (lane < BN / 64)
+            tma_load_2d(dstB + lane * 8192, &tmB, &full[stage], n0 + lane * 64, static_cast<int32_t>(brow0 + kb * 64));
+        } else {
+          if (lane == 0) tma_load_2d(dstB, &tmB, &full[stage], kb * 64, static_cast<int32_t>(brow0 + n0));
+        }
+        __syncwarp();
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // drain: wait for the copies this CTA issued so no TMA writes land after exit
+      for (int s = 0; s < STAGES; ++s) {
+        const uint32_t uses = (issued + STAGES - 1 - s) / STAGES;  // loads issued into stage s
+        if (uses == 0) continue;
+        const uint32_t par = (uses - 1) & 1u;
+        const uint32_t a = smem_u32(&full[s]);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(a, par) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc_i = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        int b, m0, nt;
+        gemm_tile_coords(p, tile, b, m0, nt);
+        const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, nt * BN);
+        if (nkb == 0) continue;
+        const int acc = acc_i & 1;
+        const uint32_t acc_par = (acc_i >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, kDevErrTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sw128_desc(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = (BMODE == kBTileK) ? make_sw128_desc(b0 + kk * 32, 16, 1024)
+                                                   : make_sw128_desc(b0 + kk * 2048, 8192, 1024);
+            umma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        ++acc_i;
+      }
+      // all MMAs issued by this thread are complete once `drain` flips
+      umma_commit(drain);
+      const uint32_t a = smem_u32(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = quarter * 32 + lane;
+    int acc_i = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int b, m0, nt;
+      gemm_tile_coords(p, tile, b, m0, nt);
+      const int n0 = nt * BN;
+      const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, n0);
+      const int row = m0 + row_in_tile;
+      const bool row_ok = row < p.M;
+      if (nkb > 0) {
+        const int acc = acc_i & 1;
+        const uint32_t acc_par = (acc_i >> 1) & 1;
+        if (!mbar_wait(&tfull[acc], acc_par, abort_flag, kDevErrTimeoutEpilogue)) break;
+        tc_fence_after();
+      }
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        if (nkb > 0) {
+          uint32_t r[32];
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>((acc_i & 1) * BN + c * 32), r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+        }
+        if (!row_ok) continue;
+        const int col0 = n0 + c * 32;
+        if (col0 >= p.N) continue;
+        if (EPI == kEpiF32) {
+          float* o = reinterpret_cast<float*>(p.out) + static_cast<int64_t>(b) * p.out_bstride +
+                     static_cast<int64_t>(row) * p.ldo + col0;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float x = v[e] * p.scale;
+            if (CAUSAL == kCausalMaskScores && static_cast<int64_t>(col0 + e) > static_cast<int64_t>(row) + p.causal_off)
+              x = -__int_as_float(0x7f800000);
+            v[e] = x;
+          }
+          if (col0 + 32 <= p.N) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          } else {
+            for (int e = 0; col0 + e < p.N; ++e) o[e] = v[e];
+          }
+        } else {
+          uint16_t* o = reinterpret_cast<uint16_t*>(p.out) + static_cast<int64_t>(b) * p.out_bstride +
+                        static_cast<int64_t>(row) * p.ldo + col0;
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            h[e] = *reinterpret_cast<const uint32_t*>(&t);
+          }
+          if (col0 + 32 <= p.N) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<uint4*>(o + 2 * e) = make_uint4(h[e], h[e + 1], h[e + 2], h[e + 3]);
+          } else {
+            for (int e = 0; col0 + e < p.N; ++e) o[e] = static_cast<uint16_t>(h[e >> 1] >> (16 * (e & 1)));
+          }
+        }
+      }
+      if (nkb > 0) {
+        tc_fence_before();
+        mbar_arrive(&tempty[acc_i & 1]);
+        ++acc_i;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace rmm

@@ -1,0 +1,619 @@
+// C ABI of the RMM library: argument checks, workspace layout, tensor maps and
+// the launch sequence of each entry point.  See include/rmm.h for the contract.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "rmm.h"
+#include "ptx.cuh"
+#include "colsq.cuh"
+#include "select.cuh"
+#include "pack.cuh"
+#include "gemm.cuh"
+
+using namespace rmm;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+rmm_status fail(rmm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+rmm_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(RMM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+inline int64_t ceil_div(int64_t x, int64_t m) { return (x + m - 1) / m; }
+
+constexpr int64_t kMaxSelectD = 32768;
+constexpr int64_t kIntMax = 2147483647LL;
+
+// ---------------------------------------------------------------- device facts
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 or fp32 tensor map with 128-byte swizzle; OOB elements read as 0.
+rmm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(RMM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RMM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return RMM_OK;
+}
+
+// ---------------------------------------------------------------- workspace carving
+struct Carver {
+  uint8_t* base;
+  size_t cur = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(int64_t count) {
+    cur = (cur + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + cur) : nullptr;
+    cur += static_cast<size_t>(count) * sizeof(T);
+    return p;
+  }
+  size_t bytes() const { return (cur + 255) & ~size_t(255); }
+};
+
+// ---------------------------------------------------------------- launches
+rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64_t n, int64_t d, int64_t lda,
+                        bool causal, int64_t off, double* colsq, cudaStream_t s) {
+  int C = 1;
+  while (C < 8 && n / (2 * C) >= 128) C *= 2;
+  const int64_t target = 2LL * num_sms();
+  int TX = 32;
+  while (TX > 4 && ceil_div(d, TX * 8) * batch * C < target) TX /= 2;
+  const int64_t strips = ceil_div(d, TX * 8);
+  if (strips * C > kIntMax || batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "column-norm grid too large");
+  ColsqParams p{};
+  p.A = A;
+  p.batch_stride = bstride;
+  p.n = n;
+  p.d = d;
+  p.lda = lda;
+  p.causal_off = off;
+  p.colsq = colsq;
+  p.rows_per_cta = ceil_div(n, C);
+  p.csize = C;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(strips * C), static_cast<unsigned>(batch), 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
+#define RMM_COLSQ_CASE(tx)                                                          \
+  case tx:                                                                          \
+    e = causal ? cudaLaunchKernelEx(&cfg, colsq_kernel<tx, true>, p)               \
+               : cudaLaunchKernelEx(&cfg, colsq_kernel<tx, false>, p);             \
+    break;
+  switch (TX) {
+    RMM_COLSQ_CASE(32)
+    RMM_COLSQ_CASE(16)
+    RMM_COLSQ_CASE(8)
+    RMM_COLSQ_CASE(4)
+  }
+#undef RMM_COLSQ_CASE
+  if (e != cudaSuccess) return cuda_fail(e, "column-norm launch");
+  return RMM_OK;
+}
+
+rmm_status launch_select(const double* colsq, int64_t batch, int64_t d, int64_t k, int32_t* idx, double* retained,
+                         cudaStream_t s) {
+  SelectParams p{colsq, d, k, idx, retained};
+  const unsigned g = static_cast<unsigned>(batch);
+  if (d <= 128) select_kernel<1, 128><<<g, 128, 0, s>>>(p);
+  else if (d <= 1024) select_kernel<1, 1024><<<g, 1024, 0, s>>>(p);
+  else if (d <= 2048) select_kernel<2, 1024><<<g, 1024, 0, s>>>(p);
+  else if (d <= 4096) select_kernel<4, 1024><<<g, 1024, 0, s>>>(p);
+  else if (d <= 8192) select_kernel<8, 1024><<<g, 1024, 0, s>>>(p);
+  else if (d <= 16384) select_kernel<16, 1024><<<g, 1024, 0, s>>>(p);
+  else select_kernel<32, 1024><<<g, 1024, 0, s>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  return RMM_OK;
+}
+
+rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
+  const int64_t rows = p.batch * p.rows;
+  const int64_t d_round = round_up(p.d, 8);
+  const int64_t cap = 8LL * num_sms();
+  cudaError_t e;
+  if (p.d <= 1024) {
+    const size_t smem = static_cast<size_t>(8 * d_round * 2);
+    const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), cap);
+    pack_rows_warp_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round);
+  } else {
+    const size_t smem = static_cast<size_t>(d_round * 2);
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(pack_rows_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+      if (e != cudaSuccess) return cuda_fail(e, "pack attribute");
+    }
+    const int64_t grid = std::min<int64_t>(rows, cap);
+    pack_rows_cta_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return RMM_OK;
+}
+
+template <int BN, int BMODE, int EPI, int CAUSAL>
+rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t s) {
+  auto kern = rmm_gemm_kernel<BN, BMODE, EPI, CAUSAL>;
+  constexpr int smem = GemmCfg<BN>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm attribute");
+  const int64_t tiles = static_cast<int64_t>(p.batch) * p.m_tiles * p.n_tiles;
+  if (tiles > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many output tiles");
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  kern<<<grid, 192, smem, s>>>(ta, tb, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return RMM_OK;
+}
+
+GemmParams gemm_defaults() {
+  GemmParams p{};
+  p.batch = 1;
+  p.b_g_outer = 1;
+  p.b_g_inner = 1;
+  p.b_s_outer = 0;
+  p.b_s_inner = 0;
+  p.scale = 1.f;
+  return p;
+}
+
+rmm_status check_rho(double rho) {
+  if (!(rho > 0.0 && rho <= 1.0)) return fail(RMM_ERR_INVALID_ARG, "rho must lie in (0, 1], got %g", rho);
+  return RMM_OK;
+}
+
+}  // namespace
+
+// ============================================================== public API
+extern "C" {
+
+int64_t rmm_k(double rho, int64_t d) {
+  if (!(rho > 0.0 && rho <= 1.0) || d < 1) return -1;
+  const double x = rho * static_cast<double>(d);
+  int64_t k = static_cast<int64_t>(std::ceil(x - 1e-9 * x));
+  if (k < 1) k = 1;
+  if (k > d) k = d;
+  return k;
+}
+
+const char* rmm_status_string(rmm_status s) {
+  switch (s) {
+    case RMM_OK: return "ok";
+    case RMM_ERR_INVALID_ARG: return "invalid argument";
+    case RMM_ERR_UNSUPPORTED: return "unsupported layout or size";
+    case RMM_ERR_WORKSPACE: return "workspace too small";
+    case RMM_ERR_CUDA: return "CUDA error";
+    case RMM_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* rmm_last_error(void) { return t_last_error.c_str(); }
+
+const char* rmm_version(void) { return "rmm-b200 0.1"; }
+
+rmm_status rmm_device_error(int32_t* code_out) {
+  if (code_out == nullptr) return fail(RMM_ERR_INVALID_ARG, "code_out is null");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "device synchronise");
+  int32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  const int32_t zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+  *code_out = v;
+  return RMM_OK;
+}
+
+// ---------------------------------------------------------------- select
+size_t rmm_select_workspace_bytes(int64_t batch, int64_t n, int64_t d) {
+  (void)n;
+  if (batch < 1 || d < 1) return 0;
+  Carver c(nullptr);
+  c.take<double>(batch * d);
+  return c.bytes();
+}
+
+rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, int64_t n, int64_t d, int64_t lda,
+                      int causal, double rho, int32_t* idx_out, double* colsq_out, double* retained_out, void* ws,
+                      size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (A == nullptr || idx_out == nullptr) return fail(RMM_ERR_INVALID_ARG, "A and idx_out are required");
+  if (batch < 1 || n < 1 || d < 1) return fail(RMM_ERR_INVALID_ARG, "batch, n and d must be >= 1");
+  if (lda < d) return fail(RMM_ERR_INVALID_ARG, "lda < d");
+  if (batch > 1 && batch_stride < (n - 1) * lda + d) return fail(RMM_ERR_INVALID_ARG, "batch_stride too small");
+  if (causal != 0 && causal != 1) return fail(RMM_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (d > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "d > %lld", static_cast<long long>(kMaxSelectD));
+  if (n > kIntMax || batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "n or batch too large");
+  if (!aligned16(A) || (lda % 8) != 0 || (batch > 1 && (batch_stride % 8) != 0))
+    return fail(RMM_ERR_UNSUPPORTED, "A must be 16-byte aligned with lda and batch_stride multiples of 8");
+  const int64_t k = rmm_k(rho, d);
+  double* colsq = colsq_out;
+  if (colsq == nullptr) {
+    const size_t need = rmm_select_workspace_bytes(batch, n, d);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    Carver c(ws);
+    colsq = c.take<double>(batch * d);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t off = d - n;
+  if (rmm_status st = launch_colsq(A, batch, batch_stride, n, d, lda, causal != 0, off, colsq, s)) return st;
+  return launch_select(colsq, batch, d, k, idx_out, retained_out, s);
+}
+
+// ---------------------------------------------------------------- linear
+size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
+  (void)m;
+  const int64_t k = rmm_k(rho, d);
+  if (k < 0 || n < 1) return 0;
+  if (k == d) return 0;
+  Carver c(nullptr);
+  c.take<double>(d);
+  c.take<int32_t>(k);
+  c.take<uint16_t>(n * round_up(k, 8));
+  return c.bytes();
+}
+
+rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const rmm_bf16* B, int64_t m,
+                      int64_t ldb, rmm_bf16* Y, int64_t ldy, double rho, int32_t* idx_out, void* ws, size_t ws_bytes,
+                      rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (A == nullptr || B == nullptr || Y == nullptr) return fail(RMM_ERR_INVALID_ARG, "A, B and Y are required");
+  if (n < 1 || d < 1 || m < 1) return fail(RMM_ERR_INVALID_ARG, "n, d and m must be >= 1");
+  if (lda < d || ldb < m || ldy < m) return fail(RMM_ERR_INVALID_ARG, "leading dimension too small");
+  if (!aligned16(A) || !aligned16(B) || !aligned16(Y) || (lda % 8) || (ldb % 8) || (ldy % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
+  if (n > kIntMax - 128 || m > kIntMax - 256 || d > kIntMax - 64)
+    return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  const int64_t k = rmm_k(rho, d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemmParams g = gemm_defaults();
+  g.M = static_cast<int>(n);
+  g.N = static_cast<int>(m);
+  g.out = Y;
+  g.ldo = ldy;
+  g.m_tiles = static_cast<int>(ceil_div(n, 128));
+  g.n_tiles = static_cast<int>(ceil_div(m, 256));
+  CUtensorMap ta, tb;
+  if (k == d) {
+    // rho = 1: the dense product, I = [0, d)
+    if (rmm_status st = make_tmap(&ta, A, d, n, lda * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, B, m, d, ldb * 2, 64, 64)) return st;
+    g.k = static_cast<int>(d);
+    g.num_kb = static_cast<int>(ceil_div(d, 64));
+    if (idx_out != nullptr) {
+      iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024)), 256, 0, s>>>(idx_out, 1, d);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+    }
+    return launch_gemm<256, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  }
+  if (d > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "d > %lld", static_cast<long long>(kMaxSelectD));
+  const size_t need = rmm_linear_workspace_bytes(n, d, m, rho);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  const int64_t k_pad = round_up(k, 8);
+  Carver c(ws);
+  double* colsq = c.take<double>(d);
+  int32_t* idx_ws = c.take<int32_t>(k);
+  uint16_t* apack = c.take<uint16_t>(n * k_pad);
+  int32_t* idx = idx_out ? idx_out : idx_ws;
+
+  if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
+  if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
+  PackParams pk{};
+  pk.src = A;
+  pk.src_ld = lda;
+  pk.rows = n;
+  pk.d = d;
+  pk.g_outer = 1;
+  pk.g_inner = 1;
+  pk.idx = idx;
+  pk.k = k;
+  pk.k_pad = k_pad;
+  pk.dst = apack;
+  pk.batch = 1;
+  if (rmm_status st = launch_pack(pk, s)) return st;
+  if (rmm_status st = make_tmap(&ta, apack, k_pad, n, k_pad * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tb, B, m, d, ldb * 2, 64, 1)) return st;
+  g.k = static_cast<int>(k);
+  g.num_kb = static_cast<int>(ceil_div(k, 64));
+  g.idx = idx;
+  g.b_oob_row = static_cast<int>(d);
+  return launch_gemm<256, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+}
+
+// ---------------------------------------------------------------- QK^T
+size_t rmm_qk_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh,
+                              double rho) {
+  (void)hkv;
+  const int64_t k = rmm_k(rho, dh);
+  if (k < 0 || batch < 1 || hq < 1 || nq < 1 || nk < 1) return 0;
+  if (k == dh) return 0;
+  const int64_t items = batch * hq;
+  const int64_t k_pad = round_up(k, 8);
+  Carver c(nullptr);
+  c.take<double>(items * dh);
+  c.take<int32_t>(items * k);
+  c.take<uint16_t>(items * nq * k_pad);
+  c.take<uint16_t>(items * nk * k_pad);
+  return c.bytes();
+}
+
+rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch, int64_t hq, int64_t hkv, int64_t nq,
+                  int64_t nk, int64_t dh, int causal, float scale, double rho, int32_t* idx_out, void* ws,
+                  size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (Q == nullptr || K == nullptr || S == nullptr) return fail(RMM_ERR_INVALID_ARG, "Q, K and S are required");
+  if (batch < 1 || hq < 1 || hkv < 1 || nq < 1 || nk < 1 || dh < 1)
+    return fail(RMM_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (hq % hkv) return fail(RMM_ERR_INVALID_ARG, "Hq (%lld) must be a multiple of Hkv (%lld)",
+                            static_cast<long long>(hq), static_cast<long long>(hkv));
+  if (causal != 0 && causal != 1) return fail(RMM_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (!std::isfinite(scale)) return fail(RMM_ERR_INVALID_ARG, "scale must be finite");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(S) || (dh % 8) || (nk % 4))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned, dh % 8 == 0 and nk % 4 == 0");
+  if (dh > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "dh too large");
+  const int64_t items = batch * hq;
+  if (items > 65535 || items * nq > kIntMax - 128 || batch * hkv * nk > kIntMax - 256 || items * nk > kIntMax - 256)
+    return fail(RMM_ERR_UNSUPPORTED, "problem too large");
+  const int64_t k = rmm_k(rho, dh);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemmParams g = gemm_defaults();
+  g.M = static_cast<int>(nq);
+  g.N = static_cast<int>(nk);
+  g.batch = static_cast<int>(items);
+  g.m_tiles = static_cast<int>(ceil_div(nq, 128));
+  g.n_tiles = static_cast<int>(ceil_div(nk, 256));
+  g.a_rows_per_batch = static_cast<int>(nq);
+  g.out = S;
+  g.ldo = nk;
+  g.out_bstride = nq * nk;
+  g.scale = scale;
+  g.causal_off = nk - nq;
+  CUtensorMap ta, tb;
+  if (k == dh) {
+    if (rmm_status st = make_tmap(&ta, Q, dh, items * nq, dh * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, K, dh, batch * hkv * nk, dh * 2, 64, 256)) return st;
+    g.k = static_cast<int>(dh);
+    g.num_kb = static_cast<int>(ceil_div(dh, 64));
+    g.b_g_outer = static_cast<int>(hq);
+    g.b_g_inner = static_cast<int>(hq / hkv);
+    g.b_s_outer = hkv * nk;
+    g.b_s_inner = nk;
+    if (idx_out != nullptr) {
+      iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(items * dh, 256), 1024)), 256, 0, s>>>(
+          idx_out, items, dh);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+    }
+  } else {
+    const size_t need = rmm_qk_workspace_bytes(batch, hq, hkv, nq, nk, dh, rho);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    const int64_t k_pad = round_up(k, 8);
+    Carver c(ws);
+    double* colsq = c.take<double>(items * dh);
+    int32_t* idx_ws = c.take<int32_t>(items * k);
+    uint16_t* qpack = c.take<uint16_t>(items * nq * k_pad);
+    uint16_t* kpack = c.take<uint16_t>(items * nk * k_pad);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(Q, items, nq * dh, nq, dh, dh, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s)) return st;
+    PackParams pq{};
+    pq.src = Q;
+    pq.src_ld = dh;
+    pq.rows = nq;
+    pq.d = dh;
+    pq.g_outer = 1;
+    pq.g_inner = 1;
+    pq.s_outer = nq * dh;
+    pq.s_inner = 0;
+    pq.idx = idx;
+    pq.k = k;
+    pq.k_pad = k_pad;
+    pq.dst = qpack;
+    pq.batch = items;
+    if (rmm_status st = launch_pack(pq, s)) return st;
+    PackParams pkk = pq;
+    pkk.src = K;
+    pkk.rows = nk;
+    pkk.g_outer = hq;
+    pkk.g_inner = hq / hkv;
+    pkk.s_outer = hkv * nk * dh;
+    pkk.s_inner = nk * dh;
+    pkk.dst = kpack;
+    if (rmm_status st = launch_pack(pkk, s)) return st;
+    if (rmm_status st = make_tmap(&ta, qpack, k_pad, items * nq, k_pad * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, kpack, k_pad, items * nk, k_pad * 2, 64, 256)) return st;
+    g.k = static_cast<int>(k);
+    g.num_kb = static_cast<int>(ceil_div(k, 64));
+    g.b_g_outer = 1;
+    g.b_g_inner = 1;
+    g.b_s_outer = nk;
+  }
+  if (causal) return launch_gemm<256, kBTileK, kEpiF32, kCausalMaskScores>(ta, tb, g, s);
+  return launch_gemm<256, kBTileK, kEpiF32, kCausalNone>(ta, tb, g, s);
+}
+
+// ---------------------------------------------------------------- PV
+size_t rmm_pv_workspace_bytes(int64_t batch, int64_t h, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, double rho) {
+  (void)hkv;
+  (void)dh;
+  const int64_t k = rmm_k(rho, nk);
+  if (k < 0 || batch < 1 || h < 1 || nq < 1) return 0;
+  if (k == nk) return 0;
+  const int64_t items = batch * h;
+  Carver c(nullptr);
+  c.take<double>(items * nk);
+  c.take<int32_t>(items * k);
+  c.take<uint16_t>(items * nq * round_up(k, 8));
+  return c.bytes();
+}
+
+rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t batch, int64_t h, int64_t hkv,
+                  int64_t nq, int64_t nk, int64_t dh, int causal, double rho, int32_t* idx_out, void* ws,
+                  size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (P == nullptr || V == nullptr || O == nullptr) return fail(RMM_ERR_INVALID_ARG, "P, V and O are required");
+  if (batch < 1 || h < 1 || hkv < 1 || nq < 1 || nk < 1 || dh < 1)
+    return fail(RMM_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (h % hkv) return fail(RMM_ERR_INVALID_ARG, "H must be a multiple of Hkv");
+  if (causal != 0 && causal != 1) return fail(RMM_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (!aligned16(P) || !aligned16(V) || !aligned16(O) || (nk % 8) || (dh != 64 && dh != 128))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned, nk % 8 == 0 and dh in {64, 128}");
+  if (nk > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "nk > %lld", static_cast<long long>(kMaxSelectD));
+  const int64_t items = batch * h;
+  if (items > 65535 || items * nq > kIntMax - 128 || batch * hkv * nk > kIntMax - 64)
+    return fail(RMM_ERR_UNSUPPORTED, "problem too large");
+  const int64_t k = rmm_k(rho, nk);
+  const int64_t off = nk - nq;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemmParams g = gemm_defaults();
+  g.M = static_cast<int>(nq);
+  g.N = static_cast<int>(dh);
+  g.batch = static_cast<int>(items);
+  g.m_tiles = static_cast<int>(ceil_div(nq, 128));
+  g.n_tiles = 1;
+  g.a_rows_per_batch = static_cast<int>(nq);
+  g.out = O;
+  g.ldo = dh;
+  g.out_bstride = nq * dh;
+  g.causal_off = off;
+  g.b_g_outer = static_cast<int>(h);
+  g.b_g_inner = static_cast<int>(h / hkv);
+  g.b_s_outer = hkv * nk;
+  g.b_s_inner = nk;
+  g.b_oob_row = static_cast<int>(batch * hkv * nk);
+  CUtensorMap ta, tb;
+  const bool dense = (k == nk);
+  if (dense) {
+    if (rmm_status st = make_tmap(&ta, P, nk, items * nq, nk * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, V, dh, batch * hkv * nk, dh * 2, 64, 64)) return st;
+    g.k = static_cast<int>(nk);
+    g.num_kb = static_cast<int>(ceil_div(nk, 64));
+    g.idx = nullptr;
+    if (idx_out != nullptr) {
+      iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(items * nk, 256), 4096)), 256, 0, s>>>(
+          idx_out, items, nk);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+    }
+  } else {
+    const size_t need = rmm_pv_workspace_bytes(batch, h, hkv, nq, nk, dh, rho);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    const int64_t k_pad = round_up(k, 8);
+    Carver c(ws);
+    double* colsq = c.take<double>(items * nk);
+    int32_t* idx_ws = c.take<int32_t>(items * k);
+    uint16_t* ppack = c.take<uint16_t>(items * nq * k_pad);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(P, items, nq * nk, nq, nk, nk, causal != 0, off, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, items, nk, k, idx, nullptr, s)) return st;
+    PackParams pp{};
+    pp.src = P;
+    pp.src_ld = nk;
+    pp.rows = nq;
+    pp.d = nk;
+    pp.g_outer = 1;
+    pp.g_inner = 1;
+    pp.s_outer = nq * nk;
+    pp.idx = idx;
+    pp.k = k;
+    pp.k_pad = k_pad;
+    pp.dst = ppack;
+    pp.batch = items;
+    pp.causal = causal;
+    pp.causal_off = off;
+    if (rmm_status st = launch_pack(pp, s)) return st;
+    if (rmm_status st = make_tmap(&ta, ppack, k_pad, items * nq, k_pad * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, V, dh, batch * hkv * nk, dh * 2, 64, 1)) return st;
+    g.k = static_cast<int>(k);
+    g.num_kb = static_cast<int>(ceil_div(k, 64));
+    g.idx = idx;
+    g.idx_bstride = k;
+  }
+  if (dh == 128) {
+    if (dense)
+      return causal ? launch_gemm<128, kBTileMN, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
+                    : launch_gemm<128, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
+    return causal ? launch_gemm<128, kBGather, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
+                  : launch_gemm<128, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  }
+  if (dense)
+    return causal ? launch_gemm<64, kBTileMN, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
+                  : launch_gemm<64, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  return causal ? launch_gemm<64, kBGather, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
+                : launch_gemm<64, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load and export every function include/rmm.h declares, agree
+with the hand-derived k table, and reject bad arguments with the documented
+status before touching the device (on a machine without a GPU any device call
+would surface as RMM_ERR_CUDA instead, so the exact codes below also show that
+nothing was enqueued).
+"""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+import input_adaptive_reduced_colnorm_b200 as rmm
+from input_adaptive_reduced_colnorm_b200 import build as rmm_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rmm.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA_ERR, TIMEOUT = range(6)
+P16 = 0x10000  # a 16-byte aligned fake device address (never dereferenced)
+P_MIS = 0x10002
+
+
+@pytest.fixture(scope="module")
+def L():
+    rmm_build.build()
+    return rmm.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rmm_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"rmm_select", "rmm_linear", "rmm_qk", "rmm_pv", "rmm_k"} <= set(names)
+    for name in names:
+        assert hasattr(L, name), name
+    assert L.rmm_version().startswith(b"rmm-b200")
+
+
+def test_k_table_matches_hand_fixture(L):
+    with open(os.path.join(ROOT, "tests", "golden", "retention_count.json")) as f:
+        fx = json.load(f)
+    for rho, d, k in fx["cases"]:
+        assert L.rmm_k(rho, d) == k, (rho, d)
+    for rho, d in fx["invalid"]:
+        assert L.rmm_k(float(rho), d) == -1
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.rmm_status_string(s)
+    assert L.rmm_last_error() is not None
+
+
+def lin(L, A=P16, n=64, d=128, lda=128, B=P16, m=64, ldb=64, Y=P16, ldy=64, rho=0.5, idx=None, ws=None, wsb=0):
+    return L.rmm_linear(A, n, d, lda, B, m, ldb, Y, ldy, rho, idx, ws, wsb, None)
+
+
+@pytest.mark.parametrize("rho", [0.0, -0.5, 1.0000001, float("nan"), float("inf")])
+def test_linear_rejects_bad_rho(L, rho):
+    assert lin(L, rho=rho) == INVALID
+    assert b"rho" in L.rmm_last_error()
+
+
+def test_linear_argument_errors(L):
+    assert lin(L, A=None) == INVALID
+    assert lin(L, Y=None) == INVALID
+    assert lin(L, n=0) == INVALID
+    assert lin(L, lda=64) == INVALID          # lda < d
+    assert lin(L, ldb=32) == INVALID          # ldb < m
+    assert lin(L, A=P_MIS) == UNSUPPORTED     # misaligned pointer
+    assert lin(L, lda=132) == UNSUPPORTED     # leading dim not a multiple of 8
+    need = L.rmm_linear_workspace_bytes(64, 128, 64, 0.5)
+    assert need > 0
+    assert lin(L, ws=None, wsb=0) == WORKSPACE
+    assert lin(L, ws=P16, wsb=need - 1) == WORKSPACE
+    assert b"workspace" in L.rmm_last_error()
+
+
+def test_select_argument_errors(L):
+    def sel(A=P16, batch=1, bs=0, n=16, d=64, lda=64, causal=0, rho=0.5, idx=P16, cs=None, rt=None, ws=None, wsb=0):
+        return L.rmm_select(A, batch, bs, n, d, lda, causal, rho, idx, cs, rt, ws, wsb, None)
+    assert sel(idx=None) == INVALID
+    assert sel(rho=2.0) == INVALID
+    assert sel(causal=2) == INVALID
+    assert sel(batch=2, bs=8) == INVALID           # batch items overlap
+    assert sel(d=40000, lda=40000) == UNSUPPORTED  # beyond the documented d limit
+    assert sel(lda=68) == UNSUPPORTED
+    assert sel(ws=None) == WORKSPACE               # no colsq_out and no workspace
+
+
+def test_qk_pv_argument_errors(L):
+    def qk(Q=P16, K=P16, S=P16, b=1, hq=4, hkv=2, nq=64, nk=64, dh=128, causal=1, scale=1.0, rho=0.5, ws=None,
+           wsb=0):
+        return L.rmm_qk(Q, K, S, b, hq, hkv, nq, nk, dh, causal, scale, rho, None, ws, wsb, None)
+    assert qk(hkv=3) == INVALID          # Hq % Hkv != 0
+    assert qk(scale=float("nan")) == INVALID
+    assert qk(dh=100) == UNSUPPORTED
+    assert qk(nk=66) == UNSUPPORTED
+    assert qk() == WORKSPACE
+
+    def pv(P=P16, V=P16, O=P16, b=1, h=4, hkv=4, nq=64, nk=64, dh=128, causal=1, rho=0.5, ws=None, wsb=0):
+        return L.rmm_pv(P, V, O, b, h, hkv, nq, nk, dh, causal, rho, None, ws, wsb, None)
+    assert pv(hkv=3) == INVALID
+    assert pv(O=None) == INVALID
+    assert pv(dh=96) == UNSUPPORTED
+    assert pv(nk=60) == UNSUPPORTED
+    assert pv() == WORKSPACE
+
+
+def test_workspace_queries(L):
+    assert L.rmm_linear_workspace_bytes(4096, 4096, 4096, 1.0) == 0
+    a = L.rmm_linear_workspace_bytes(4096, 4096, 4096, 0.5)
+    b = L.rmm_linear_workspace_bytes(4096, 4096, 4096, 0.9)
+    assert 0 < a < b
+    assert a >= 4096 * 2048 * 2
+    assert L.rmm_qk_workspace_bytes(1, 32, 8, 4096, 4096, 128, 1.0) == 0
+    assert L.rmm_qk_workspace_bytes(1, 32, 8, 4096, 4096, 128, 0.5) >= 2 * 32 * 4096 * 64 * 2
+    assert L.rmm_pv_workspace_bytes(1, 32, 32, 1024, 1024, 128, 0.5) >= 32 * 1024 * 512 * 2
+    assert L.rmm_select_workspace_bytes(3, 10, 100) >= 3 * 100 * 8
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    A = torch.zeros((4, 16), dtype=torch.bfloat16)
+    B = torch.zeros((16, 8), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        rmm.linear(A, B, 0.5)

@@ -1,0 +1,114 @@
+"""GPU parity of rmm_linear (column norms -> TopK -> pack -> tcgen05 gathered GEMM)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from parity import check_close, check_index_set
+
+pytestmark = pytest.mark.gpu
+
+rmm = pytest.importorskip("input_adaptive_reduced_colnorm_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from input_adaptive_reduced_colnorm_b200 import build
+    build.build()
+    yield
+    assert rmm.device_error() == 0
+
+
+def parity_linear(A, B, rho, rows=None):
+    """Run the CUDA path and compare with the oracle (all rows, or sampled ``rows``)."""
+    Ad, Bd = A.cuda(), B.cuda()
+    Y, idx = rmm.linear(Ad, Bd, rho, return_idx=True)
+    torch.cuda.synchronize()
+    Aw, Bw = synthetic.widen(A), synthetic.widen(B)
+    q = oracle.column_sq_norms(Aw)
+    k = oracle.retention_count(rho, A.shape[1])
+    I = idx.cpu().numpy().astype(np.int64)
+    ties = check_index_set(I, q, k)
+    if rows is None:
+        ref = oracle.reduced_product(Aw, Bw, I)
+        got = synthetic.widen(Y.cpu())
+    else:
+        ref = oracle.rmm_linear_rows(Aw, Bw, I, rows)
+        got = synthetic.widen(Y[torch.as_tensor(rows, device=Y.device)].cpu())
+    check_close(got, ref, f"linear n={A.shape[0]} d={A.shape[1]} m={B.shape[1]} rho={rho}")
+    return Y, idx, ties
+
+
+def test_linear_single_layer_128x1024():
+    A, B = synthetic.linear_small()
+    Y, idx, _ = parity_linear(A, B, 0.5)
+    assert idx.numel() == 512
+    # independent second reference: cuBLAS on the GPU's own index set
+    I = idx.long()
+    Ad, Bd = A.cuda(), B.cuda()
+    ref = (Ad[:, I].float() @ Bd[I, :].float())
+    err = (Y.float() - ref).norm() / ref.norm()
+    assert err.item() < 1e-2
+    # bitwise determinism
+    Y2, idx2 = rmm.linear(Ad, Bd, 0.5, return_idx=True)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(Y, Y2)
+
+
+SMALL = [(1, 12, 8), (5, 64, 64), (130, 200, 72), (257, 1000, 300), (128, 1024, 1024), (300, 2056, 520),
+         (64, 4096, 4096 + 8)]
+
+
+@pytest.mark.parametrize("n,d,m", SMALL)
+@pytest.mark.parametrize("rho", [0.5, 0.7, 1.0])
+def test_linear_ragged_shapes(n, d, m, rho):
+    g = synthetic.rng(n * 131 + d * 7 + m)
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, n, d, 1.5))
+    B = synthetic.to_bf16(synthetic.gaussian_weight(g, d, m))
+    parity_linear(A, B, rho)
+
+
+def test_linear_k1_and_tiny_rho():
+    g = synthetic.rng(21)
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, 40, 333, 1.5))
+    B = synthetic.to_bf16(synthetic.gaussian_weight(g, 333, 96))
+    Y, idx, _ = parity_linear(A, B, 1e-4)
+    assert idx.numel() == 1
+
+
+def test_linear_strided_operands():
+    g = synthetic.rng(23)
+    Abig = synthetic.to_bf16(synthetic.outlier_activations(g, 200, 1040, 1.5)).cuda()
+    Bbig = synthetic.to_bf16(synthetic.gaussian_weight(g, 1000, 264)).cuda()
+    A = Abig[:, :1000]          # lda = 1040
+    B = Bbig[:, :256]           # ldb = 264
+    Ybig = torch.zeros((200, 272), dtype=torch.bfloat16, device="cuda")
+    Y = Ybig[:, :256]           # ldy = 272
+    rmm.linear(A, B, 0.6, out=Y)
+    torch.cuda.synchronize()
+    Aw, Bw = synthetic.widen(A.cpu()), synthetic.widen(B.cpu())
+    I, _, _ = oracle.select(Aw, 0.6)
+    check_close(synthetic.widen(Y.cpu()), oracle.reduced_product(Aw, Bw, I), "strided")
+    assert torch.count_nonzero(Ybig[:, 256:]).item() == 0
+
+
+def test_linear_identity_weight_keeps_selected_columns():
+    g = synthetic.rng(29)
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, 64, 256, 1.0))
+    B = torch.eye(256, dtype=torch.bfloat16)
+    Y, idx = rmm.linear(A.cuda(), B.cuda(), 0.5, return_idx=True)
+    torch.cuda.synchronize()
+    expect = torch.zeros_like(A)
+    I = idx.cpu().long()
+    expect[:, I] = A[:, I]
+    assert torch.equal(Y.cpu(), expect)
+
+
+@pytest.mark.parametrize("name", ["q_proj", "gate_proj", "down_proj"])
+@pytest.mark.parametrize("rho", [0.5, 0.9, 1.0])
+def test_linear_llama8b_prefill_sampled(name, rho):
+    """Full-size Llama-3.1-8B projection shapes (n = 4096), sampled output rows."""
+    A, W = synthetic.prefill_projection(name)
+    rows = np.concatenate([np.arange(0, 4096, 97), [4095]])
+    parity_linear(A, W, rho, rows=rows)
