@@ -65,3 +65,14 @@ def check_colsq(q_gpu, q_ref, rel=2e-6):
     bad = np.abs(q - r) > rel * scale
     assert not np.any(bad & (r > 0)), f"column sums of squares off at {np.nonzero(bad)[0][:10]}"
     assert np.all(q[r == 0] == 0)
+
+
+def device_padded(t, mult=8):
+    """Copy a 2-D CPU tensor to the GPU in a buffer whose row stride is a multiple of
+    ``mult`` elements (the library's leading-dimension rule); returns the view."""
+    import torch
+    rows, cols = t.shape
+    ld = (cols + mult - 1) // mult * mult
+    buf = torch.zeros((rows, ld), dtype=t.dtype, device="cuda")
+    buf[:, :cols].copy_(t)
+    return buf[:, :cols]

@@ -5,7 +5,7 @@ import torch
 
 import oracle
 import synthetic
-from parity import check_close, check_index_set
+from parity import check_close, check_index_set, device_padded
 
 pytestmark = pytest.mark.gpu
 
@@ -22,8 +22,9 @@ def built():
 
 def parity_linear(A, B, rho, rows=None):
     """Run the CUDA path and compare with the oracle (all rows, or sampled ``rows``)."""
-    Ad, Bd = A.cuda(), B.cuda()
-    Y, idx = rmm.linear(Ad, Bd, rho, return_idx=True)
+    Ad, Bd = device_padded(A), device_padded(B)
+    Y = device_padded(torch.zeros((A.shape[0], B.shape[1]), dtype=torch.bfloat16))
+    Y, idx = rmm.linear(Ad, Bd, rho, out=Y, return_idx=True)
     torch.cuda.synchronize()
     Aw, Bw = synthetic.widen(A), synthetic.widen(B)
     q = oracle.column_sq_norms(Aw)

@@ -5,7 +5,7 @@ import torch
 
 import oracle
 import synthetic
-from parity import check_colsq, check_index_set
+from parity import check_colsq, check_index_set, device_padded
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +21,7 @@ def built():
 
 
 def run_select(A_cpu, rho, causal=False):
-    A = A_cpu.cuda()
+    A = device_padded(A_cpu)
     idx, cs, rt = rmm.select(A, rho, causal=causal)
     torch.cuda.synchronize()
     return idx.cpu().numpy(), cs.cpu().numpy(), rt.cpu().numpy()
