@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the RMM hot path on one B200 (or N weak-scaled replicas).
+
+Workload: the Llama-3.1-8B prefill projections q_proj (4096x4096), gate_proj and
+up_proj (4096x14336) and down_proj (14336x4096) at n = 4096 tokens, synthetic
+bf16 activations with outlier channels and N(0, 1/d) weights.  One step = the
+whole reduced path for all four projections at rho = 0.5: column scores, TopK
+selection, pack of A[:, I] and the tensor-core product with B[I, :] gathered by
+row.  Metric: kept-FLOP TFLOP/s (2 n k m per projection with k = ceil(rho d)),
+plus GB/s over the kept bytes and the speedup over the library's own rho = 1
+path at rho in {0.9, 0.7, 0.5}.
+
+`--impl reference` times the CPU oracle instead (a deliberately slow program:
+fp64 numpy on the host cores, a bounded sample of rows per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "kept-FLOP TFLOP/s, GB/s & speedup vs own ρ=1 path at ρ∈{0.9,0.7,0.5}"
+PROJ = ["q_proj", "gate_proj", "up_proj", "down_proj"]
+N_TOKENS = 4096
+RHO_MAIN = 0.5
+RHO_SWEEP = (0.9, 0.7)
+GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm.cuh", "input_adaptive_reduced_colnorm_b200/csrc/ptx.cuh"]
+TRAFFIC_PROFILE = "profiles/gemm_gather_llama8b_gate.md"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="rows per projection in the CPU-oracle sample")
+    return ap.parse_args()
+
+
+def shapes():
+    from synthetic import PREFILL_SHAPES
+    return [(p, N_TOKENS) + PREFILL_SHAPES[p] for p in PROJ]  # (name, n, d, m)
+
+
+def k_of(rho, d):
+    # same rule as the library's rmm_k (ceil with a 1e-9 relative guard)
+    import math
+    x = rho * d
+    return max(1, min(d, math.ceil(x - 1e-9 * x)))
+
+
+def kept_flops(n, d, m, rho):
+    return 2.0 * n * k_of(rho, d) * m
+
+
+def kept_bytes(n, d, m, rho):
+    k = k_of(rho, d)
+    if k == d:
+        return 2.0 * (n * d + d * m + n * m)
+    return 2.0 * (n * d + n * k + k * m + n * m)
+
+
+def step_flops(rho):
+    return sum(kept_flops(n, d, m, rho) for _, n, d, m in shapes())
+
+
+def step_bytes(rho):
+    return sum(kept_bytes(n, d, m, rho) for _, n, d, m in shapes())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        for b, name in self.REASONS.items():
+            if bits & b:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ helpers
+def gemm_source_sha1():
+    h = hashlib.sha1()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per gathered-GEMM launch from the committed ncu summary, if the
+    kernel source is unchanged since that capture; else None."""
+    path = os.path.join(ROOT, TRAFFIC_PROFILE)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"source_sha1:\s*([0-9a-f]{40})", text)
+    if not m or not s or s.group(1) != gemm_source_sha1():
+        return None
+    return float(m.group(1))
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def oracle_step(host_inputs, rows, rho):
+    """One bounded oracle step: selection over all rows, product for ``rows`` rows."""
+    import oracle
+    flops = 0.0
+    for name, (Aw, Ww) in host_inputs.items():
+        I, _, _ = oracle.select(Aw, rho)
+        oracle.rmm_linear_rows(Aw, Ww, I, rows)
+        flops += 2.0 * len(rows) * len(I) * Ww.shape[1]
+    return flops
+
+
+def cpu_oracle_inputs():
+    import synthetic
+    out = {}
+    for name in PROJ:
+        A, W = synthetic.prefill_projection(name)
+        out[name] = (synthetic.widen(A), synthetic.widen(W))
+    return out
+
+
+def cpu_baseline(nrows):
+    import numpy as np
+    host = cpu_oracle_inputs()
+    rows = np.linspace(0, N_TOKENS - 1, nrows).astype(np.int64)
+    t0 = time.perf_counter()
+    flops = oracle_step(host, rows, RHO_MAIN)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "seconds": dt,
+            "sample": f"q/gate/up/down at rho={RHO_MAIN}: fp64 column norms and TopK over all {N_TOKENS} rows, "
+                      f"reduced product for {nrows} of {N_TOKENS} rows per projection (kept FLOPs of those rows / "
+                      f"wall time of the whole sample)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    host = cpu_oracle_inputs()
+    rows = np.linspace(0, N_TOKENS - 1, 16).astype(np.int64)
+    for _ in range(args.warmup):
+        oracle_step(host, rows, RHO_MAIN)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += oracle_step(host, rows, RHO_MAIN)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = (f"q/gate/up/down at rho={RHO_MAIN}: fp64 norms + TopK over all {N_TOKENS} rows and the reduced "
+              f"product for 16 rows per projection, per step")
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "llama3.1-8b prefill projections (oracle sample)", "n": N_TOKENS,
+                       "rho": RHO_MAIN, "projections": PROJ},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU leg
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            t = torch.zeros(1, device=dev)
+            dist.all_reduce(t)
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    from input_adaptive_reduced_colnorm_b200 import build as rmm_build
+    rmm_build.build()
+    import input_adaptive_reduced_colnorm_b200 as rmm
+    import synthetic
+    import ctypes
+
+    L = rmm.lib()
+    stream = torch.cuda.current_stream(dev)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+
+    # inputs: each rank draws its own replica (weak scaling, no data-path collective)
+    bufs = []
+    for name, n, d, m in shapes():
+        A, W = synthetic.prefill_projection(name, seed=synthetic.seed_for(2) + 1000 * rank)
+        b = {"name": name, "n": n, "d": d, "m": m, "A": A.to(dev), "W": W.to(dev),
+             "Y": torch.empty((n, m), dtype=torch.bfloat16, device=dev),
+             "A_host": A.pin_memory(), "Y_host": torch.empty((n, m), dtype=torch.bfloat16).pin_memory()}
+        kmax = k_of(0.9, d)
+        b["idx"] = torch.empty(kmax, dtype=torch.int32, device=dev)
+        b["colsq"] = torch.empty(d, dtype=torch.float64, device=dev)
+        b["apack"] = torch.empty(n * ((kmax + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
+        b["ws"] = torch.empty(max(L.rmm_linear_workspace_bytes(n, d, m, 0.9), 256), dtype=torch.uint8, device=dev)
+        bufs.append(b)
+    del A, W
+
+    def call(status):
+        if status != 0:
+            raise RuntimeError(f"rmm call failed: {L.rmm_status_string(status).decode()}: "
+                               f"{L.rmm_last_error().decode()}")
+
+    def step_stages(rho, ev=None):
+        """One step through the stage entry points (select, gather_columns, gather_gemm)."""
+        for i, b in enumerate(bufs):
+            n, d, m = b["n"], b["d"], b["m"]
+            k = k_of(rho, d)
+            ldp = (k + 7) // 8 * 8
+            call(L.rmm_select(b["A"].data_ptr(), 1, n * d, n, d, d, 0, rho, b["idx"].data_ptr(),
+                              b["colsq"].data_ptr(), None, None, 0, sptr))
+            call(L.rmm_gather_columns(b["A"].data_ptr(), n, d, d, b["idx"].data_ptr(), k, b["apack"].data_ptr(), ldp,
+                                      sptr))
+            if ev is not None:
+                ev[i][0].record(stream)
+            call(L.rmm_gather_gemm(b["apack"].data_ptr(), n, k, ldp, b["W"].data_ptr(), d, m, m,
+                                   b["idx"].data_ptr(), b["Y"].data_ptr(), m, sptr))
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    def step_linear(rho):
+        """One step through the public rmm_linear call."""
+        for b in bufs:
+            n, d, m = b["n"], b["d"], b["m"]
+            call(L.rmm_linear(b["A"].data_ptr(), n, d, d, b["W"].data_ptr(), m, m, b["Y"].data_ptr(), m, rho, None,
+                              b["ws"].data_ptr(), b["ws"].numel(), sptr))
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / steps)
+
+    K, W = args.steps, args.warmup
+    # ---- main timed region: rho = 0.5 through the stage entry points, GEMM bracketed by events
+    for _ in range(W):
+        step_stages(RHO_MAIN)
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in bufs]
+           for _ in range(K)]
+    barrier()
+    sampler = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        e0.record(stream)
+        for s in range(K):
+            step_stages(RHO_MAIN, evs[s])
+        e1.record(stream)
+        barrier()
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / K)
+    gemm_ms = [statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)) for i in range(len(bufs))]
+    gemm_ms = [max_over_ranks(x) for x in gemm_ms]
+
+    # ---- rho sweep and the rho = 1 dense path through rmm_linear
+    ms_rho = {RHO_MAIN: ms_step}
+    for rho in RHO_SWEEP:
+        ms_rho[rho] = timed(lambda: step_linear(rho), K, W)
+    ms_linear_main = timed(lambda: step_linear(RHO_MAIN), K, W)
+    ms_dense = timed(lambda: step_linear(1.0), K, W)
+
+    def step_cublas():
+        for b in bufs:
+            torch.matmul(b["A"], b["W"], out=b["Y"])
+    ms_cublas = timed(step_cublas, K, W)
+
+    # ---- end to end: host activations in, host outputs out, through rmm.linear
+    def step_e2e():
+        for b in bufs:
+            b["A"].copy_(b["A_host"], non_blocking=True)
+            rmm.linear(b["A"], b["W"], RHO_MAIN, out=b["Y"], workspace=b["ws"])
+            b["Y_host"].copy_(b["Y"], non_blocking=True)
+    ms_e2e = timed(step_e2e, max(3, K // 4), W)
+    h2d = sum(b["A"].numel() * 2 for b in bufs)
+    d2h = sum(b["Y"].numel() * 2 for b in bufs)
+
+    # ---- numbers
+    flops = step_flops(RHO_MAIN)
+    nbytes = step_bytes(RHO_MAIN)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    gate = [i for i, b in enumerate(bufs) if b["name"] == "gate_proj"][0]
+    b = bufs[gate]
+    gate_flops = kept_flops(b["n"], b["d"], b["m"], RHO_MAIN)
+    achieved = gate_flops / (gemm_ms[gate] * 1e-3) / 1e12
+    all_gemm = sum(kept_flops(x["n"], x["d"], x["m"], RHO_MAIN) for x in bufs) / (sum(gemm_ms) * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "llama3.1-8b prefill projections q/gate/up/down, n=4096 tokens, rho=0.5",
+                   "n": N_TOKENS, "rho": RHO_MAIN, "projections": PROJ, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (about 0.7 GB touched per step)"},
+        "gbs": world * nbytes / (ms_step * 1e-3) / 1e9,
+        "rho_sweep": {str(r): {"ms_per_step": ms_rho[r], "tflops": world * step_flops(r) / (ms_rho[r] * 1e-3) / 1e12,
+                               "gbs": world * step_bytes(r) / (ms_rho[r] * 1e-3) / 1e9,
+                               "speedup_vs_rho1": ms_dense / ms_rho[r]} for r in (0.9, 0.7, 0.5)},
+        "speedup_vs_rho1": {str(r): ms_dense / ms_rho[r] for r in (0.9, 0.7, 0.5)},
+        "rho1": {"ms_per_step": ms_dense, "tflops": world * step_flops(1.0) / (ms_dense * 1e-3) / 1e12,
+                 "cublas_ms_per_step": ms_cublas, "speedup_vs_cublas": ms_cublas / ms_dense},
+        "rmm_linear_ms_per_step_rho0.5": ms_linear_main,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "kernel": "rmm_gemm_kernel<256, gather> on gate_proj (4096 x 14336, k=2048)",
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                     "all_gemm_launches_tflops": all_gemm},
+        "gemm_ms_per_launch": {x["name"]: gemm_ms[i] for i, x in enumerate(bufs)},
+        "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": 16 * K,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

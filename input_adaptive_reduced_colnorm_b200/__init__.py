@@ -13,7 +13,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["lib", "rmm_k", "select", "linear", "qk", "pv", "RMMError", "device_error", "library_path"]
+__all__ = ["lib", "rmm_k", "select", "linear", "gather_columns", "gather_gemm", "qk", "pv", "RMMError", "device_error", "library_path"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -44,6 +44,9 @@ _SIGNATURES = {
     "rmm_linear_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_linear": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_dbl, _c_p, _c_p,
                             _c_size, _c_p]),
+    "rmm_gather_columns": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_i64, _c_p]),
+    "rmm_gather_gemm": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64,
+                                 _c_p]),
     "rmm_qk_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_qk": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_float, _c_dbl,
                         _c_p, _c_p, _c_size, _c_p]),
@@ -168,6 +171,34 @@ def linear(A, B, rho: float, *, out=None, return_idx: bool = False, workspace=No
     _check(L.rmm_linear(_ptr(A), n, d, A.stride(0), _ptr(B), m, B.stride(0), _ptr(out), out.stride(0), float(rho),
                         _ptr(idx), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
     return (out, idx) if return_idx else out
+
+
+def gather_columns(A, idx, out=None, ld_pack=None):
+    """A_pack[:, :k] = A[:, idx], zero-padded; returns the [n, ld_pack] buffer."""
+    import torch
+    _require(A, "A", torch.bfloat16, 2)
+    n, d = A.shape
+    k = idx.numel()
+    if out is None:
+        ld = ((k + 7) // 8) * 8 if ld_pack is None else ld_pack
+        out = torch.empty((n, ld), dtype=torch.bfloat16, device=A.device)
+    _check(lib().rmm_gather_columns(_ptr(A), n, d, A.stride(0), _ptr(idx), k, _ptr(out), out.stride(0),
+                                    _stream(A.device)))
+    return out
+
+
+def gather_gemm(A_pack, k, B, idx, out=None):
+    """Y = A_pack[:, :k] . B[idx, :] (tensor cores, B rows gathered by index)."""
+    import torch
+    _require(A_pack, "A_pack", torch.bfloat16, 2)
+    _require(B, "B", torch.bfloat16, 2)
+    n = A_pack.shape[0]
+    d, m = B.shape
+    if out is None:
+        out = torch.empty((n, m), dtype=torch.bfloat16, device=B.device)
+    _check(lib().rmm_gather_gemm(_ptr(A_pack), n, int(k), A_pack.stride(0), _ptr(B), d, m, B.stride(0), _ptr(idx),
+                                 _ptr(out), out.stride(0), _stream(B.device)))
+    return out
 
 
 def qk(Q, K, rho: float, *, causal: bool = True, scale: float = 1.0, out=None, return_idx: bool = False,

@@ -224,6 +224,44 @@ rmm_status check_rho(double rho) {
   return RMM_OK;
 }
 
+// S3 of the linear path: A_pack = A[:, I] (zero-padded to ld_pack columns).
+rmm_status pack_columns(const uint16_t* A, int64_t n, int64_t d, int64_t lda, const int32_t* idx, int64_t k,
+                        uint16_t* apack, int64_t ld_pack, cudaStream_t s) {
+  PackParams pk{};
+  pk.src = A;
+  pk.src_ld = lda;
+  pk.rows = n;
+  pk.d = d;
+  pk.g_outer = 1;
+  pk.g_inner = 1;
+  pk.idx = idx;
+  pk.k = k;
+  pk.k_pad = ld_pack;
+  pk.dst = apack;
+  pk.batch = 1;
+  return launch_pack(pk, s);
+}
+
+// S4 of the linear path: Y = A_pack[:, :k] . B[I, :] with B rows gathered by TMA.
+rmm_status gather_gemm(const uint16_t* apack, int64_t n, int64_t k, int64_t ld_pack, const uint16_t* B, int64_t d,
+                       int64_t m, int64_t ldb, const int32_t* idx, uint16_t* Y, int64_t ldy, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (rmm_status st = make_tmap(&ta, apack, ld_pack, n, ld_pack * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tb, B, m, d, ldb * 2, 64, 1)) return st;
+  GemmParams g = gemm_defaults();
+  g.M = static_cast<int>(n);
+  g.N = static_cast<int>(m);
+  g.out = Y;
+  g.ldo = ldy;
+  g.m_tiles = static_cast<int>(ceil_div(n, 128));
+  g.n_tiles = static_cast<int>(ceil_div(m, 256));
+  g.k = static_cast<int>(k);
+  g.num_kb = static_cast<int>(ceil_div(k, 64));
+  g.idx = idx;
+  g.b_oob_row = static_cast<int>(d);
+  return launch_gemm<256, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+}
+
 }  // namespace
 
 // ============================================================== public API
@@ -367,26 +405,32 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
 
   if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
   if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
-  PackParams pk{};
-  pk.src = A;
-  pk.src_ld = lda;
-  pk.rows = n;
-  pk.d = d;
-  pk.g_outer = 1;
-  pk.g_inner = 1;
-  pk.idx = idx;
-  pk.k = k;
-  pk.k_pad = k_pad;
-  pk.dst = apack;
-  pk.batch = 1;
-  if (rmm_status st = launch_pack(pk, s)) return st;
-  if (rmm_status st = make_tmap(&ta, apack, k_pad, n, k_pad * 2, 64, 128)) return st;
-  if (rmm_status st = make_tmap(&tb, B, m, d, ldb * 2, 64, 1)) return st;
-  g.k = static_cast<int>(k);
-  g.num_kb = static_cast<int>(ceil_div(k, 64));
-  g.idx = idx;
-  g.b_oob_row = static_cast<int>(d);
-  return launch_gemm<256, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  if (rmm_status st = pack_columns(A, n, d, lda, idx, k, apack, k_pad, s)) return st;
+  return gather_gemm(apack, n, k, k_pad, B, d, m, ldb, idx, Y, ldy, s);
+}
+
+rmm_status rmm_gather_columns(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int32_t* idx, int64_t k,
+                              rmm_bf16* A_pack, int64_t ld_pack, rmm_stream stream) {
+  t_last_error.clear();
+  if (A == nullptr || idx == nullptr || A_pack == nullptr) return fail(RMM_ERR_INVALID_ARG, "null pointer");
+  if (n < 1 || d < 1 || k < 1 || k > d || lda < d || ld_pack < k)
+    return fail(RMM_ERR_INVALID_ARG, "need n, d >= 1, 1 <= k <= d, lda >= d, ld_pack >= k");
+  if (!aligned16(A) || !aligned16(A_pack) || (lda % 8) || (ld_pack % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
+  if (d > kMaxSelectD || n > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  return pack_columns(A, n, d, lda, idx, k, A_pack, ld_pack, static_cast<cudaStream_t>(stream));
+}
+
+rmm_status rmm_gather_gemm(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t ld_pack, const rmm_bf16* B, int64_t d,
+                           int64_t m, int64_t ldb, const int32_t* idx, rmm_bf16* Y, int64_t ldy, rmm_stream stream) {
+  t_last_error.clear();
+  if (A_pack == nullptr || B == nullptr || idx == nullptr || Y == nullptr) return fail(RMM_ERR_INVALID_ARG, "null pointer");
+  if (n < 1 || k < 1 || d < k || m < 1 || ld_pack < k || ldb < m || ldy < m)
+    return fail(RMM_ERR_INVALID_ARG, "need n, m >= 1, 1 <= k <= d, ld_pack >= k, ldb and ldy >= m");
+  if (!aligned16(A_pack) || !aligned16(B) || !aligned16(Y) || (ld_pack % 8) || (ldb % 8) || (ldy % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
+  if (n > kIntMax - 128 || m > kIntMax - 256 || d > kIntMax - 64) return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  return gather_gemm(A_pack, n, k, ld_pack, B, d, m, ldb, idx, Y, ldy, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- QK^T

@@ -113,3 +113,21 @@ def test_linear_llama8b_prefill_sampled(name, rho):
     A, W = synthetic.prefill_projection(name)
     rows = np.concatenate([np.arange(0, 4096, 97), [4095]])
     parity_linear(A, W, rho, rows=rows)
+
+
+def test_stage_entry_points_compose_to_rmm_linear():
+    """rmm_select -> rmm_gather_columns -> rmm_gather_gemm gives the same bits as rmm_linear."""
+    g = synthetic.rng(31)
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, 300, 1000, 1.5)).cuda()
+    B = synthetic.to_bf16(synthetic.gaussian_weight(g, 1000, 520)).cuda()
+    Y, idx = rmm.linear(A, B, 0.7, return_idx=True)
+    idx2, _, _ = rmm.select(A, 0.7)
+    k = idx2.numel()
+    ap = rmm.gather_columns(A, idx2, ld_pack=712)
+    Y2 = rmm.gather_gemm(ap, k, B, idx2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2)
+    assert torch.equal(Y, Y2)
+    expect = torch.zeros((300, 712), dtype=torch.bfloat16)
+    expect[:, :k] = A.cpu()[:, idx2.cpu().long()]
+    assert torch.equal(ap.cpu(), expect)
