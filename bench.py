@@ -5,8 +5,7 @@ Workload: the Llama-3.1-8B prefill projections q_proj (4096x4096), gate_proj and
 up_proj (4096x14336) and down_proj (14336x4096) at n = 4096 tokens, synthetic
 bf16 activations with outlier channels and N(0, 1/d) weights.  One step = the
 whole reduced path for all four projections at rho = 0.5: column scores, TopK
-selection, pack of A[:, I] and the tensor-core product with B[I, :] gathered by
-row.  Metric: kept-FLOP TFLOP/s (2 n k m per projection with k = ceil(rho d)),
+selection, pack of A[:, I], row pack of B[I, :] and the tensor-core product.  Metric: kept-FLOP TFLOP/s (2 n k m per projection with k = ceil(rho d)),
 plus GB/s over the kept bytes and the speedup over the library's own rho = 1
 path at rho in {0.9, 0.7, 0.5}.
 
@@ -35,7 +34,7 @@ N_TOKENS = 4096
 RHO_MAIN = 0.5
 RHO_SWEEP = (0.9, 0.7)
 GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm.cuh", "input_adaptive_reduced_colnorm_b200/csrc/ptx.cuh"]
-TRAFFIC_PROFILE = "profiles/gemm_gather_llama8b_gate.md"
+TRAFFIC_PROFILE = "profiles/gemm_packed_llama8b_gate.md"
 
 
 def parse_args():
@@ -45,7 +44,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=256, help="rows per projection in the CPU-oracle sample")
+    ap.add_argument("--cpu-rows", type=int, default=4096, help="rows per projection in the CPU-oracle sample")
     return ap.parse_args()
 
 
@@ -151,7 +150,7 @@ def gemm_source_sha1():
 
 
 def profiled_traffic():
-    """DRAM bytes per gathered-GEMM launch from the committed ncu summary, if the
+    """DRAM bytes per packed-GEMM launch from the committed ncu summary, if the
     kernel source is unchanged since that capture; else None."""
     path = os.path.join(ROOT, TRAFFIC_PROFILE)
     if not os.path.exists(path):
@@ -295,6 +294,7 @@ def run_ours(args):
         b["idx"] = torch.empty(kmax, dtype=torch.int32, device=dev)
         b["colsq"] = torch.empty(d, dtype=torch.float64, device=dev)
         b["apack"] = torch.empty(n * ((kmax + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
+        b["bpack"] = torch.empty(kmax * ((m + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)
         b["ws"] = torch.empty(max(L.rmm_linear_workspace_bytes(n, d, m, 0.9), 256), dtype=torch.uint8, device=dev)
         bufs.append(b)
     del A, W
@@ -305,19 +305,23 @@ def run_ours(args):
                                f"{L.rmm_last_error().decode()}")
 
     def step_stages(rho, ev=None):
-        """One step through the stage entry points (select, gather_columns, gather_gemm)."""
+        """One step through the stage entry points: select, gather_columns,
+        gather_rows, gemm_packed (the same kernels rmm_linear launches)."""
         for i, b in enumerate(bufs):
             n, d, m = b["n"], b["d"], b["m"]
             k = k_of(rho, d)
             ldp = (k + 7) // 8 * 8
+            ldm = (m + 7) // 8 * 8
             call(L.rmm_select(b["A"].data_ptr(), 1, n * d, n, d, d, 0, rho, b["idx"].data_ptr(),
                               b["colsq"].data_ptr(), None, None, 0, sptr))
             call(L.rmm_gather_columns(b["A"].data_ptr(), n, d, d, b["idx"].data_ptr(), k, b["apack"].data_ptr(), ldp,
                                       sptr))
+            call(L.rmm_gather_rows(b["W"].data_ptr(), d, m, m, b["idx"].data_ptr(), k, b["bpack"].data_ptr(), ldm,
+                                   sptr))
             if ev is not None:
                 ev[i][0].record(stream)
-            call(L.rmm_gather_gemm(b["apack"].data_ptr(), n, k, ldp, b["W"].data_ptr(), d, m, m,
-                                   b["idx"].data_ptr(), b["Y"].data_ptr(), m, sptr))
+            call(L.rmm_gemm_packed(b["apack"].data_ptr(), n, k, ldp, b["bpack"].data_ptr(), m, ldm,
+                                   b["Y"].data_ptr(), m, sptr))
             if ev is not None:
                 ev[i][1].record(stream)
 
@@ -410,13 +414,13 @@ def run_ours(args):
         "rmm_linear_ms_per_step_rho0.5": ms_linear_main,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(),
-                     "kernel": "rmm_gemm_kernel<256, gather> on gate_proj (4096 x 14336, k=2048)",
+                     "kernel": "rmm_gemm_kernel<256, MN tile> on packed gate_proj operands (4096 x 14336, k=2048)",
                      "peak_source": f"bf16_tflops_sustained of {peak_src}",
                      "all_gemm_launches_tflops": all_gemm},
         "gemm_ms_per_launch": {x["name"]: gemm_ms[i] for i, x in enumerate(bufs)},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-        "gpu_launches": 16 * K,
+        "gpu_launches": 20 * K,
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

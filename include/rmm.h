@@ -106,24 +106,30 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
                       rmm_stream stream);
 
 /* ---------------------------------------------------------------- linear stages
- * The two steps that follow the selection in rmm_linear, exposed so a caller
- * can run (or time) them on their own; rmm_linear with rho < 1 and n > 32 is
- * rmm_select's kernels followed by exactly these two calls.
+ * The steps that follow the selection in rmm_linear, exposed so a caller can
+ * run (or time) them on their own.  rmm_linear with rho < 1 is rmm_select's
+ * kernels followed by exactly rmm_gather_columns, rmm_gather_rows and
+ * rmm_gemm_packed; with rho = 1 it is rmm_gemm_packed on A and B themselves.
  *
  * rmm_gather_columns: A_pack[i, t] = A[i, idx[t]] for t < k and 0 for
  * k <= t < ld_pack -- the gathered A[:, I] of "Core Approach", stored K-major.
  *   A       device bf16 [n][lda], n x d.
- *   idx     device int32 [k], every entry in [0, d) (not checked on the host).
+ *   idx     device int32 [k], entries in [0, d) (not checked on the host).
  *   A_pack  device bf16 [n][ld_pack]; ld_pack >= k and a multiple of 8.
- * rmm_gather_gemm: Y = A_pack[:, :k] . B[idx, :] on the tensor cores; the k
- * rows of B are gathered by index straight from B ("Core Approach":
- * A[:, I] B[I, :]).
- *   B  device bf16 [d][ldb], d x m;  Y  device bf16 [n][ldy], n x m.
- * Neither call needs a workspace. */
+ * rmm_gather_rows: B_pack[t, :] = B[idx[t], :] for t < k -- the kept rows
+ * B[I, :] of "Core Approach", copied row-contiguous.
+ *   B       device bf16 [d][ldb], d x m;  B_pack device bf16 [k][ld_pack],
+ *   ld_pack >= m and a multiple of 8.
+ * rmm_gemm_packed: Y = A_pack[:, :k] . B_pack[:k, :] on the tensor cores
+ * (tcgen05, fp32 accumulation in tensor memory, bf16 output).
+ *   A_pack [n][lda] (lda >= k), B_pack [k][ldb] (ldb >= m), Y [n][ldy].
+ * None of the three needs a workspace. */
 rmm_status rmm_gather_columns(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int32_t* idx, int64_t k,
                               rmm_bf16* A_pack, int64_t ld_pack, rmm_stream stream);
-rmm_status rmm_gather_gemm(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t ld_pack, const rmm_bf16* B, int64_t d,
-                           int64_t m, int64_t ldb, const int32_t* idx, rmm_bf16* Y, int64_t ldy, rmm_stream stream);
+rmm_status rmm_gather_rows(const rmm_bf16* B, int64_t d, int64_t m, int64_t ldb, const int32_t* idx, int64_t k,
+                           rmm_bf16* B_pack, int64_t ld_pack, rmm_stream stream);
+rmm_status rmm_gemm_packed(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t lda, const rmm_bf16* B_pack,
+                           int64_t m, int64_t ldb, rmm_bf16* Y, int64_t ldy, rmm_stream stream);
 
 /* ---------------------------------------------------------------- attention scores
  * rmm_qk: per query head h, I_h = TopK of the column norms of Q_h over its nq

@@ -13,7 +13,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["lib", "rmm_k", "select", "linear", "gather_columns", "gather_gemm", "qk", "pv", "RMMError", "device_error", "library_path"]
+__all__ = ["lib", "rmm_k", "select", "linear", "gather_columns", "gather_rows", "gemm_packed", "qk", "pv", "RMMError", "device_error", "library_path"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -45,8 +45,8 @@ _SIGNATURES = {
     "rmm_linear": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_dbl, _c_p, _c_p,
                             _c_size, _c_p]),
     "rmm_gather_columns": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_i64, _c_p]),
-    "rmm_gather_gemm": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64,
-                                 _c_p]),
+    "rmm_gather_rows": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_i64, _c_p]),
+    "rmm_gemm_packed": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p]),
     "rmm_qk_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_qk": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_float, _c_dbl,
                         _c_p, _c_p, _c_size, _c_p]),
@@ -187,17 +187,30 @@ def gather_columns(A, idx, out=None, ld_pack=None):
     return out
 
 
-def gather_gemm(A_pack, k, B, idx, out=None):
-    """Y = A_pack[:, :k] . B[idx, :] (tensor cores, B rows gathered by index)."""
+def gather_rows(B, idx, out=None, ld_pack=None):
+    """B_pack[t, :] = B[idx[t], :]; returns the [k, ld_pack] buffer."""
+    import torch
+    _require(B, "B", torch.bfloat16, 2)
+    d, m = B.shape
+    k = idx.numel()
+    if out is None:
+        ld = ((m + 7) // 8) * 8 if ld_pack is None else ld_pack
+        out = torch.empty((k, ld), dtype=torch.bfloat16, device=B.device)
+    _check(lib().rmm_gather_rows(_ptr(B), d, m, B.stride(0), _ptr(idx), k, _ptr(out), out.stride(0),
+                                 _stream(B.device)))
+    return out
+
+
+def gemm_packed(A_pack, k, B_pack, m, out=None):
+    """Y = A_pack[:, :k] . B_pack[:k, :m] on the tensor cores."""
     import torch
     _require(A_pack, "A_pack", torch.bfloat16, 2)
-    _require(B, "B", torch.bfloat16, 2)
+    _require(B_pack, "B_pack", torch.bfloat16, 2)
     n = A_pack.shape[0]
-    d, m = B.shape
     if out is None:
-        out = torch.empty((n, m), dtype=torch.bfloat16, device=B.device)
-    _check(lib().rmm_gather_gemm(_ptr(A_pack), n, int(k), A_pack.stride(0), _ptr(B), d, m, B.stride(0), _ptr(idx),
-                                 _ptr(out), out.stride(0), _stream(B.device)))
+        out = torch.empty((n, m), dtype=torch.bfloat16, device=A_pack.device)
+    _check(lib().rmm_gemm_packed(_ptr(A_pack), n, int(k), A_pack.stride(0), _ptr(B_pack), int(m), B_pack.stride(0),
+                                 _ptr(out), out.stride(0), _stream(A_pack.device)))
     return out
 
 

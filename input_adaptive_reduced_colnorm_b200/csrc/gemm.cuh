@@ -5,10 +5,14 @@
 //
 // Persistent, warp-specialised tcgen05 kernel, one CTA per SM:
 //   warp 0      TMA producer: A tile (K-major, 128 x 64 bf16, 128-byte swizzle)
-//               and B tile, either gathered row by row from B[I, :] with
-//               tile::gather4 (four kept rows per copy), loaded as a plain
-//               MN-major tile (rho = 1 path, I = [0, d)), or loaded as a K-major
-//               tile (per-head Q K^T where K is packed like Q).
+//               and B tile, either MN-major (64 contraction rows x BN columns,
+//               B[I, :] packed row-contiguous beforehand, or B itself on the
+//               rho = 1 path) or K-major (per-head Q K^T, K packed like Q).
+//               Kept rows are packed before the GEMM rather than gathered per
+//               tile: on B200 a TMA row gather (tile::gather4, 4 rows x 128 B per
+//               copy) or a 512-byte bulk copy per row stages only ~7-8 B/clk/SM,
+//               while 64 x 64 tiles stage ~44 B/clk/SM, so the per-copy cost of
+//               small TMA copies, not DRAM, would bound the product.
 //   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma (M=128,
 //               N=BN, K=16 per instruction) into a double-buffered fp32
 //               accumulator in TMEM and commits to mbarriers.
@@ -23,7 +27,7 @@
 
 namespace rmm {
 
-enum BMode : int { kBGather = 0, kBTileMN = 1, kBTileK = 2 };
+enum BMode : int { kBTileMN = 1, kBTileK = 2 };
 enum EpiMode : int { kEpiBf16 = 0, kEpiF32 = 1 };
 enum CausalMode : int { kCausalNone = 0, kCausalMaskScores = 1, kCausalLimitK = 2 };
 
@@ -34,14 +38,13 @@ struct GemmParams {
   int batch;
   int m_tiles, n_tiles;
   int a_rows_per_batch;  // A tensor-map row of (b, m) = b * a_rows_per_batch + m
-  // B tensor-map row of batch item b: b_row_base(b) + I_b[t] (gather), + t (MN
-  // tile) or + n (K-major tile), b_row_base(b) = (b / b_g_outer) * b_s_outer +
+  // B tensor-map row of batch item b: b_row_base(b) + t (MN tile, contraction
+  // row t) or + n (K-major tile), b_row_base(b) = (b / b_g_outer) * b_s_outer +
   // ((b % b_g_outer) / b_g_inner) * b_s_inner
-  const int32_t* idx;    // [batch][k] ascending kept indices, or null for I = [0, k)
+  const int32_t* idx;    // [batch][k] ascending kept indices (causal k-limit), or null for I = [0, k)
   int64_t idx_bstride;
   int b_g_outer, b_g_inner;
   int64_t b_s_outer, b_s_inner;
-  int b_oob_row;         // a row index outside the B tensor (reads zeros)
   // output
   void* out;
   int64_t ldo;           // elements between output rows
@@ -159,7 +162,6 @@ __global__ void __launch_bounds__(192, 1)
       const int n0 = nt * BN;
       const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, n0);
       const int a_row = b * p.a_rows_per_batch + m0;
-      const int32_t* I = p.idx + static_cast<int64_t>(b) * p.idx_bstride;
       const int64_t brow0 = gemm_b_row_base(p, b);
       for (int kb = 0; kb < nkb; ++kb) {
         int w = 1;
@@ -175,20 +177,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
         uint8_t* dstB = sB + stage * C::B_BYTES;
-        if (BMODE == kBGather) {
-          // 16 groups of 4 kept rows x (BN / 64) column chunks of 64
-          constexpr int OPS = 16 * (BN / 64);
-          for (int op = lane; op < OPS; op += 32) {
-            const int g = op & 15, c = op >> 4;
-            int32_t r[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int t = kb * 64 + g * 4 + q;
-              r[q] = (t < p.k) ? static_cast<int32_t>(brow0 + __ldg(I + t)) : p.b_oob_row;
-            }
-            tma_gather4(dstB + c * 8192 + g * 512, &tmB, &full[stage], n0 + c * 64, r[0], r[1], r[2], r[3]);
-          }
-        } else if (BMODE == kBTileMN) {
+        if (BMODE == kBTileMN) {
           if (lane < BN / 64)
             tma_load_2d(dstB + lane * 8192, &tmB, &full[stage], n0 + lane * 64, static_cast<int32_t>(brow0 + kb * 64));
         } else {

@@ -127,4 +127,61 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p) 
   }
 }
 
+// Row pack of the kept contraction rows of the second operand:
+// dst[b][t, :] = src_item(b)[I_b[t], :] for t < k, zero rows for k <= t < rows_out
+// ("Algorithm Deep-Dive: RMM", Core Approach: B[I, :]).  Whole rows are
+// contiguous, so this is a fully coalesced 16-byte copy at HBM speed; the
+// tensor-core GEMM then streams B[I, :] with large TMA tiles.
+struct RowPackParams {
+  const uint16_t* src;
+  int64_t src_ld;                             // elements between source rows
+  int64_t cols;                               // columns copied per row
+  const int32_t* idx;                         // [batch][k]
+  int64_t k;
+  int64_t rows_out;                           // rows per batch item in dst (>= k)
+  uint16_t* dst;
+  int64_t dst_ld;                             // multiple of 8, >= cols
+  int64_t batch;
+  int64_t g_outer, g_inner, s_outer, s_inner; // source item of b (as in PackParams)
+};
+
+__global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackParams p) {
+  constexpr int ILP = 4;
+  const int64_t vpr = (p.cols + 7) / 8;  // 16-byte vectors per row
+  const int64_t total = p.batch * p.rows_out * vpr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v0 < total; v0 += ILP * stride) {
+    uint4 val[ILP];
+    int64_t out_off[ILP];
+#pragma unroll
+    for (int u = 0; u < ILP; ++u) {
+      const int64_t v = v0 + u * stride;
+      val[u] = make_uint4(0u, 0u, 0u, 0u);
+      out_off[u] = -1;
+      if (v < total) {
+        const int64_t row = v / vpr;
+        const int64_t c = v - row * vpr;
+        const int64_t b = row / p.rows_out;
+        const int64_t t = row - b * p.rows_out;
+        out_off[u] = row * p.dst_ld + c * 8;
+        if (t < p.k) {
+          const int64_t j = __ldg(p.idx + b * p.k + t);
+          const int64_t item = (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+          const uint16_t* src = p.src + item + j * p.src_ld + c * 8;
+          if (c * 8 + 8 <= p.cols) {
+            val[u] = ldg_nc_v4(src);
+          } else {
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            for (int e = 0; c * 8 + e < p.cols; ++e) w[e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
+            val[u] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < ILP; ++u)
+      if (out_off[u] >= 0) *reinterpret_cast<uint4*>(p.dst + out_off[u]) = val[u];
+  }
+}
+
 }  // namespace rmm

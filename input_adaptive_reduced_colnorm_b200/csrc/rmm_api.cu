@@ -193,6 +193,15 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
   return RMM_OK;
 }
 
+rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
+  const int64_t total = p.batch * p.rows_out * ((p.cols + 7) / 8);
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256 * 4), 8LL * num_sms()));
+  pack_rows_gather_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "row pack launch");
+  return RMM_OK;
+}
+
 template <int BN, int BMODE, int EPI, int CAUSAL>
 rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t s) {
   auto kern = rmm_gemm_kernel<BN, BMODE, EPI, CAUSAL>;
@@ -242,12 +251,31 @@ rmm_status pack_columns(const uint16_t* A, int64_t n, int64_t d, int64_t lda, co
   return launch_pack(pk, s);
 }
 
-// S4 of the linear path: Y = A_pack[:, :k] . B[I, :] with B rows gathered by TMA.
-rmm_status gather_gemm(const uint16_t* apack, int64_t n, int64_t k, int64_t ld_pack, const uint16_t* B, int64_t d,
-                       int64_t m, int64_t ldb, const int32_t* idx, uint16_t* Y, int64_t ldy, cudaStream_t s) {
+// B_pack[t, :] = B[I[t], :] (row stride ld_pack, a multiple of 8).
+rmm_status gather_rows(const uint16_t* B, int64_t m, int64_t ldb, const int32_t* idx, int64_t k, uint16_t* bpack,
+                       int64_t ld_pack, cudaStream_t s) {
+  RowPackParams rp{};
+  rp.src = B;
+  rp.src_ld = ldb;
+  rp.cols = m;
+  rp.idx = idx;
+  rp.k = k;
+  rp.rows_out = k;
+  rp.dst = bpack;
+  rp.dst_ld = ld_pack;
+  rp.batch = 1;
+  rp.g_outer = 1;
+  rp.g_inner = 1;
+  return launch_rowpack(rp, s);
+}
+
+// Dense tensor-core product Y = A[:, :k] . B[:k, :], A K-major [n][lda], B
+// MN-major [k][ldb] (rows past k and columns past the extents read as zero).
+rmm_status gemm_packed(const uint16_t* A, int64_t n, int64_t k, int64_t lda, const uint16_t* B, int64_t m, int64_t ldb,
+                       uint16_t* Y, int64_t ldy, cudaStream_t s) {
   CUtensorMap ta, tb;
-  if (rmm_status st = make_tmap(&ta, apack, ld_pack, n, ld_pack * 2, 64, 128)) return st;
-  if (rmm_status st = make_tmap(&tb, B, m, d, ldb * 2, 64, 1)) return st;
+  if (rmm_status st = make_tmap(&ta, A, k, n, lda * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tb, B, m, k, ldb * 2, 64, 64)) return st;
   GemmParams g = gemm_defaults();
   g.M = static_cast<int>(n);
   g.N = static_cast<int>(m);
@@ -257,9 +285,7 @@ rmm_status gather_gemm(const uint16_t* apack, int64_t n, int64_t k, int64_t ld_p
   g.n_tiles = static_cast<int>(ceil_div(m, 256));
   g.k = static_cast<int>(k);
   g.num_kb = static_cast<int>(ceil_div(k, 64));
-  g.idx = idx;
-  g.b_oob_row = static_cast<int>(d);
-  return launch_gemm<256, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  return launch_gemm<256, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
 }
 
 }  // namespace
@@ -346,7 +372,6 @@ rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, in
 
 // ---------------------------------------------------------------- linear
 size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
-  (void)m;
   const int64_t k = rmm_k(rho, d);
   if (k < 0 || n < 1) return 0;
   if (k == d) return 0;
@@ -354,6 +379,7 @@ size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
   c.take<double>(d);
   c.take<int32_t>(k);
   c.take<uint16_t>(n * round_up(k, 8));
+  c.take<uint16_t>(k * round_up(m, 8));
   return c.bytes();
 }
 
@@ -371,42 +397,33 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
     return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
   const int64_t k = rmm_k(rho, d);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  GemmParams g = gemm_defaults();
-  g.M = static_cast<int>(n);
-  g.N = static_cast<int>(m);
-  g.out = Y;
-  g.ldo = ldy;
-  g.m_tiles = static_cast<int>(ceil_div(n, 128));
-  g.n_tiles = static_cast<int>(ceil_div(m, 256));
-  CUtensorMap ta, tb;
   if (k == d) {
     // rho = 1: the dense product, I = [0, d)
-    if (rmm_status st = make_tmap(&ta, A, d, n, lda * 2, 64, 128)) return st;
-    if (rmm_status st = make_tmap(&tb, B, m, d, ldb * 2, 64, 64)) return st;
-    g.k = static_cast<int>(d);
-    g.num_kb = static_cast<int>(ceil_div(d, 64));
     if (idx_out != nullptr) {
       iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024)), 256, 0, s>>>(idx_out, 1, d);
       const cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail(e, "iota launch");
     }
-    return launch_gemm<256, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
+    return gemm_packed(A, n, d, lda, B, m, ldb, Y, ldy, s);
   }
   if (d > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "d > %lld", static_cast<long long>(kMaxSelectD));
   const size_t need = rmm_linear_workspace_bytes(n, d, m, rho);
   if (ws == nullptr || ws_bytes < need)
     return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
   const int64_t k_pad = round_up(k, 8);
+  const int64_t m_pad = round_up(m, 8);
   Carver c(ws);
   double* colsq = c.take<double>(d);
   int32_t* idx_ws = c.take<int32_t>(k);
   uint16_t* apack = c.take<uint16_t>(n * k_pad);
+  uint16_t* bpack = c.take<uint16_t>(k * m_pad);
   int32_t* idx = idx_out ? idx_out : idx_ws;
 
   if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
   if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
   if (rmm_status st = pack_columns(A, n, d, lda, idx, k, apack, k_pad, s)) return st;
-  return gather_gemm(apack, n, k, k_pad, B, d, m, ldb, idx, Y, ldy, s);
+  if (rmm_status st = gather_rows(B, m, ldb, idx, k, bpack, m_pad, s)) return st;
+  return gemm_packed(apack, n, k, k_pad, bpack, m, m_pad, Y, ldy, s);
 }
 
 rmm_status rmm_gather_columns(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int32_t* idx, int64_t k,
@@ -421,16 +438,27 @@ rmm_status rmm_gather_columns(const rmm_bf16* A, int64_t n, int64_t d, int64_t l
   return pack_columns(A, n, d, lda, idx, k, A_pack, ld_pack, static_cast<cudaStream_t>(stream));
 }
 
-rmm_status rmm_gather_gemm(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t ld_pack, const rmm_bf16* B, int64_t d,
-                           int64_t m, int64_t ldb, const int32_t* idx, rmm_bf16* Y, int64_t ldy, rmm_stream stream) {
+rmm_status rmm_gather_rows(const rmm_bf16* B, int64_t d, int64_t m, int64_t ldb, const int32_t* idx, int64_t k,
+                           rmm_bf16* B_pack, int64_t ld_pack, rmm_stream stream) {
   t_last_error.clear();
-  if (A_pack == nullptr || B == nullptr || idx == nullptr || Y == nullptr) return fail(RMM_ERR_INVALID_ARG, "null pointer");
-  if (n < 1 || k < 1 || d < k || m < 1 || ld_pack < k || ldb < m || ldy < m)
-    return fail(RMM_ERR_INVALID_ARG, "need n, m >= 1, 1 <= k <= d, ld_pack >= k, ldb and ldy >= m");
-  if (!aligned16(A_pack) || !aligned16(B) || !aligned16(Y) || (ld_pack % 8) || (ldb % 8) || (ldy % 8))
+  if (B == nullptr || idx == nullptr || B_pack == nullptr) return fail(RMM_ERR_INVALID_ARG, "null pointer");
+  if (d < 1 || m < 1 || k < 1 || k > d || ldb < m || ld_pack < m)
+    return fail(RMM_ERR_INVALID_ARG, "need d, m >= 1, 1 <= k <= d, ldb and ld_pack >= m");
+  if (!aligned16(B) || !aligned16(B_pack) || (ldb % 8) || (ld_pack % 8))
     return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
-  if (n > kIntMax - 128 || m > kIntMax - 256 || d > kIntMax - 64) return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
-  return gather_gemm(A_pack, n, k, ld_pack, B, d, m, ldb, idx, Y, ldy, static_cast<cudaStream_t>(stream));
+  return gather_rows(B, m, ldb, idx, k, B_pack, ld_pack, static_cast<cudaStream_t>(stream));
+}
+
+rmm_status rmm_gemm_packed(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t lda, const rmm_bf16* B_pack,
+                           int64_t m, int64_t ldb, rmm_bf16* Y, int64_t ldy, rmm_stream stream) {
+  t_last_error.clear();
+  if (A_pack == nullptr || B_pack == nullptr || Y == nullptr) return fail(RMM_ERR_INVALID_ARG, "null pointer");
+  if (n < 1 || k < 1 || m < 1 || lda < k || ldb < m || ldy < m)
+    return fail(RMM_ERR_INVALID_ARG, "need n, k, m >= 1, lda >= k, ldb and ldy >= m");
+  if (!aligned16(A_pack) || !aligned16(B_pack) || !aligned16(Y) || (lda % 8) || (ldb % 8) || (ldy % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
+  if (n > kIntMax - 128 || m > kIntMax - 256 || k > kIntMax - 64) return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  return gemm_packed(A_pack, n, k, lda, B_pack, m, ldb, Y, ldy, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- QK^T
@@ -550,7 +578,6 @@ rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch,
 // ---------------------------------------------------------------- PV
 size_t rmm_pv_workspace_bytes(int64_t batch, int64_t h, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, double rho) {
   (void)hkv;
-  (void)dh;
   const int64_t k = rmm_k(rho, nk);
   if (k < 0 || batch < 1 || h < 1 || nq < 1) return 0;
   if (k == nk) return 0;
@@ -559,6 +586,7 @@ size_t rmm_pv_workspace_bytes(int64_t batch, int64_t h, int64_t hkv, int64_t nq,
   c.take<double>(items * nk);
   c.take<int32_t>(items * k);
   c.take<uint16_t>(items * nq * round_up(k, 8));
+  c.take<uint16_t>(items * round_up(k, 64) * dh);
   return c.bytes();
 }
 
@@ -596,7 +624,6 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
   g.b_g_inner = static_cast<int>(h / hkv);
   g.b_s_outer = hkv * nk;
   g.b_s_inner = nk;
-  g.b_oob_row = static_cast<int>(batch * hkv * nk);
   CUtensorMap ta, tb;
   const bool dense = (k == nk);
   if (dense) {
@@ -620,6 +647,8 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
     double* colsq = c.take<double>(items * nk);
     int32_t* idx_ws = c.take<int32_t>(items * k);
     uint16_t* ppack = c.take<uint16_t>(items * nq * k_pad);
+    const int64_t k_rows = round_up(k, 64);
+    uint16_t* vpack = c.take<uint16_t>(items * k_rows * dh);
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if (rmm_status st = launch_colsq(P, items, nq * nk, nq, nk, nk, causal != 0, off, colsq, s)) return st;
     if (rmm_status st = launch_select(colsq, items, nk, k, idx, nullptr, s)) return st;
@@ -639,25 +668,38 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
     pp.causal = causal;
     pp.causal_off = off;
     if (rmm_status st = launch_pack(pp, s)) return st;
+    // V_pack[b][t, :] = V_g(b)[I_b[t], :], zero rows up to a multiple of 64
+    RowPackParams rp{};
+    rp.src = V;
+    rp.src_ld = dh;
+    rp.cols = dh;
+    rp.idx = idx;
+    rp.k = k;
+    rp.rows_out = k_rows;
+    rp.dst = vpack;
+    rp.dst_ld = dh;
+    rp.batch = items;
+    rp.g_outer = h;
+    rp.g_inner = h / hkv;
+    rp.s_outer = hkv * nk * dh;
+    rp.s_inner = nk * dh;
+    if (rmm_status st = launch_rowpack(rp, s)) return st;
     if (rmm_status st = make_tmap(&ta, ppack, k_pad, items * nq, k_pad * 2, 64, 128)) return st;
-    if (rmm_status st = make_tmap(&tb, V, dh, batch * hkv * nk, dh * 2, 64, 1)) return st;
+    if (rmm_status st = make_tmap(&tb, vpack, dh, items * k_rows, dh * 2, 64, 64)) return st;
     g.k = static_cast<int>(k);
     g.num_kb = static_cast<int>(ceil_div(k, 64));
     g.idx = idx;
     g.idx_bstride = k;
+    g.b_g_outer = 1;
+    g.b_g_inner = 1;
+    g.b_s_outer = k_rows;
+    g.b_s_inner = 0;
   }
-  if (dh == 128) {
-    if (dense)
-      return causal ? launch_gemm<128, kBTileMN, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
-                    : launch_gemm<128, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
-    return causal ? launch_gemm<128, kBGather, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
-                  : launch_gemm<128, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
-  }
-  if (dense)
-    return causal ? launch_gemm<64, kBTileMN, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
-                  : launch_gemm<64, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
-  return causal ? launch_gemm<64, kBGather, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
-                : launch_gemm<64, kBGather, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  if (dh == 128)
+    return causal ? launch_gemm<128, kBTileMN, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
+                  : launch_gemm<128, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
+  return causal ? launch_gemm<64, kBTileMN, kEpiBf16, kCausalLimitK>(ta, tb, g, s)
+                : launch_gemm<64, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
 }
 
 }  // extern "C"

@@ -116,7 +116,8 @@ def test_linear_llama8b_prefill_sampled(name, rho):
 
 
 def test_stage_entry_points_compose_to_rmm_linear():
-    """rmm_select -> rmm_gather_columns -> rmm_gather_gemm gives the same bits as rmm_linear."""
+    """rmm_select -> rmm_gather_columns -> rmm_gather_rows -> rmm_gemm_packed gives
+    the same bits as rmm_linear."""
     g = synthetic.rng(31)
     A = synthetic.to_bf16(synthetic.outlier_activations(g, 300, 1000, 1.5)).cuda()
     B = synthetic.to_bf16(synthetic.gaussian_weight(g, 1000, 520)).cuda()
@@ -124,10 +125,13 @@ def test_stage_entry_points_compose_to_rmm_linear():
     idx2, _, _ = rmm.select(A, 0.7)
     k = idx2.numel()
     ap = rmm.gather_columns(A, idx2, ld_pack=712)
-    Y2 = rmm.gather_gemm(ap, k, B, idx2)
+    bp = rmm.gather_rows(B, idx2, ld_pack=528)
+    Y2 = rmm.gemm_packed(ap, k, bp, 520)
     torch.cuda.synchronize()
     assert torch.equal(idx, idx2)
     assert torch.equal(Y, Y2)
+    I = idx2.cpu().long()
     expect = torch.zeros((300, 712), dtype=torch.bfloat16)
-    expect[:, :k] = A.cpu()[:, idx2.cpu().long()]
+    expect[:, :k] = A.cpu()[:, I]
     assert torch.equal(ap.cpu(), expect)
+    assert torch.equal(bp.cpu()[:, :520], B.cpu()[I, :])
