@@ -87,6 +87,32 @@ rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, in
                       int causal, double rho, int32_t* idx_out, double* colsq_out, double* retained_out, void* ws,
                       size_t ws_bytes, rmm_stream stream);
 
+/* rmm_select_noalloc: rmm_select for callers that cannot allocate device memory.
+ * This entry point has no counterpart on the pages; it exists for hosts whose
+ * device memory is owned by someone else (a framework allocator or a fixed
+ * memory budget reserved up front) and for latency-critical paths where a
+ * cudaMalloc/cudaFree, which may synchronise the device, is not acceptable.
+ * It computes exactly what rmm_select computes (same kernels, same results)
+ * but takes no workspace and returns no scores: the fp64 column scores live in
+ * one fixed scratch array inside the library, RMM_SELECT_NOALLOC_MAX_SCORES
+ * doubles (2 MiB) that every device which loads the library keeps until the
+ * process exits.  Nothing is allocated by this call.
+ *   - batch * d must not exceed RMM_SELECT_NOALLOC_MAX_SCORES; larger problems
+ *     return RMM_ERR_UNSUPPORTED with a message naming the limit.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that
+ *     first call before any stream capture on the device.
+ *   - Every call on a device shares the one array.  Calls whose kernels can
+ *     overlap on the GPU (different streams without ordering between them)
+ *     race on it and give undefined results; order them on one stream or with
+ *     events.  The array keeps the last call's scores, and each call rewrites
+ *     all batch * d scores it uses before reading them.
+ * Arguments, layouts and error behaviour are those of rmm_select. */
+#define RMM_SELECT_NOALLOC_MAX_SCORES 262144
+rmm_status rmm_select_noalloc(const rmm_bf16* A, int64_t batch, int64_t batch_stride, int64_t n, int64_t d,
+                              int64_t lda, int causal, double rho, int32_t* idx_out, double* retained_out,
+                              rmm_stream stream);
+
 /* ---------------------------------------------------------------- linear
  * rmm_linear: Y = A[:, I] . B[I, :] with I selected on A (linear and MLP
  * projections X.W reduce the activation hidden dim: "Core Approach",

@@ -370,6 +370,68 @@ rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, in
   return launch_select(colsq, batch, d, k, idx_out, retained_out, s);
 }
 
+// ---------------------------------------------------------------- selection without allocation
+// For callers that may not allocate device memory at all: the fp64 column
+// scores that rmm_select keeps in the caller's workspace live instead in one
+// fixed array inside the library.  Every device that loads the library holds
+// this array (2 MiB) until the process exits.
+}  // extern "C"
+
+namespace {
+constexpr int64_t kNoAllocScores = 262144;  // equals RMM_SELECT_NOALLOC_MAX_SCORES in rmm.h
+static __device__ __align__(256) double g_noalloc_scores[kNoAllocScores];
+
+// Device address of g_noalloc_scores for the current device.  In host code the
+// array's name only stands for the symbol, so the address is looked up once per
+// device with cudaGetSymbolAddress and cached.
+rmm_status noalloc_scores(double** out) {
+  static std::mutex mu;
+  static double* cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(RMM_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scores);
+    if (e != cudaSuccess || ptr == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(score scratch)");
+    cached[dev] = static_cast<double*>(ptr);
+  }
+  *out = cached[dev];
+  return RMM_OK;
+}
+}  // namespace
+
+extern "C" {
+
+rmm_status rmm_select_noalloc(const rmm_bf16* A, int64_t batch, int64_t batch_stride, int64_t n, int64_t d,
+                              int64_t lda, int causal, double rho, int32_t* idx_out, double* retained_out,
+                              rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (A == nullptr || idx_out == nullptr) return fail(RMM_ERR_INVALID_ARG, "A and idx_out are required");
+  if (batch < 1 || n < 1 || d < 1) return fail(RMM_ERR_INVALID_ARG, "batch, n and d must be >= 1");
+  if (lda < d) return fail(RMM_ERR_INVALID_ARG, "lda < d");
+  if (batch > 1 && batch_stride < (n - 1) * lda + d) return fail(RMM_ERR_INVALID_ARG, "batch_stride too small");
+  if (causal != 0 && causal != 1) return fail(RMM_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (d > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "d > %lld", static_cast<long long>(kMaxSelectD));
+  if (batch * d > kNoAllocScores)
+    return fail(RMM_ERR_UNSUPPORTED,
+                "rmm_select_noalloc holds at most %lld scores (batch * d); got %lld -- use rmm_select with a workspace",
+                static_cast<long long>(kNoAllocScores), static_cast<long long>(batch * d));
+  if (n > kIntMax || batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "n or batch too large");
+  if (!aligned16(A) || (lda % 8) != 0 || (batch > 1 && (batch_stride % 8) != 0))
+    return fail(RMM_ERR_UNSUPPORTED, "A must be 16-byte aligned with lda and batch_stride multiples of 8");
+  double* colsq = nullptr;
+  if (rmm_status st = noalloc_scores(&colsq)) return st;
+  // every score of [0, batch * d) is rewritten below, so nothing needs clearing
+  const int64_t k = rmm_k(rho, d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rmm_status st = launch_colsq(A, batch, batch_stride, n, d, lda, causal != 0, d - n, colsq, s)) return st;
+  return launch_select(colsq, batch, d, k, idx_out, retained_out, s);
+}
+
 // ---------------------------------------------------------------- linear
 size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
   const int64_t k = rmm_k(rho, d);
