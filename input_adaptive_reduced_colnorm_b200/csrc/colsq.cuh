@@ -57,10 +57,12 @@ __global__ void __launch_bounds__(256) colsq_kernel(const ColsqParams p) {
 
   if (col0 < p.d) {
     const bool full = (col0 + 8 <= p.d);
-    for (int64_t i = r_begin + ty; i < r_end; i += 4 * TY) {
-      uint32_t w[4][4];
+    // bursts of U rows: all U 16-byte loads are in flight before any is used
+    constexpr int U = 8;
+    for (int64_t i = r_begin + ty; i < r_end; i += U * TY) {
+      uint32_t w[U][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int64_t row = i + u * TY;
         w[u][0] = w[u][1] = w[u][2] = w[u][3] = 0u;
         if (row < r_end) {
@@ -74,21 +76,25 @@ __global__ void __launch_bounds__(256) colsq_kernel(const ColsqParams p) {
           }
         }
       }
-      float a32[8];
+      // four rows at a time in fp32 (bf16 squares are exact in fp32), then fp64
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a32[e] = 0.f;
+      for (int g = 0; g < U; g += 4) {
+        float a32[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t lim = CAUSAL ? (i + u * TY + p.causal_off) : 0;
+        for (int e = 0; e < 8; ++e) a32[e] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float x = (e & 1) ? bf16hi(w[u][e >> 1]) : bf16lo(w[u][e >> 1]);
-          if (CAUSAL && col0 + e > lim) x = 0.f;
-          a32[e] = fmaf(x, x, a32[e]);
+        for (int u = g; u < g + 4; ++u) {
+          const int64_t lim = CAUSAL ? (i + u * TY + p.causal_off) : 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float x = (e & 1) ? bf16hi(w[u][e >> 1]) : bf16lo(w[u][e >> 1]);
+            if (CAUSAL && col0 + e > lim) x = 0.f;
+            a32[e] = fmaf(x, x, a32[e]);
+          }
         }
-      }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
+        for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
+      }
     }
   }
 

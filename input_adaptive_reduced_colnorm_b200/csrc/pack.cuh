@@ -6,7 +6,9 @@
 // A column gather of a row-major matrix touches nearly every 32-byte sector of
 // a row, so each row is first staged in shared memory with coalesced 16-byte
 // loads and the gather runs out of shared memory; writes are 16-byte vectors.
-// Rows of at most 1024 columns are handled one per warp; longer rows one per CTA.
+// Rows of at most 1024 columns are handled one per warp; longer rows one per
+// CTA, with the next row's cp.async copy in flight while the current row is
+// gathered and the index set held in shared memory as 16-bit offsets.
 // With ``causal`` the entry (i, t) is kept only if I[t] <= i + causal_off (the
 // masked upper triangle of an attention-probability matrix reads as zero), and
 // only the visible prefix of the row is read.
@@ -97,31 +99,84 @@ __global__ void __launch_bounds__(256) pack_rows_warp_kernel(const PackParams p,
   }
 }
 
-// one row per CTA; dynamic shared memory: d_round bf16
-__global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p) {
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ int64_t pack_visible(const PackParams& p, int64_t i) {
+  if (!p.causal) return p.d;
+  int64_t lim = i + p.causal_off + 1;
+  return lim > p.d ? p.d : (lim < 0 ? 0 : lim);
+}
+
+// async copy of the first `lim` columns of one row into shared memory
+__device__ __forceinline__ void pack_stage_async(uint16_t* buf, const uint16_t* src, int64_t lim, int64_t d) {
+  const int64_t nvec = (lim + 7) / 8;
+  for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+    const int64_t c = v * 8;
+    const int64_t rem = d - c;
+    cp_async16_zfill(buf + c, src + c, rem >= 8 ? 16u : static_cast<uint32_t>(rem * 2));
+  }
+}
+
+// Contiguous row range per CTA, double-buffered rows.  Dynamic shared memory:
+// 16-bit index offsets [k_pad] (0xFFFF marks padding) + two row buffers [d_round].
+__global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, int64_t d_round, int64_t idx_elems) {
   extern __shared__ __align__(16) uint16_t pk_smem[];
+  uint16_t* s_idx = pk_smem;
+  uint16_t* bufs[2] = {pk_smem + idx_elems, pk_smem + idx_elems + d_round};
   const int64_t total = p.batch * p.rows;
-  for (int64_t r = blockIdx.x; r < total; r += gridDim.x) {
-    int64_t b, i;
-    const uint16_t* src = pack_src_row(p, r, b, i);
-    int64_t lim = p.d;
-    if (p.causal) {
-      lim = i + p.causal_off + 1;
-      if (lim > p.d) lim = p.d;
-      if (lim < 0) lim = 0;
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * per;
+  int64_t r_end = r_begin + per;
+  if (r_end > total) r_end = total;
+  if (r_begin >= r_end) return;
+
+  int64_t b, i;
+  const uint16_t* src = pack_src_row(p, r_begin, b, i);
+  pack_stage_async(bufs[0], src, pack_visible(p, i), p.d);
+  cp_async_commit();
+  int64_t cur_b = -1;
+  for (int64_t r = r_begin; r < r_end; ++r) {
+    const int64_t rb = r / p.rows;
+    const int64_t ri = r - rb * p.rows;
+    if (r + 1 < r_end) {
+      int64_t nb, ni;
+      const uint16_t* nsrc = pack_src_row(p, r + 1, nb, ni);
+      pack_stage_async(bufs[(r + 1 - r_begin) & 1], nsrc, pack_visible(p, ni), p.d);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    pack_stage(pk_smem, src, lim, p.d, threadIdx.x, 256);
+    if (rb != cur_b) {  // (re)load this batch item's index set as 16-bit offsets
+      const int32_t* I = p.idx + rb * p.k;
+      for (int64_t t = threadIdx.x; t < p.k_pad; t += blockDim.x)
+        s_idx[t] = (t < p.k) ? static_cast<uint16_t>(__ldg(I + t)) : uint16_t(0xFFFF);
+      cur_b = rb;
+    }
     __syncthreads();
-    const int32_t* idx = p.idx + b * p.k;
+    const uint16_t* row = bufs[(r - r_begin) & 1];
+    const int64_t lim = pack_visible(p, ri);
     uint16_t* dst = p.dst + r * p.k_pad;
-    for (int64_t t0 = static_cast<int64_t>(threadIdx.x) * 8; t0 < p.k_pad; t0 += 2048) {
-      const uint4 v = pack_gather8(p, pk_smem, idx, t0, lim);
-      if (t0 + 8 <= p.k_pad) {
-        *reinterpret_cast<uint4*>(dst + t0) = v;
-      } else {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        for (int e = 0; t0 + e < p.k_pad; ++e) dst[t0 + e] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+    for (int64_t t0 = static_cast<int64_t>(threadIdx.x) * 8; t0 < p.k_pad; t0 += 8 * blockDim.x) {
+      const uint4 iv = *reinterpret_cast<const uint4*>(s_idx + t0);
+      const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const uint32_t j0 = iw[h] & 0xFFFFu, j1 = iw[h] >> 16;
+        const uint32_t v0 = (j0 < lim) ? row[j0] : 0u;   // 0xFFFF padding is never < lim (d <= 32768)
+        const uint32_t v1 = (j1 < lim) ? row[j1] : 0u;
+        w[h] = v0 | (v1 << 16);
       }
+      *reinterpret_cast<uint4*>(dst + t0) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     __syncthreads();
   }
@@ -145,42 +200,46 @@ struct RowPackParams {
   int64_t g_outer, g_inner, s_outer, s_inner; // source item of b (as in PackParams)
 };
 
-__global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackParams p) {
-  constexpr int ILP = 4;
-  const int64_t vpr = (p.cols + 7) / 8;  // 16-byte vectors per row
-  const int64_t total = p.batch * p.rows_out * vpr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v0 < total; v0 += ILP * stride) {
-    uint4 val[ILP];
-    int64_t out_off[ILP];
+// 2-D layout: 2^tpr_log2 threads per output row, 256 >> tpr_log2 rows per CTA;
+// each thread copies every (2^tpr_log2)-th 16-byte vector of its row.
+__global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackParams p, int tpr_log2) {
+  constexpr int ILP = 8;
+  const int tpr = 1 << tpr_log2;
+  const int tx = threadIdx.x & (tpr - 1);
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (256 >> tpr_log2) + (threadIdx.x >> tpr_log2);
+  if (row >= p.batch * p.rows_out) return;
+  const int64_t b = row / p.rows_out;
+  const int64_t t = row - b * p.rows_out;
+  uint16_t* dst = p.dst + row * p.dst_ld;
+  const int vpr = static_cast<int>((p.cols + 7) / 8);
+  const uint16_t* src = nullptr;
+  if (t < p.k) {
+    const int64_t j = __ldg(p.idx + b * p.k + t);
+    const int64_t item = (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+    src = p.src + item + j * p.src_ld;
+  }
+  const bool full_tail = (p.cols % 8) == 0;
+  for (int c0 = tx; c0 < vpr; c0 += tpr * ILP) {
+    uint4 v[ILP];
 #pragma unroll
     for (int u = 0; u < ILP; ++u) {
-      const int64_t v = v0 + u * stride;
-      val[u] = make_uint4(0u, 0u, 0u, 0u);
-      out_off[u] = -1;
-      if (v < total) {
-        const int64_t row = v / vpr;
-        const int64_t c = v - row * vpr;
-        const int64_t b = row / p.rows_out;
-        const int64_t t = row - b * p.rows_out;
-        out_off[u] = row * p.dst_ld + c * 8;
-        if (t < p.k) {
-          const int64_t j = __ldg(p.idx + b * p.k + t);
-          const int64_t item = (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
-          const uint16_t* src = p.src + item + j * p.src_ld + c * 8;
-          if (c * 8 + 8 <= p.cols) {
-            val[u] = ldg_nc_v4(src);
-          } else {
-            uint32_t w[4] = {0u, 0u, 0u, 0u};
-            for (int e = 0; c * 8 + e < p.cols; ++e) w[e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
-            val[u] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+      const int c = c0 + u * tpr;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (src != nullptr && c < vpr) {
+        if (full_tail || c + 1 < vpr) {
+          v[u] = ldg_nc_v4(src + c * 8);
+        } else {
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
+          for (int e = 0; c * 8 + e < p.cols; ++e) w[e >> 1] |= static_cast<uint32_t>(__ldg(src + c * 8 + e)) << (16 * (e & 1));
+          v[u] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < ILP; ++u)
-      if (out_off[u] >= 0) *reinterpret_cast<uint4*>(p.dst + out_off[u]) = val[u];
+    for (int u = 0; u < ILP; ++u) {
+      const int c = c0 + u * tpr;
+      if (c < vpr) *reinterpret_cast<uint4*>(dst + c * 8) = v[u];
+    }
   }
 }
 

@@ -153,40 +153,51 @@ rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64
   return RMM_OK;
 }
 
-rmm_status launch_select(const double* colsq, int64_t batch, int64_t d, int64_t k, int32_t* idx, double* retained,
-                         cudaStream_t s) {
-  SelectParams p{colsq, d, k, idx, retained};
-  const unsigned g = static_cast<unsigned>(batch);
-  if (d <= 128) select_kernel<1, 128><<<g, 128, 0, s>>>(p);
-  else if (d <= 1024) select_kernel<1, 1024><<<g, 1024, 0, s>>>(p);
-  else if (d <= 2048) select_kernel<2, 1024><<<g, 1024, 0, s>>>(p);
-  else if (d <= 4096) select_kernel<4, 1024><<<g, 1024, 0, s>>>(p);
-  else if (d <= 8192) select_kernel<8, 1024><<<g, 1024, 0, s>>>(p);
-  else if (d <= 16384) select_kernel<16, 1024><<<g, 1024, 0, s>>>(p);
-  else select_kernel<32, 1024><<<g, 1024, 0, s>>>(p);
+template <int KPT, int NT>
+rmm_status launch_select_t(const SelectParams& p, int64_t batch, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(NT) * KPT * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "select attribute");
+  }
+  select_kernel<KPT, NT><<<static_cast<unsigned>(batch), NT, smem, s>>>(p);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   return RMM_OK;
 }
 
+rmm_status launch_select(const double* colsq, int64_t batch, int64_t d, int64_t k, int32_t* idx, double* retained,
+                         cudaStream_t s) {
+  SelectParams p{colsq, d, k, idx, retained};
+  if (d <= 128) return launch_select_t<1, 128>(p, batch, s);
+  if (d <= 1024) return launch_select_t<1, 1024>(p, batch, s);
+  if (d <= 2048) return launch_select_t<2, 1024>(p, batch, s);
+  if (d <= 4096) return launch_select_t<4, 1024>(p, batch, s);
+  if (d <= 8192) return launch_select_t<8, 1024>(p, batch, s);
+  if (d <= 16384) return launch_select_t<16, 1024>(p, batch, s);
+  return launch_select_t<32, 1024>(p, batch, s);
+}
+
 rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
   const int64_t rows = p.batch * p.rows;
   const int64_t d_round = round_up(p.d, 8);
-  const int64_t cap = 8LL * num_sms();
   cudaError_t e;
   if (p.d <= 1024) {
     const size_t smem = static_cast<size_t>(8 * d_round * 2);
-    const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), cap);
+    const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), 8LL * num_sms());
     pack_rows_warp_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round);
   } else {
-    const size_t smem = static_cast<size_t>(d_round * 2);
+    const int64_t idx_elems = round_up(p.k_pad, 8);
+    const size_t smem = static_cast<size_t>((idx_elems + 2 * d_round) * 2);
     if (smem > 48 * 1024) {
       e = cudaFuncSetAttribute(pack_rows_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
       if (e != cudaSuccess) return cuda_fail(e, "pack attribute");
     }
-    const int64_t grid = std::min<int64_t>(rows, cap);
-    pack_rows_cta_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p);
+    const int64_t per_sm = std::max<int64_t>(1, std::min<int64_t>(8, (200 * 1024) / static_cast<int64_t>(smem)));
+    const int64_t grid = std::min<int64_t>(rows, per_sm * num_sms());
+    pack_rows_cta_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round, idx_elems);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
@@ -194,9 +205,13 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
 }
 
 rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
-  const int64_t total = p.batch * p.rows_out * ((p.cols + 7) / 8);
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256 * 4), 8LL * num_sms()));
-  pack_rows_gather_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p);
+  const int64_t vpr = (p.cols + 7) / 8;
+  int tpr_log2 = 0;
+  while ((1LL << tpr_log2) < vpr && tpr_log2 < 8) ++tpr_log2;
+  const int64_t rows = p.batch * p.rows_out;
+  const int64_t grid = ceil_div(rows, 256 >> tpr_log2);
+  if (grid > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "row pack grid too large");
+  pack_rows_gather_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p, tpr_log2);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "row pack launch");
   return RMM_OK;

@@ -3,16 +3,20 @@
 // Approach: keep the TopK-largest ceil(rho d); tie rule and order are readings).
 //
 // One CTA per selection row.  Keys are the fp64 sums of squares q_j; for
-// non-negative doubles the IEEE bit pattern orders like the value, so the
-// k-th largest key is found by an MSB-first radix select on the 64-bit
-// pattern, 8 bits per pass.  The top 32 bits of every key live in registers
-// (thread t owns the contiguous indices [t*KPT, (t+1)*KPT)); the low 32 bits
-// are fetched from global memory only for keys that still tie on the top 32
-// bits, which happens only for (near-)exact ties.  A pass stops early as soon
-// as the bucket holding the k-th key is taken whole.  The final compaction is
-// two block-wide prefix scans in index order, which yields the lower-index tie
-// rule and the ascending order without any sort.  All counts are integers, so
-// the result does not depend on atomic ordering.
+// non-negative doubles the IEEE bit pattern orders like the value, so the k-th
+// largest key is found by an MSB-first radix select on the 64-bit pattern:
+//   * the top 32 bits of every key are staged in shared memory with coalesced
+//     loads (thread t then owns the contiguous indices [t*KPT, (t+1)*KPT) and
+//     keeps them in registers);
+//   * leading bits shared by all keys are skipped (block-wide AND/OR), and each
+//     pass resolves the next 12 bits with one 4096-bin shared histogram;
+//   * the low 32 bits are fetched from global memory only for keys that still
+//     tie on the top 32 bits (exact or near-exact ties);
+//   * a pass stops early as soon as the bucket holding the k-th key is taken
+//     whole.
+// The final compaction is two block-wide prefix scans in index order, which
+// gives the lower-index tie rule and the ascending order without any sort.
+// All counts are integers, so the result does not depend on atomic ordering.
 #pragma once
 #include "ptx.cuh"
 
@@ -25,6 +29,9 @@ struct SelectParams {
   int32_t* idx;         // [batch][k]
   double* retained;     // [batch] or nullptr: sum_{j in I} q_j / sum_j q_j
 };
+
+constexpr int kSelBits = 12;
+constexpr int kSelBins = 1 << kSelBits;
 
 template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* s_total) {
@@ -69,106 +76,140 @@ __device__ __forceinline__ double block_sum_f64(double v, double* s_buf) {
   return t;  // valid in thread 0 only
 }
 
+// dynamic shared memory: hi32 keys [NT * KPT] (uint32)
 template <int KPT, int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   constexpr int NW = NT / 32;
-  __shared__ uint32_t whist[NW][256];
-  __shared__ uint32_t hist[256];
-  __shared__ int s_digit, s_above, s_cnt;
+  constexpr int BPT = kSelBins / NT;  // histogram bins scanned per thread
+  static_assert(kSelBins % NT == 0, "bins must split evenly");
+  extern __shared__ __align__(16) uint32_t s_keys[];
+  __shared__ uint32_t hist[kSelBins];
   __shared__ int s_warp[32];
   __shared__ int s_total;
+  __shared__ int s_digit, s_above, s_cnt;
+  __shared__ uint32_t s_and[32], s_or[32];
   __shared__ double s_sum[32];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t b = blockIdx.x;
   const double* q = p.colsq + b * p.d;
   int32_t* out = p.idx + b * p.k;
-  const int64_t j0 = static_cast<int64_t>(threadIdx.x) * KPT;
+  const int d = static_cast<int>(p.d);
+  const int j0 = threadIdx.x * KPT;
 
+  // coalesced staging of the top 32 bits of every key
+  for (int j = threadIdx.x; j < d; j += NT)
+    s_keys[j] = static_cast<uint32_t>(static_cast<uint64_t>(__double_as_longlong(q[j])) >> 32);
+  __syncthreads();
   uint32_t hi[KPT];
   uint32_t valid = 0;
+  uint32_t kand = 0xffffffffu, kor = 0u;
 #pragma unroll
   for (int e = 0; e < KPT; ++e) {
-    const int64_t j = j0 + e;
     hi[e] = 0u;
-    if (j < p.d) {
-      hi[e] = static_cast<uint32_t>(static_cast<uint64_t>(__double_as_longlong(q[j])) >> 32);
+    if (j0 + e < d) {
+      hi[e] = s_keys[j0 + e];
       valid |= 1u << e;
+      kand &= hi[e];
+      kor |= hi[e];
     }
   }
+  // bits on which all keys agree need no pass
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+  }
+  if (lane == 0) {
+    s_and[warp] = kand;
+    s_or[warp] = kor;
+  }
+  __syncthreads();
+  kand = 0xffffffffu;
+  kor = 0u;
+  for (int w = 0; w < NW; ++w) {
+    kand &= s_and[w];
+    kor |= s_or[w];
+  }
+  const uint32_t differ = kand ^ kor;  // bits not shared by every key
 
   uint32_t pre_hi = 0, msk_hi = 0, pre_lo = 0, msk_lo = 0;
   int need = static_cast<int>(p.k);
-  bool take_bucket = (p.k == p.d);  // everything is kept: nothing to rank
+  bool take_bucket = (p.k == p.d);
+  if (!take_bucket && differ == 0u) {
+    // all top-32 bits equal: decide on the low 32 bits
+    msk_hi = 0xffffffffu;
+    pre_hi = kand;
+  } else if (!take_bucket) {
+    const int top = 31 - __clz(differ);  // highest differing bit
+    msk_hi = (top == 31) ? 0u : (0xffffffffu << (top + 1));
+    pre_hi = kand & msk_hi;
+  }
+  // bit cursor: position (in the 64-bit key) just above the next digit
+  int cursor = 32 + ((msk_hi == 0xffffffffu) ? 0 : (32 - __popc(msk_hi)));
 
-  for (int pass = 0; pass < 8 && !take_bucket; ++pass) {
-    for (int i = threadIdx.x; i < NW * 256; i += NT) (&whist[0][0])[i] = 0u;
+  while (!take_bucket && cursor > 0) {
+    const int width = cursor >= kSelBits ? kSelBits : cursor;
+    const int shift = cursor - width;  // bit position of the digit in the 64-bit key
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = threadIdx.x; i < kSelBins; i += NT) hist[i] = 0u;
     __syncthreads();
-    const int shift = 24 - 8 * (pass & 3);
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
-      bool m = ((valid >> e) & 1u) && ((hi[e] & msk_hi) == pre_hi);
-      uint32_t dig = 0;
-      if (m) {
-        if (pass < 4) {
-          dig = (hi[e] >> shift) & 255u;
+      if (!((valid >> e) & 1u) || (hi[e] & msk_hi) != pre_hi) continue;
+      uint32_t dig;
+      if (shift >= 32) {
+        dig = (hi[e] >> (shift - 32)) & dmask;
+      } else {
+        const uint32_t lo = static_cast<uint32_t>(__double_as_longlong(q[j0 + e]));
+        if ((lo & msk_lo) != pre_lo) continue;
+        if (shift + width > 32) {  // digit straddles the two halves
+          const uint64_t full = (static_cast<uint64_t>(hi[e]) << 32) | lo;
+          dig = static_cast<uint32_t>(full >> shift) & dmask;
         } else {
-          const uint32_t lo = static_cast<uint32_t>(__double_as_longlong(q[j0 + e]));
-          m = (lo & msk_lo) == pre_lo;
-          dig = (lo >> shift) & 255u;
+          dig = (lo >> shift) & dmask;
         }
       }
-      const uint32_t key = m ? dig : (256u + lane);
-      const uint32_t grp = __match_any_sync(0xffffffffu, key);
-      if (m && lane == __ffs(grp) - 1) atomicAdd(&whist[warp][dig], static_cast<uint32_t>(__popc(grp)));
+      atomicAdd(&hist[dig], 1u);
     }
     __syncthreads();
-    for (int bin = threadIdx.x; bin < 256; bin += NT) {
-      uint32_t s = 0;
-      for (int w = 0; w < NW; ++w) s += whist[w][bin];
-      hist[bin] = s;
+    // descending suffix sums: bin b's "above" = count of larger digits
+    uint32_t c[BPT];
+    uint32_t ls = 0;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      c[i] = hist[threadIdx.x * BPT + i];
+      ls += c[i];
     }
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t c[8];
-      uint32_t ls = 0;
+    // exclusive scan in descending thread order: reverse the thread index
+    const int before = block_exclusive_scan<NT>(static_cast<int>(ls), s_warp, &s_total);
+    const uint32_t total = static_cast<uint32_t>(s_total);
+    uint32_t above = total - static_cast<uint32_t>(before) - ls;  // digits held by higher threads
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c[i] = hist[lane * 8 + i];
-        ls += c[i];
+    for (int i = BPT - 1; i >= 0; --i) {
+      const int bin = threadIdx.x * BPT + i;
+      if (bin <= static_cast<int>(dmask) && above < static_cast<uint32_t>(need) &&
+          static_cast<uint32_t>(need) <= above + c[i]) {
+        s_digit = bin;
+        s_above = static_cast<int>(above);
+        s_cnt = static_cast<int>(c[i]);
       }
-      // sum over lanes above this one (bins with larger digits)
-      uint32_t incl = ls;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += y;
-      }
-      uint32_t above = incl - ls;
-#pragma unroll
-      for (int i = 7; i >= 0; --i) {
-        if (above < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= above + c[i]) {
-          s_digit = lane * 8 + i;
-          s_above = static_cast<int>(above);
-          s_cnt = static_cast<int>(c[i]);
-        }
-        above += c[i];
-      }
+      above += c[i];
     }
     __syncthreads();
     need -= s_above;
-    if (pass < 4) {
-      pre_hi |= static_cast<uint32_t>(s_digit) << shift;
-      msk_hi |= 255u << shift;
-    } else {
-      pre_lo |= static_cast<uint32_t>(s_digit) << shift;
-      msk_lo |= 255u << shift;
-    }
+    const uint64_t dg = static_cast<uint64_t>(s_digit) << shift;
+    const uint64_t dm = static_cast<uint64_t>(dmask) << shift;
+    pre_hi |= static_cast<uint32_t>(dg >> 32);
+    msk_hi |= static_cast<uint32_t>(dm >> 32);
+    pre_lo |= static_cast<uint32_t>(dg);
+    msk_lo |= static_cast<uint32_t>(dm);
     if (s_cnt == need) take_bucket = true;
+    cursor = shift;
     __syncthreads();
   }
 
-  // classify the owned keys: greater than the threshold bucket, or inside it
+  // classify the owned keys: above the threshold bucket, or inside it
   uint32_t gt = 0, eq = 0;
 #pragma unroll
   for (int e = 0; e < KPT; ++e) {
@@ -203,12 +244,12 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   }
   const int pos0 = block_exclusive_scan<NT>(__popc(sel), s_warp, &s_total);
   int pos = pos0;
-  double kept = 0.0, all = 0.0;
 #pragma unroll
   for (int e = 0; e < KPT; ++e) {
-    if ((sel >> e) & 1u) out[pos++] = static_cast<int32_t>(j0 + e);
+    if ((sel >> e) & 1u) out[pos++] = j0 + e;
   }
   if (p.retained != nullptr) {
+    double kept = 0.0, all = 0.0;
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
       if ((valid >> e) & 1u) {
