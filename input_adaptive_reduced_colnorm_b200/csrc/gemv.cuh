@@ -1,0 +1,295 @@
+// Decode-shaped reduced product (n <= 32 activation rows):
+//   Y[n x m] = x[:, I] . W[I, :]        ("Algorithm Deep-Dive: RMM", Core
+//   Approach, applied to a linear projection at decode time)
+// It is bound by HBM reads of the k kept weight rows (k * m * 2 bytes), so only
+// those rows are read, once, straight from W -- no packed copy of W[I, :].
+//
+// Tensor cores with the operands swapped: D[128 weight columns x N rows] =
+// W_I^T (M = 128, MN-major) . x_I^T (N = 16 or 32, K-major), fp32 accumulator
+// in tensor memory.
+//   warps 0-3  producers: every kept-row segment (128 columns = 256 bytes) is
+//              loaded with 16-byte cp.async straight into the 128-byte-swizzled
+//              MN-major operand layout (a TMA row gather stages only ~7 B/clk/SM
+//              on B200, 16-byte cp.async ~35 B/clk/SM; HBM speed needs ~22);
+//              thread 0 also brings the packed activations x_I with a TMA tile.
+//   warp 4     allocates TMEM; one thread issues tcgen05.mma (M=128, N, K=16).
+//   warps 5-8  epilogue: tcgen05.ld -> fp32 partial sums in global memory.
+// Work split (stream-K): the (M tile, 64-row k-block) units are cut into one
+// contiguous range per CTA; a CTA writes one partial tile per M tile it
+// touches, into slot (tile + cta), and gemv_fixup_kernel adds the partials of
+// each tile in CTA order, so the result is deterministic.
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace rmm {
+
+struct GemvParams {
+  const uint16_t* W;   // [d][ldw] bf16
+  int64_t ldw;
+  const int32_t* idx;  // [k] kept rows, ascending, or null for rows [0, k)
+  int k;
+  int m;               // columns of W and Y
+  int n;               // rows of x and Y (<= N)
+  int m_tiles;         // ceil(m / 128)
+  int kb_total;        // ceil(k / 64)
+  int64_t units;       // m_tiles * kb_total
+  float* partial;      // [m_tiles + gridDim.x][n][128]
+};
+
+constexpr int kGemvStages = 6;
+constexpr int kGemvLag = 3;  // cp.async groups a producer keeps in flight before signalling
+
+__device__ __forceinline__ int64_t gemv_unit_begin(int64_t c, int64_t units, int64_t G) { return (c * units) / G; }
+
+__device__ __forceinline__ void cp_async16_z(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns (thread t: row lane_base + t).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// exactly N (16 or 32) accumulator columns of this warp's 32 lanes
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
+  static_assert(N == 16 || N == 32, "N must be 16 or 32");
+  if constexpr (N == 16) {
+    uint32_t r[16];
+    tmem_ld16(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  } else {
+    uint32_t r[32];
+    tmem_ld32(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+
+template <int N>
+__global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CUtensorMap tmX, const GemvParams p) {
+  constexpr int A_BYTES = 128 * 64 * 2;  // 64 kept rows x 128 columns
+  constexpr int X_BYTES = N * 64 * 2;
+  constexpr uint32_t IDESC = make_idesc_bf16(128, N, 1, 0);
+  constexpr uint32_t TMEM_COLS = (2 * N < 32) ? 32 : 2 * N;
+
+  extern __shared__ uint8_t gv_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gv_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sX = smem + kGemvStages * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + kGemvStages * X_BYTES);
+  uint64_t* empty = full + kGemvStages;
+  uint64_t* tfull = empty + kGemvStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGemvStages; ++s) {
+      mbar_init(&full[s], 128 + 1);  // 128 producer arrivals + the TMA issuer's expect_tx
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmX);
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t G = gridDim.x;
+  const int64_t u_begin = gemv_unit_begin(blockIdx.x, p.units, G);
+  const int64_t u_end = gemv_unit_begin(blockIdx.x + 1, p.units, G);
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ producers
+    const int tid = threadIdx.x;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t u = u_begin; u < u_end; ++u) {
+      const int tile = static_cast<int>(u / p.kb_total);
+      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * p.kb_total);
+      const int m0 = tile * 128;
+      if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer)) {
+        ok = false;
+        break;
+      }
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&full[stage], X_BYTES);
+        tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * 64, 0);
+      }
+      uint8_t* dstA = sA + stage * A_BYTES;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int ch = i * 128 + tid;     // 16-byte chunk of the 64 x 128 tile
+        const int r = ch >> 4;            // kept row within the k-block
+        const int c16 = ch & 15;          // 16-byte column within the 256-byte segment
+        const int a = c16 >> 3;           // 64-column atom
+        const int cw = c16 & 7;           // 16-byte column within the atom
+        const int t = kb * 64 + r;
+        const int col = m0 + a * 64 + cw * 8;
+        const uint16_t* src = p.W;
+        uint32_t bytes = 0;
+        if (t < p.k && col < p.m) {
+          const int64_t row = (p.idx != nullptr) ? static_cast<int64_t>(__ldg(p.idx + t)) : t;
+          src = p.W + row * p.ldw + col;
+          bytes = (col + 8 <= p.m) ? 16u : static_cast<uint32_t>((p.m - col) * 2);
+        }
+        cp_async16_z(dstA + a * 8192 + r * 128 + ((cw ^ (r & 7)) << 4), src, bytes);
+      }
+      cp_async_commit_group();
+      ++issued;
+      if (issued > kGemvLag) {
+        // the copies of the stage issued kGemvLag groups ago have landed
+        cp_async_wait_group<kGemvLag>();
+        fence_proxy_async_smem();
+        const int s_old = static_cast<int>((issued - 1 - kGemvLag) % kGemvStages);
+        mbar_arrive(&full[s_old]);
+      }
+      if (++stage == kGemvStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    // signal the stages still in flight (also on the abort path, so nothing lands late)
+    cp_async_wait_group<0>();
+    fence_proxy_async_smem();
+    if (ok) {
+      const int64_t first = issued > kGemvLag ? issued - kGemvLag : 0;
+      for (int64_t g = first; g < issued; ++g) mbar_arrive(&full[static_cast<int>(g % kGemvStages)]);
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int seg = 0;
+      bool ok = true;
+      int64_t u = u_begin;
+      while (u < u_end && ok) {
+        const int tile = static_cast<int>(u / p.kb_total);
+        const int64_t tile_end = static_cast<int64_t>(tile + 1) * p.kb_total;
+        const int64_t seg_end = u_end < tile_end ? u_end : tile_end;
+        const int acc = seg & 1;
+        if (!mbar_wait(&tempty[acc], ((seg >> 1) & 1) ^ 1u, abort_flag, kDevErrTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * N);
+        for (int64_t v = u; v < seg_end; ++v) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t x0 = smem_u32(sX + stage * X_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sw128_desc(a0 + kk * 2048, 8192, 1024);
+            const uint64_t bd = make_sw128_desc(x0 + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, IDESC, (v != u || kk != 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kGemvStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        ++seg;
+        u = seg_end;
+      }
+      umma_commit(drain);
+      const uint32_t a = smem_u32(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int col_in_tile = quarter * 32 + lane;
+    int seg = 0;
+    int64_t u = u_begin;
+    while (u < u_end) {
+      const int tile = static_cast<int>(u / p.kb_total);
+      const int64_t tile_end = static_cast<int64_t>(tile + 1) * p.kb_total;
+      const int64_t seg_end = u_end < tile_end ? u_end : tile_end;
+      const int acc = seg & 1;
+      if (!mbar_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, kDevErrTimeoutEpilogue)) break;
+      tc_fence_after();
+      float v[N];
+      tmem_ld_cols<N>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * N), v);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      float* part = p.partial + (static_cast<int64_t>(tile) + blockIdx.x) * p.n * 128;
+#pragma unroll
+      for (int r = 0; r < N; ++r)
+        if (r < p.n) part[r * 128 + col_in_tile] = v[r];
+      ++seg;
+      u = seg_end;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Y[r, m0 + i] = bf16( sum over the CTAs c that touched tile t, in increasing c,
+// of partial[t + c][r][i] ).  One thread per (tile, column).
+__global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy) {
+  const int tile = blockIdx.x;
+  const int i = threadIdx.x;
+  const int col = tile * 128 + i;
+  if (col >= p.m) return;
+  const int64_t U = p.units, G = grid;
+  const int64_t u_lo = static_cast<int64_t>(tile) * p.kb_total;
+  const int64_t u_hi = u_lo + p.kb_total - 1;
+  const int64_t c_lo = ((u_lo + 1) * G - 1) / U;  // owner of unit u_lo
+  const int64_t c_hi = ((u_hi + 1) * G - 1) / U;  // owner of unit u_hi
+  for (int r = 0; r < p.n; ++r) {
+    float s = 0.f;
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      if ((c * U) / G == ((c + 1) * U) / G) continue;  // this CTA had no units at all
+      s += p.partial[(tile + c) * p.n * 128 + r * 128 + i];
+    }
+    const __nv_bfloat16 h = __float2bfloat16_rn(s);
+    Y[static_cast<int64_t>(r) * ldy + col] = *reinterpret_cast<const uint16_t*>(&h);
+  }
+}
+
+}  // namespace rmm

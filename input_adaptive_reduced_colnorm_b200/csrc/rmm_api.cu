@@ -17,6 +17,7 @@
 #include "select.cuh"
 #include "pack.cuh"
 #include "gemm.cuh"
+#include "gemv.cuh"
 
 using namespace rmm;
 
@@ -303,6 +304,53 @@ rmm_status gemm_packed(const uint16_t* A, int64_t n, int64_t k, int64_t lda, con
   return launch_gemm<256, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
 }
 
+// Decode path (n <= 32): Y = x[:, I] . W[I, :] streaming only the kept rows of W.
+constexpr int64_t kDecodeMaxRows = 32;
+
+int decode_grid(int64_t units) { return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms()))); }
+
+size_t decode_partial_floats(int64_t n, int64_t m, int64_t k) {
+  const int64_t m_tiles = ceil_div(m, 128);
+  const int64_t units = m_tiles * ceil_div(k, 64);
+  return static_cast<size_t>((m_tiles + decode_grid(units)) * n * 128);
+}
+
+rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint16_t* W, int64_t k, int64_t m,
+                          int64_t ldw, const int32_t* idx, float* partial, uint16_t* Y, int64_t ldy, cudaStream_t s) {
+  GemvParams g{};
+  g.W = W;
+  g.ldw = ldw;
+  g.idx = idx;
+  g.k = static_cast<int>(k);
+  g.m = static_cast<int>(m);
+  g.n = static_cast<int>(n);
+  g.m_tiles = static_cast<int>(ceil_div(m, 128));
+  g.kb_total = static_cast<int>(ceil_div(k, 64));
+  g.units = static_cast<int64_t>(g.m_tiles) * g.kb_total;
+  g.partial = partial;
+  const int grid = decode_grid(g.units);
+  const int N = (n <= 16) ? 16 : 32;
+  CUtensorMap tx;
+  // x_I (or x itself) as the K-major operand: N rows (rows past n read zero) x 64 columns per box
+  if (rmm_status st = make_tmap(&tx, xp, k, n, ldx * 2, 64, static_cast<uint32_t>(N))) return st;
+  const int smem = 1024 + kGemvStages * (128 * 64 * 2 + N * 64 * 2) + 256;
+  cudaError_t e;
+  if (N == 16) {
+    e = cudaFuncSetAttribute(gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) gemv_kernel<16><<<grid, 288, smem, s>>>(tx, g);
+  } else {
+    e = cudaFuncSetAttribute(gemv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) gemv_kernel<32><<<grid, 288, smem, s>>>(tx, g);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode attribute");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  gemv_fixup_kernel<<<g.m_tiles, 128, 0, s>>>(g, grid, Y, ldy);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode fix-up launch");
+  return RMM_OK;
+}
+
 }  // namespace
 
 // ============================================================== public API
@@ -450,9 +498,18 @@ rmm_status rmm_select_noalloc(const rmm_bf16* A, int64_t batch, int64_t batch_st
 // ---------------------------------------------------------------- linear
 size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
   const int64_t k = rmm_k(rho, d);
-  if (k < 0 || n < 1) return 0;
-  if (k == d) return 0;
+  if (k < 0 || n < 1 || m < 1) return 0;
   Carver c(nullptr);
+  if (n <= kDecodeMaxRows) {
+    if (k < d) {
+      c.take<double>(d);
+      c.take<int32_t>(k);
+      c.take<uint16_t>(n * round_up(k, 8));
+    }
+    c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
+    return c.bytes();
+  }
+  if (k == d) return 0;
   c.take<double>(d);
   c.take<int32_t>(k);
   c.take<uint16_t>(n * round_up(k, 8));
@@ -474,6 +531,33 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
     return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
   const int64_t k = rmm_k(rho, d);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n <= kDecodeMaxRows) {
+    // decode: stream only the kept rows of B (all rows when rho = 1)
+    if (d > kMaxSelectD && k < d) return fail(RMM_ERR_UNSUPPORTED, "d > %lld", static_cast<long long>(kMaxSelectD));
+    const size_t need = rmm_linear_workspace_bytes(n, d, m, rho);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    Carver c(ws);
+    if (k == d) {
+      float* partial = c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
+      if (idx_out != nullptr) {
+        iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024)), 256, 0, s>>>(idx_out, 1, d);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+      }
+      return decode_product(A, n, lda, B, d, m, ldb, nullptr, partial, Y, ldy, s);
+    }
+    const int64_t k_pad = round_up(k, 8);
+    double* colsq = c.take<double>(d);
+    int32_t* idx_ws = c.take<int32_t>(k);
+    uint16_t* xpack = c.take<uint16_t>(n * k_pad);
+    float* partial = c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
+    if (rmm_status st = pack_columns(A, n, d, lda, idx, k, xpack, k_pad, s)) return st;
+    return decode_product(xpack, n, k_pad, B, k, m, ldb, idx, partial, Y, ldy, s);
+  }
   if (k == d) {
     // rho = 1: the dense product, I = [0, d)
     if (idx_out != nullptr) {

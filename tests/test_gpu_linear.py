@@ -135,3 +135,38 @@ def test_stage_entry_points_compose_to_rmm_linear():
     expect[:, :k] = A.cpu()[:, I]
     assert torch.equal(ap.cpu(), expect)
     assert torch.equal(bp.cpu()[:, :520], B.cpu()[I, :])
+
+
+_DECODE_W = {}
+
+
+def decode_weight():
+    if "W" not in _DECODE_W:
+        _, _DECODE_W["W"] = synthetic.decode_gemv(1)
+    return _DECODE_W["W"]
+
+
+@pytest.mark.parametrize("n", [1, 8, 32])
+@pytest.mark.parametrize("rho", [0.5, 0.7, 0.9, 1.0])
+def test_linear_decode_llama70b_mlp_up(n, rho):
+    """Decode GEMV on the Llama-3.1-70B MLP-up shape: x n x 8192, W 8192 x 28672."""
+    A, _ = synthetic.decode_gemv(n, weight=False)
+    parity_linear(A, decode_weight(), rho)
+
+
+@pytest.mark.parametrize("n,d,m", [(2, 300, 1000), (16, 64, 136), (17, 4100, 264), (31, 1000, 8), (32, 12, 4096)])
+@pytest.mark.parametrize("rho", [0.3, 1.0])
+def test_linear_decode_ragged(n, d, m, rho):
+    g = synthetic.rng(n * 7919 + d * 31 + m)
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, n, d, 1.5))
+    B = synthetic.to_bf16(synthetic.gaussian_weight(g, d, m))
+    parity_linear(A, B, rho)
+
+
+def test_linear_decode_deterministic():
+    A, _ = synthetic.decode_gemv(8, weight=False)
+    Ad, Wd = A.cuda(), decode_weight().cuda()
+    a = rmm.linear(Ad, Wd, 0.7, return_idx=True)
+    b = rmm.linear(Ad, Wd, 0.7, return_idx=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
