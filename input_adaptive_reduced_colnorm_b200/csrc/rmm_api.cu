@@ -156,8 +156,9 @@ rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64
 
 template <int KPT, int NT>
 rmm_status launch_select_t(const SelectParams& p, int64_t batch, cudaStream_t s) {
+  // dynamic keys plus ~17 KB of static histogram and scan space can pass 48 KB
   const size_t smem = static_cast<size_t>(NT) * KPT * sizeof(uint32_t);
-  if (smem > 48 * 1024) {
+  {
     const cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e, "select attribute");
