@@ -44,6 +44,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the per-call timings of the other workloads")
     ap.add_argument("--cpu-rows", type=int, default=4096, help="rows per projection in the CPU-oracle sample")
     return ap.parse_args()
 
@@ -246,6 +247,119 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ the other workloads
+def bench_workloads(dev, stream, L, reps=10, warm=3):
+    """Per-call timings of the other four workloads (single linear layer, decode GEMV,
+    GQA QK^T, long-context PV) at their rho values and at rho = 1, each against its
+    roofline: kept FLOPs at the bf16 peak or algorithmic bytes at the HBM peak."""
+    import ctypes
+    import torch
+    import synthetic
+
+    peaks, src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+
+    def ok(st):
+        if st != 0:
+            raise RuntimeError(L.rmm_last_error().decode())
+
+    def timed_call(fn):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    out = {"hbm_peak_gbs": hbm, "peak_source": src, "reps": reps}
+
+    def linear_case(A, W, rho):
+        n, d = A.shape
+        m = W.shape[1]
+        Y = torch.empty((n, m), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(L.rmm_linear_workspace_bytes(n, d, m, rho), 256), dtype=torch.uint8, device=dev)
+        ms = timed_call(lambda: ok(L.rmm_linear(A.data_ptr(), n, d, d, W.data_ptr(), m, m, Y.data_ptr(), m, rho,
+                                                None, ws.data_ptr(), ws.numel(), sptr)))
+        k = k_of(rho, d)
+        nbytes = kept_bytes(n, d, m, rho)
+        return {"k": k, "ms": ms, "tflops": 2.0 * n * k * m / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9}
+
+    # single linear layer, 128 x 1024 x 1024, rho = 0.5 (latency-bound)
+    A, B = synthetic.linear_small()
+    A, B = A.to(dev), B.to(dev)
+    r05, r1 = linear_case(A, B, 0.5), linear_case(A, B, 1.0)
+    out["linear_128x1024x1024"] = {"0.5": r05, "1.0": r1, "speedup_vs_rho1": r1["ms"] / r05["ms"]}
+
+    # decode GEMV, Llama-3.1-70B MLP-up: x n x 8192, W 8192 x 28672 (HBM-bound on kept W rows)
+    _, W = synthetic.decode_gemv(1)
+    W = W.to(dev)
+    dec = {}
+    for n in (1, 8, 32):
+        x, _ = synthetic.decode_gemv(n, weight=False)
+        x = x.to(dev)
+        row = {str(r): linear_case(x, W, r) for r in (1.0, 0.9, 0.7, 0.5)}
+        for r in ("0.9", "0.7", "0.5", "1.0"):
+            row[r]["hbm_frac"] = row[r]["gbs"] / hbm
+            row[r]["speedup_vs_rho1"] = row["1.0"]["ms"] / row[r]["ms"]
+        dec[f"n={n}"] = row
+    out["decode_70b_mlp_up"] = dec
+    del W
+
+    # GQA QK^T: 32 query heads / 8 key heads, seq 4096, head_dim 128, causal fp32 scores
+    Q, K = synthetic.qk_inputs()
+    Q, K = Q.to(dev), K.to(dev)
+    b_, hq, nq, dh = Q.shape
+    hkv, nk = K.shape[1], K.shape[2]
+    S = torch.empty((b_, hq, nq, nk), dtype=torch.float32, device=dev)
+    qk = {}
+    for rho in (1.0, 0.7, 0.5):
+        ws = torch.empty(max(L.rmm_qk_workspace_bytes(b_, hq, hkv, nq, nk, dh, rho), 256), dtype=torch.uint8,
+                         device=dev)
+        ms = timed_call(lambda: ok(L.rmm_qk(Q.data_ptr(), K.data_ptr(), S.data_ptr(), b_, hq, hkv, nq, nk, dh, 1,
+                                            1.0, rho, None, ws.data_ptr(), ws.numel(), sptr)))
+        k = k_of(rho, dh)
+        flops = 2.0 * k * nq * (nq + 1) / 2 * hq * b_
+        nbytes = b_ * hq * (nq * dh * 2 + (nq + nk) * k * 2 + nq * nk * 4)
+        qk[str(rho)] = {"k": k, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                        "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm}
+    for r in qk:
+        qk[r]["speedup_vs_rho1"] = qk["1.0"]["ms"] / qk[r]["ms"]
+    out["qk_gqa_seq4096"] = qk
+    del Q, K, S, ws
+
+    # long-context PV: 32 heads, seq 16384, head_dim 128, causal softmax probabilities
+    P, V = synthetic.pv_inputs_device(dev)
+    b_, h, nq, nk = P.shape
+    dh = V.shape[3]
+    O = torch.empty((b_, h, nq, dh), dtype=torch.bfloat16, device=dev)
+    pv = {}
+    for rho in (1.0, 0.8, 0.5):
+        k = k_of(rho, nk)
+        ws = torch.empty(max(L.rmm_pv_workspace_bytes(b_, h, h, nq, nk, dh, rho), 256), dtype=torch.uint8,
+                         device=dev)
+        idx = torch.empty((b_, h, k), dtype=torch.int32, device=dev)
+        ms = timed_call(lambda: ok(L.rmm_pv(P.data_ptr(), V.data_ptr(), O.data_ptr(), b_, h, h, nq, nk, dh, 1, rho,
+                                            idx.data_ptr(), ws.data_ptr(), ws.numel(), sptr)))
+        I = idx.to(torch.float64)
+        flops = float((2.0 * dh * (nk - I)).sum())  # kept multiply-adds below the causal diagonal
+        tri = nq * (nq + 1) / 2
+        kept_p = float((nk - I).sum()) * 2  # kept columns of P below the diagonal, bf16
+        nbytes = (0 if rho == 1.0 else b_ * h * tri * 2) + kept_p + b_ * h * (k * dh * 2 + nq * dh * 2)
+        pv[str(rho)] = {"k": k, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                        "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm}
+    for r in pv:
+        pv[r]["speedup_vs_rho1"] = pv["1.0"]["ms"] / pv[r]["ms"]
+    out["pv_seq16384"] = pv
+    del P, V, O, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ GPU leg
 def run_ours(args):
     import torch
@@ -423,6 +537,8 @@ def run_ours(args):
         "gpu_launches": 20 * K,
         "clocks": sampler.summary(),
     }
+    if world == 1 and not args.no_workloads:
+        line["workloads"] = bench_workloads(dev, stream, L)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_rows)
     if world > 1:
