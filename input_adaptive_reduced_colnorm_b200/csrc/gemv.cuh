@@ -11,7 +11,9 @@
 //              loaded with 16-byte cp.async straight into the 128-byte-swizzled
 //              MN-major operand layout (a TMA row gather stages only ~7 B/clk/SM
 //              on B200, 16-byte cp.async ~35 B/clk/SM; HBM speed needs ~22);
-//              thread 0 also brings the packed activations x_I with a TMA tile.
+//              two threads per kept row, the index set read once into shared
+//              memory as 16-bit row numbers, five copy groups in flight per
+//              thread; thread 0 also brings the packed activations x_I by TMA.
 //   warp 4     allocates TMEM; one thread issues tcgen05.mma (M=128, N, K=16).
 //   warps 5-8  epilogue: tcgen05.ld -> fp32 partial sums in global memory.
 // Work split (stream-K): the (M tile, 64-row k-block) units are cut into one
@@ -37,8 +39,9 @@ struct GemvParams {
   float* partial;      // [m_tiles + gridDim.x][n][128]
 };
 
-constexpr int kGemvStages = 6;
-constexpr int kGemvLag = 3;  // cp.async groups a producer keeps in flight before signalling
+constexpr int kGemvStages = 8;
+constexpr int kGemvLag = 5;  // cp.async groups a producer keeps in flight before signalling
+constexpr int kGemvMaxK = 32768;  // kept rows held as 16-bit indices in shared memory
 
 __device__ __forceinline__ int64_t gemv_unit_begin(int64_t c, int64_t units, int64_t G) { return (c * units) / G; }
 
@@ -98,8 +101,11 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint16_t* s_idx = reinterpret_cast<uint16_t*>(smem + kGemvStages * (A_BYTES + X_BYTES) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (p.idx != nullptr)
+    for (int t = threadIdx.x; t < p.k; t += blockDim.x) s_idx[t] = static_cast<uint16_t>(__ldg(p.idx + t));
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemvStages; ++s) {
       mbar_init(&full[s], 128 + 1);  // 128 producer arrivals + the TMA issuer's expect_tx
@@ -147,23 +153,25 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
         tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * 64, 0);
       }
       uint8_t* dstA = sA + stage * A_BYTES;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int ch = i * 128 + tid;     // 16-byte chunk of the 64 x 128 tile
-        const int r = ch >> 4;            // kept row within the k-block
-        const int c16 = ch & 15;          // 16-byte column within the 256-byte segment
-        const int a = c16 >> 3;           // 64-column atom
-        const int cw = c16 & 7;           // 16-byte column within the atom
+      {
+        // thread pair (2r, 2r+1) copies kept row r of the k-block: 8 chunks of 16 bytes each
+        const int r = tid >> 1;
         const int t = kb * 64 + r;
-        const int col = m0 + a * 64 + cw * 8;
-        const uint16_t* src = p.W;
-        uint32_t bytes = 0;
-        if (t < p.k && col < p.m) {
-          const int64_t row = (p.idx != nullptr) ? static_cast<int64_t>(__ldg(p.idx + t)) : t;
-          src = p.W + row * p.ldw + col;
-          bytes = (col + 8 <= p.m) ? 16u : static_cast<uint32_t>((p.m - col) * 2);
+        const int64_t row = (t < p.k) ? ((p.idx != nullptr) ? static_cast<int64_t>(s_idx[t]) : t) : -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c16 = (tid & 1) * 8 + j;  // 16-byte column within the 256-byte segment
+          const int a = c16 >> 3;             // 64-column atom
+          const int cw = c16 & 7;             // 16-byte column within the atom
+          const int col = m0 + a * 64 + cw * 8;
+          const uint16_t* src = p.W;
+          uint32_t bytes = 0;
+          if (row >= 0 && col < p.m) {
+            src = p.W + row * p.ldw + col;
+            bytes = (col + 8 <= p.m) ? 16u : static_cast<uint32_t>((p.m - col) * 2);
+          }
+          cp_async16_z(dstA + a * 8192 + r * 128 + ((cw ^ (r & 7)) << 4), src, bytes);
         }
-        cp_async16_z(dstA + a * 8192 + r * 128 + ((cw ^ (r & 7)) << 4), src, bytes);
       }
       cp_async_commit_group();
       ++issued;

@@ -318,6 +318,7 @@ size_t decode_partial_floats(int64_t n, int64_t m, int64_t k) {
 
 rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint16_t* W, int64_t k, int64_t m,
                           int64_t ldw, const int32_t* idx, float* partial, uint16_t* Y, int64_t ldy, cudaStream_t s) {
+  if (idx != nullptr && k > kGemvMaxK) return fail(RMM_ERR_UNSUPPORTED, "decode path keeps at most %d rows", kGemvMaxK);
   GemvParams g{};
   g.W = W;
   g.ldw = ldw;
@@ -334,7 +335,8 @@ rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint
   CUtensorMap tx;
   // x_I (or x itself) as the K-major operand: N rows (rows past n read zero) x 64 columns per box
   if (rmm_status st = make_tmap(&tx, xp, k, n, ldx * 2, 64, static_cast<uint32_t>(N))) return st;
-  const int smem = 1024 + kGemvStages * (128 * 64 * 2 + N * 64 * 2) + 256;
+  const int smem = 1024 + kGemvStages * (128 * 64 * 2 + N * 64 * 2) + 256 +
+                   (idx != nullptr ? static_cast<int>(round_up(k, 8) * 2) : 0);
   cudaError_t e;
   if (N == 16) {
     e = cudaFuncSetAttribute(gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
