@@ -5,21 +5,22 @@
 // those rows are read, once, straight from W -- no packed copy of W[I, :].
 //
 // Tensor cores with the operands swapped: D[128 weight columns x N rows] =
-// W_I^T (M = 128, MN-major) . x_I^T (N = 16 or 32, K-major), fp32 accumulator
-// in tensor memory.
-//   warps 0-3  producers: every kept-row segment (128 columns = 256 bytes) is
+// W_I^T (M = 128, MN-major) . x_I^T (N = 16 or 32, K-major), fp32 accumulators
+// in tensor memory, four of them (one per 128-column tile of a super tile).
+//   warps 0-3  producers: each CTA works on a 512-column super tile, so every
+//              kept row contributes one contiguous 1 KB run per stage (runs of
+//              256 B per row reached only ~40% of HBM bandwidth); the runs are
 //              loaded with 16-byte cp.async straight into the 128-byte-swizzled
 //              MN-major operand layout (a TMA row gather stages only ~7 B/clk/SM
-//              on B200, 16-byte cp.async ~35 B/clk/SM; HBM speed needs ~22);
-//              two threads per kept row, the index set read once into shared
-//              memory as 16-bit row numbers, five copy groups in flight per
-//              thread; thread 0 also brings the packed activations x_I by TMA.
+//              on B200, 16-byte cp.async ~35 B/clk/SM); two threads per kept
+//              row, the next row number prefetched one stage ahead; thread 0
+//              also brings the packed activations x_I with a TMA tile.
 //   warp 4     allocates TMEM; one thread issues tcgen05.mma (M=128, N, K=16).
 //   warps 5-8  epilogue: tcgen05.ld -> fp32 partial sums in global memory.
-// Work split (stream-K): the (M tile, 64-row k-block) units are cut into one
-// contiguous range per CTA; a CTA writes one partial tile per M tile it
-// touches, into slot (tile + cta), and gemv_fixup_kernel adds the partials of
-// each tile in CTA order, so the result is deterministic.
+// Work split (stream-K): the (super tile, 64-row k-block) units are cut into
+// one contiguous range per CTA; a CTA writes one partial super tile per super
+// tile it touches, into slot (super tile + cta), and gemv_fixup_kernel adds the
+// partials of each column in CTA order, so the result is deterministic.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -33,15 +34,16 @@ struct GemvParams {
   int k;
   int m;               // columns of W and Y
   int n;               // rows of x and Y (<= N)
-  int m_tiles;         // ceil(m / 128)
+  int m_super;         // ceil(m / 512): 512-column super tiles (four 128-column MMA tiles)
   int kb_total;        // ceil(k / 64)
-  int64_t units;       // m_tiles * kb_total
-  float* partial;      // [m_tiles + gridDim.x][n][128]
+  int64_t units;       // m_super * kb_total
+  float* partial;      // [m_super + gridDim.x][4][n][128]
 };
 
-constexpr int kGemvStages = 8;
-constexpr int kGemvLag = 5;  // cp.async groups a producer keeps in flight before signalling
-constexpr int kGemvMaxK = 32768;  // kept rows held as 16-bit indices in shared memory
+constexpr int kGemvTiles = 4;                  // 128-column MMA tiles per super tile
+constexpr int kGemvCols = 128 * kGemvTiles;    // 512 columns = 1 KB of each kept row per stage
+constexpr int kGemvStages = 3;
+constexpr int kGemvLag = 2;  // cp.async groups a producer keeps in flight before signalling
 
 __device__ __forceinline__ int64_t gemv_unit_begin(int64_t c, int64_t units, int64_t G) { return (c * units) / G; }
 
@@ -83,12 +85,18 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
   }
 }
 
+__device__ __forceinline__ int64_t gemv_row_of(const GemvParams& p, int t) {
+  if (t >= p.k) return -1;
+  return (p.idx != nullptr) ? static_cast<int64_t>(__ldg(p.idx + t)) : t;
+}
+
 template <int N>
 __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CUtensorMap tmX, const GemvParams p) {
-  constexpr int A_BYTES = 128 * 64 * 2;  // 64 kept rows x 128 columns
+  constexpr int A_BYTES = kGemvCols * 64 * 2;  // 64 kept rows x 512 columns
   constexpr int X_BYTES = N * 64 * 2;
   constexpr uint32_t IDESC = make_idesc_bf16(128, N, 1, 0);
-  constexpr uint32_t TMEM_COLS = (2 * N < 32) ? 32 : 2 * N;
+  constexpr uint32_t ACC_COLS = kGemvTiles * N;  // one accumulator = four N-column tiles
+  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;   // double-buffered (128 or 256 columns)
 
   extern __shared__ uint8_t gv_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gv_raw) + 1023) & ~uintptr_t(1023));
@@ -101,11 +109,8 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint16_t* s_idx = reinterpret_cast<uint16_t*>(smem + kGemvStages * (A_BYTES + X_BYTES) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (p.idx != nullptr)
-    for (int t = threadIdx.x; t < p.k; t += blockDim.x) s_idx[t] = static_cast<uint16_t>(__ldg(p.idx + t));
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemvStages; ++s) {
       mbar_init(&full[s], 128 + 1);  // 128 producer arrivals + the TMA issuer's expect_tx
@@ -135,15 +140,21 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
+    // thread pair (2r, 2r+1) copies 1 KB of kept row r of the k-block, 512 B each
     const int tid = threadIdx.x;
+    const int r = tid >> 1;
     int stage = 0;
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
+    int64_t row_next = (u_begin < u_end)
+                           ? gemv_row_of(p, static_cast<int>(u_begin % p.kb_total) * 64 + r)
+                           : -1;
     for (int64_t u = u_begin; u < u_end; ++u) {
-      const int tile = static_cast<int>(u / p.kb_total);
-      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * p.kb_total);
-      const int m0 = tile * 128;
+      const int sup = static_cast<int>(u / p.kb_total);
+      const int kb = static_cast<int>(u - static_cast<int64_t>(sup) * p.kb_total);
+      const int64_t row = row_next;
+      if (u + 1 < u_end) row_next = gemv_row_of(p, static_cast<int>((u + 1) % p.kb_total) * 64 + r);
       if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer)) {
         ok = false;
         break;
@@ -153,25 +164,21 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
         tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * 64, 0);
       }
       uint8_t* dstA = sA + stage * A_BYTES;
-      {
-        // thread pair (2r, 2r+1) copies kept row r of the k-block: 8 chunks of 16 bytes each
-        const int r = tid >> 1;
-        const int t = kb * 64 + r;
-        const int64_t row = (t < p.k) ? ((p.idx != nullptr) ? static_cast<int64_t>(s_idx[t]) : t) : -1;
+      const int col_base = sup * kGemvCols;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int c16 = (tid & 1) * 8 + j;  // 16-byte column within the 256-byte segment
-          const int a = c16 >> 3;             // 64-column atom
-          const int cw = c16 & 7;             // 16-byte column within the atom
-          const int col = m0 + a * 64 + cw * 8;
-          const uint16_t* src = p.W;
-          uint32_t bytes = 0;
-          if (row >= 0 && col < p.m) {
-            src = p.W + row * p.ldw + col;
-            bytes = (col + 8 <= p.m) ? 16u : static_cast<uint32_t>((p.m - col) * 2);
-          }
-          cp_async16_z(dstA + a * 8192 + r * 128 + ((cw ^ (r & 7)) << 4), src, bytes);
+      for (int j = 0; j < 32; ++j) {
+        const int c16 = (tid & 1) * 32 + j;  // 16-byte chunk within the 1 KB row segment
+        const int tile = c16 >> 4;           // 128-column MMA tile
+        const int a = (c16 >> 3) & 1;        // 64-column atom within the tile
+        const int cw = c16 & 7;              // 16-byte column within the atom
+        const int col = col_base + c16 * 8;
+        const uint16_t* src = p.W;
+        uint32_t bytes = 0;
+        if (row >= 0 && col < p.m) {
+          src = p.W + row * p.ldw + col;
+          bytes = (col + 8 <= p.m) ? 16u : static_cast<uint32_t>((p.m - col) * 2);
         }
+        cp_async16_z(dstA + tile * 16384 + a * 8192 + r * 128 + ((cw ^ (r & 7)) << 4), src, bytes);
       }
       cp_async_commit_group();
       ++issued;
@@ -203,13 +210,13 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
       bool ok = true;
       int64_t u = u_begin;
       while (u < u_end && ok) {
-        const int tile = static_cast<int>(u / p.kb_total);
-        const int64_t tile_end = static_cast<int64_t>(tile + 1) * p.kb_total;
-        const int64_t seg_end = u_end < tile_end ? u_end : tile_end;
+        const int sup = static_cast<int>(u / p.kb_total);
+        const int64_t sup_end = static_cast<int64_t>(sup + 1) * p.kb_total;
+        const int64_t seg_end = u_end < sup_end ? u_end : sup_end;
         const int acc = seg & 1;
         if (!mbar_wait(&tempty[acc], ((seg >> 1) & 1) ^ 1u, abort_flag, kDevErrTimeoutMma)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * N);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * ACC_COLS;
         for (int64_t v = u; v < seg_end; ++v) {
           if (!mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma)) {
             ok = false;
@@ -220,9 +227,12 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
           const uint32_t x0 = smem_u32(sX + stage * X_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = make_sw128_desc(a0 + kk * 2048, 8192, 1024);
             const uint64_t bd = make_sw128_desc(x0 + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, IDESC, (v != u || kk != 0) ? 1u : 0u);
+#pragma unroll
+            for (int tl = 0; tl < kGemvTiles; ++tl) {
+              const uint64_t ad = make_sw128_desc(a0 + tl * 16384 + kk * 2048, 8192, 1024);
+              umma_bf16(d_tmem + static_cast<uint32_t>(tl * N), ad, bd, IDESC, (v != u || kk != 0) ? 1u : 0u);
+            }
           }
           umma_commit(&empty[stage]);
           if (++stage == kGemvStages) {
@@ -249,21 +259,27 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
     int seg = 0;
     int64_t u = u_begin;
     while (u < u_end) {
-      const int tile = static_cast<int>(u / p.kb_total);
-      const int64_t tile_end = static_cast<int64_t>(tile + 1) * p.kb_total;
-      const int64_t seg_end = u_end < tile_end ? u_end : tile_end;
+      const int sup = static_cast<int>(u / p.kb_total);
+      const int64_t sup_end = static_cast<int64_t>(sup + 1) * p.kb_total;
+      const int64_t seg_end = u_end < sup_end ? u_end : sup_end;
       const int acc = seg & 1;
       if (!mbar_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, kDevErrTimeoutEpilogue)) break;
       tc_fence_after();
-      float v[N];
-      tmem_ld_cols<N>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * N), v);
+      float v[kGemvTiles][N];
+#pragma unroll
+      for (int tl = 0; tl < kGemvTiles; ++tl)
+        tmem_ld_cols<N>(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc) * ACC_COLS +
+                            static_cast<uint32_t>(tl * N),
+                        v[tl]);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      float* part = p.partial + (static_cast<int64_t>(tile) + blockIdx.x) * p.n * 128;
+      float* part = p.partial + (static_cast<int64_t>(sup) + blockIdx.x) * kGemvTiles * p.n * 128;
 #pragma unroll
-      for (int r = 0; r < N; ++r)
-        if (r < p.n) part[r * 128 + col_in_tile] = v[r];
+      for (int tl = 0; tl < kGemvTiles; ++tl)
+#pragma unroll
+        for (int rr = 0; rr < N; ++rr)
+          if (rr < p.n) part[(tl * p.n + rr) * 128 + col_in_tile] = v[tl][rr];
       ++seg;
       u = seg_end;
     }
@@ -277,15 +293,16 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
   }
 }
 
-// Y[r, m0 + i] = bf16( sum over the CTAs c that touched tile t, in increasing c,
-// of partial[t + c][r][i] ).  One thread per (tile, column).
+// Y[r, col] = bf16( sum over the CTAs c that touched the column's super tile, in
+// increasing c, of their partial sums ).  One thread per output column.
 __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy) {
-  const int tile = blockIdx.x;
-  const int i = threadIdx.x;
-  const int col = tile * 128 + i;
+  const int col = blockIdx.x * 128 + threadIdx.x;
   if (col >= p.m) return;
+  const int sup = col / kGemvCols;
+  const int tl = (col % kGemvCols) / 128;
+  const int i = col % 128;
   const int64_t U = p.units, G = grid;
-  const int64_t u_lo = static_cast<int64_t>(tile) * p.kb_total;
+  const int64_t u_lo = static_cast<int64_t>(sup) * p.kb_total;
   const int64_t u_hi = u_lo + p.kb_total - 1;
   const int64_t c_lo = ((u_lo + 1) * G - 1) / U;  // owner of unit u_lo
   const int64_t c_hi = ((u_hi + 1) * G - 1) / U;  // owner of unit u_hi
@@ -293,7 +310,7 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int
     float s = 0.f;
     for (int64_t c = c_lo; c <= c_hi; ++c) {
       if ((c * U) / G == ((c + 1) * U) / G) continue;  // this CTA had no units at all
-      s += p.partial[(tile + c) * p.n * 128 + r * 128 + i];
+      s += p.partial[((sup + c) * kGemvTiles + tl) * p.n * 128 + r * 128 + i];
     }
     const __nv_bfloat16 h = __float2bfloat16_rn(s);
     Y[static_cast<int64_t>(r) * ldy + col] = *reinterpret_cast<const uint16_t*>(&h);

@@ -311,14 +311,13 @@ constexpr int64_t kDecodeMaxRows = 32;
 int decode_grid(int64_t units) { return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms()))); }
 
 size_t decode_partial_floats(int64_t n, int64_t m, int64_t k) {
-  const int64_t m_tiles = ceil_div(m, 128);
-  const int64_t units = m_tiles * ceil_div(k, 64);
-  return static_cast<size_t>((m_tiles + decode_grid(units)) * n * 128);
+  const int64_t m_super = ceil_div(m, kGemvCols);
+  const int64_t units = m_super * ceil_div(k, 64);
+  return static_cast<size_t>((m_super + decode_grid(units)) * kGemvTiles * n * 128);
 }
 
 rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint16_t* W, int64_t k, int64_t m,
                           int64_t ldw, const int32_t* idx, float* partial, uint16_t* Y, int64_t ldy, cudaStream_t s) {
-  if (idx != nullptr && k > kGemvMaxK) return fail(RMM_ERR_UNSUPPORTED, "decode path keeps at most %d rows", kGemvMaxK);
   GemvParams g{};
   g.W = W;
   g.ldw = ldw;
@@ -326,17 +325,16 @@ rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint
   g.k = static_cast<int>(k);
   g.m = static_cast<int>(m);
   g.n = static_cast<int>(n);
-  g.m_tiles = static_cast<int>(ceil_div(m, 128));
+  g.m_super = static_cast<int>(ceil_div(m, kGemvCols));
   g.kb_total = static_cast<int>(ceil_div(k, 64));
-  g.units = static_cast<int64_t>(g.m_tiles) * g.kb_total;
+  g.units = static_cast<int64_t>(g.m_super) * g.kb_total;
   g.partial = partial;
   const int grid = decode_grid(g.units);
   const int N = (n <= 16) ? 16 : 32;
   CUtensorMap tx;
   // x_I (or x itself) as the K-major operand: N rows (rows past n read zero) x 64 columns per box
   if (rmm_status st = make_tmap(&tx, xp, k, n, ldx * 2, 64, static_cast<uint32_t>(N))) return st;
-  const int smem = 1024 + kGemvStages * (128 * 64 * 2 + N * 64 * 2) + 256 +
-                   (idx != nullptr ? static_cast<int>(round_up(k, 8) * 2) : 0);
+  const int smem = 1024 + kGemvStages * (kGemvCols * 64 * 2 + N * 64 * 2) + 256;
   cudaError_t e;
   if (N == 16) {
     e = cudaFuncSetAttribute(gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -348,7 +346,7 @@ rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint
   if (e != cudaSuccess) return cuda_fail(e, "decode attribute");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  gemv_fixup_kernel<<<g.m_tiles, 128, 0, s>>>(g, grid, Y, ldy);
+  gemv_fixup_kernel<<<static_cast<unsigned>(ceil_div(m, 128)), 128, 0, s>>>(g, grid, Y, ldy);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode fix-up launch");
   return RMM_OK;
