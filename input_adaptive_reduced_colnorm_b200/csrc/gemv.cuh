@@ -140,22 +140,28 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
-    // thread pair (2r, 2r+1) copies 1 KB of kept row r of the k-block, 512 B each
+    // warp w copies kept rows 16w .. 16w+15 of the k-block; each warp instruction
+    // moves 512 contiguous bytes of one row (lane = 16-byte chunk), and lane l
+    // fetches the row number of row 16w + (l & 15), shared by shuffles
     const int tid = threadIdx.x;
-    const int r = tid >> 1;
     int stage = 0;
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
     int64_t row_next = (u_begin < u_end)
-                           ? gemv_row_of(p, static_cast<int>(u_begin % p.kb_total) * 64 + r)
+                           ? gemv_row_of(p, static_cast<int>(u_begin % p.kb_total) * 64 + warp * 16 + (lane & 15))
                            : -1;
     for (int64_t u = u_begin; u < u_end; ++u) {
       const int sup = static_cast<int>(u / p.kb_total);
       const int kb = static_cast<int>(u - static_cast<int64_t>(sup) * p.kb_total);
-      const int64_t row = row_next;
-      if (u + 1 < u_end) row_next = gemv_row_of(p, static_cast<int>((u + 1) % p.kb_total) * 64 + r);
-      if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer)) {
+      const int64_t my_row = row_next;
+      if (u + 1 < u_end)
+        row_next = gemv_row_of(p, static_cast<int>((u + 1) % p.kb_total) * 64 + warp * 16 + (lane & 15));
+      // one lane per warp waits, so the warp leaves the loop together (shuffles below)
+      int go = 1;
+      if (lane == 0) go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) {
         ok = false;
         break;
       }
@@ -167,10 +173,12 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
       const int col_base = sup * kGemvCols;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const int c16 = (tid & 1) * 32 + j;  // 16-byte chunk within the 1 KB row segment
-        const int tile = c16 >> 4;           // 128-column MMA tile
-        const int a = (c16 >> 3) & 1;        // 64-column atom within the tile
-        const int cw = c16 & 7;              // 16-byte column within the atom
+        const int r = warp * 16 + (j >> 1);   // kept row within the k-block
+        const int64_t row = __shfl_sync(0xffffffffu, my_row, j >> 1);
+        const int c16 = (j & 1) * 32 + lane;  // 16-byte chunk within the 1 KB row segment
+        const int tile = c16 >> 4;            // 128-column MMA tile
+        const int a = (c16 >> 3) & 1;         // 64-column atom within the tile
+        const int cw = c16 & 7;               // 16-byte column within the atom
         const int col = col_base + c16 * 8;
         const uint16_t* src = p.W;
         uint32_t bytes = 0;
