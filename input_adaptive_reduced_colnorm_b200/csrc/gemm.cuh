@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(192, 1)
       if (nkb > 0) {
         const int acc = acc_i & 1;
         const uint32_t acc_par = (acc_i >> 1) & 1;
-        if (!mbar_wait(&tfull[acc], acc_par, abort_flag, kDevErrTimeoutEpilogue)) break;
+        if (!mbar_wait(&tfull[acc], acc_par, abort_flag, kDevErrTimeoutEpilogue, 64)) break;
         tc_fence_after();
       }
       for (int c = 0; c < BN / 32; ++c) {

@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
       const int64_t sup_end = static_cast<int64_t>(sup + 1) * p.kb_total;
       const int64_t seg_end = u_end < sup_end ? u_end : sup_end;
       const int acc = seg & 1;
-      if (!mbar_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, kDevErrTimeoutEpilogue)) break;
+      if (!mbar_wait(&tfull[acc], (seg >> 1) & 1, abort_flag, kDevErrTimeoutEpilogue, 256)) break;
       tc_fence_after();
       float v[kGemvTiles][N];
 #pragma unroll

@@ -71,11 +71,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of ``bar`` with parity ``parity`` to complete.  Gives up
 // after kWaitTimeoutNs without progress, or as soon as *abort is set by another
 // role of the same CTA; on a timeout it sets *abort and records ``code``.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t code) {
+// ``sleep_ns`` > 0 backs off between polls: threads that wait long (epilogue
+// warps waiting for a finished accumulator) then leave the issue slots to the
+// warps that are moving data.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t code,
+                                          uint32_t sleep_ns = 0) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
