@@ -85,9 +85,9 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
   }
 }
 
-__device__ __forceinline__ int64_t gemv_row_of(const GemvParams& p, int t) {
+__device__ __forceinline__ int gemv_row_of(const GemvParams& p, int t) {
   if (t >= p.k) return -1;
-  return (p.idx != nullptr) ? static_cast<int64_t>(__ldg(p.idx + t)) : t;
+  return (p.idx != nullptr) ? __ldg(p.idx + t) : t;
 }
 
 template <int N>
@@ -148,13 +148,13 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
-    int64_t row_next = (u_begin < u_end)
+    int row_next = (u_begin < u_end)
                            ? gemv_row_of(p, static_cast<int>(u_begin % p.kb_total) * 64 + warp * 16 + (lane & 15))
                            : -1;
     for (int64_t u = u_begin; u < u_end; ++u) {
       const int sup = static_cast<int>(u / p.kb_total);
       const int kb = static_cast<int>(u - static_cast<int64_t>(sup) * p.kb_total);
-      const int64_t my_row = row_next;
+      const int my_row = row_next;
       if (u + 1 < u_end)
         row_next = gemv_row_of(p, static_cast<int>((u + 1) % p.kb_total) * 64 + warp * 16 + (lane & 15));
       // one lane per warp waits, so the warp leaves the loop together (shuffles below)
@@ -171,10 +171,15 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
       }
       uint8_t* dstA = sA + stage * A_BYTES;
       const int col_base = sup * kGemvCols;
+      // all 16 row numbers first: shuffles are volatile asm like cp.async, so a
+      // shuffle placed between two copies would hold the second copy back
+      int rows[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) rows[q] = __shfl_sync(0xffffffffu, my_row, q);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int r = warp * 16 + (j >> 1);   // kept row within the k-block
-        const int64_t row = __shfl_sync(0xffffffffu, my_row, j >> 1);
+        const int64_t row = rows[j >> 1];
         const int c16 = (j & 1) * 32 + lane;  // 16-byte chunk within the 1 KB row segment
         const int tile = c16 >> 4;            // 128-column MMA tile
         const int a = (c16 >> 3) & 1;         // 64-column atom within the tile
