@@ -141,23 +141,32 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
   if (warp < 4) {
     // ------------------------------------------------------------ producers
     // warp w copies kept rows 16w .. 16w+15 of the k-block; each warp instruction
-    // moves 512 contiguous bytes of one row (lane = 16-byte chunk), and lane l
-    // fetches the row number of row 16w + (l & 15), shared by shuffles
+    // moves 512 contiguous bytes of one row (lane = 16-byte chunk).  Every lane
+    // holds the warp's 16 row numbers in registers, loaded one stage ahead
+    // (same-address loads, no cross-lane traffic between the copies).
     const int tid = threadIdx.x;
     int stage = 0;
     uint32_t phase = 0;
     int64_t issued = 0;
     bool ok = true;
-    int row_next = (u_begin < u_end)
-                           ? gemv_row_of(p, static_cast<int>(u_begin % p.kb_total) * 64 + warp * 16 + (lane & 15))
-                           : -1;
+    int rows_next[16];
+    if (u_begin < u_end) {
+      const int t0 = static_cast<int>(u_begin % p.kb_total) * 64 + warp * 16;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) rows_next[q] = gemv_row_of(p, t0 + q);
+    }
     for (int64_t u = u_begin; u < u_end; ++u) {
       const int sup = static_cast<int>(u / p.kb_total);
       const int kb = static_cast<int>(u - static_cast<int64_t>(sup) * p.kb_total);
-      const int my_row = row_next;
-      if (u + 1 < u_end)
-        row_next = gemv_row_of(p, static_cast<int>((u + 1) % p.kb_total) * 64 + warp * 16 + (lane & 15));
-      // one lane per warp waits, so the warp leaves the loop together (shuffles below)
+      int rows[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) rows[q] = rows_next[q];
+      if (u + 1 < u_end) {
+        const int t0 = static_cast<int>((u + 1) % p.kb_total) * 64 + warp * 16;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) rows_next[q] = gemv_row_of(p, t0 + q);
+      }
+      // one lane per warp waits, so the warp leaves the loop together
       int go = 1;
       if (lane == 0) go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
       go = __shfl_sync(0xffffffffu, go, 0);
@@ -171,11 +180,6 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
       }
       uint8_t* dstA = sA + stage * A_BYTES;
       const int col_base = sup * kGemvCols;
-      // all 16 row numbers first: shuffles are volatile asm like cp.async, so a
-      // shuffle placed between two copies would hold the second copy back
-      int rows[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) rows[q] = __shfl_sync(0xffffffffu, my_row, q);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int r = warp * 16 + (j >> 1);   // kept row within the k-block
