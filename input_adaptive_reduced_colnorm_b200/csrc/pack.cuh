@@ -157,8 +157,19 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
     }
     if (rb != cur_b) {  // (re)load this batch item's index set as 16-bit offsets
       const int32_t* I = p.idx + rb * p.k;
-      for (int64_t t = threadIdx.x; t < p.k_pad; t += blockDim.x)
-        s_idx[t] = (t < p.k) ? static_cast<uint16_t>(__ldg(I + t)) : uint16_t(0xFFFF);
+      for (int64_t t0 = threadIdx.x; t0 < p.k_pad; t0 += 8 * static_cast<int64_t>(blockDim.x)) {
+        int32_t v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {  // eight loads in flight per thread
+          const int64_t t = t0 + e * static_cast<int64_t>(blockDim.x);
+          v[e] = (t < p.k) ? __ldg(I + t) : 0xFFFF;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int64_t t = t0 + e * static_cast<int64_t>(blockDim.x);
+          if (t < p.k_pad) s_idx[t] = static_cast<uint16_t>(v[e]);
+        }
+      }
       cur_b = rb;
     }
     __syncthreads();

@@ -97,9 +97,21 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   const int d = static_cast<int>(p.d);
   const int j0 = threadIdx.x * KPT;
 
-  // coalesced staging of the top 32 bits of every key
-  for (int j = threadIdx.x; j < d; j += NT)
-    s_keys[j] = static_cast<uint32_t>(static_cast<uint64_t>(__double_as_longlong(q[j])) >> 32);
+  // coalesced staging of the top 32 bits of every key: all KPT loads of a
+  // thread are in flight before the first store
+  {
+    uint32_t v[KPT];
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+      const int j = e * NT + threadIdx.x;
+      v[e] = (j < d) ? static_cast<uint32_t>(static_cast<uint64_t>(__double_as_longlong(__ldg(q + j))) >> 32) : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+      const int j = e * NT + threadIdx.x;
+      if (j < d) s_keys[j] = v[e];
+    }
+  }
   __syncthreads();
   uint32_t hi[KPT];
   uint32_t valid = 0;
