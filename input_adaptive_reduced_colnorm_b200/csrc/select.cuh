@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
       c[i] = hist[threadIdx.x * BPT + i];
       ls += c[i];
     }
-    // exclusive scan in descending thread order: reverse the thread index
+    // larger digits live in higher threads: their count is total - before - own
     const int before = block_exclusive_scan<NT>(static_cast<int>(ls), s_warp, &s_total);
     const uint32_t total = static_cast<uint32_t>(s_total);
     uint32_t above = total - static_cast<uint32_t>(before) - ls;  // digits held by higher threads
