@@ -311,10 +311,11 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
 }
 
 // Y[r, col] = bf16( sum over the CTAs c that touched the column's super tile, in
-// increasing c, of their partial sums ).  One thread per output column; the
-// owning CTAs are found once per thread, the rows are summed in registers.
+// increasing c, of their partial sums ).  One thread per (output column, row r =
+// blockIdx.y); the owning CTAs are found from the same unit split as the kernel.
 __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy) {
   const int col = blockIdx.x * 128 + threadIdx.x;
+  const int r = blockIdx.y;
   if (col >= p.m) return;
   const int sup = col / kGemvCols;
   const int tl = (col % kGemvCols) / 128;
@@ -324,27 +325,16 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int
   const int64_t u_hi = u_lo + p.kb_total - 1;
   const int c_lo = static_cast<int>(((u_lo + 1) * G - 1) / U);  // owner of unit u_lo
   const int c_hi = static_cast<int>(((u_hi + 1) * G - 1) / U);  // owner of unit u_hi
-  float acc[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) acc[r] = 0.f;
+  float acc = 0.f;
   int64_t start_c = (static_cast<int64_t>(c_lo) * U) / G;
   for (int c = c_lo; c <= c_hi; ++c) {
     const int64_t start_next = (static_cast<int64_t>(c + 1) * U) / G;
-    if (start_next > start_c) {  // CTA c had at least one unit
-      const float* part = p.partial + ((static_cast<int64_t>(sup) + c) * kGemvTiles + tl) * p.n * 128 + i;
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-        if (r < p.n) acc[r] += part[r * 128];
-    }
+    if (start_next > start_c)  // CTA c had at least one unit
+      acc += p.partial[((static_cast<int64_t>(sup) + c) * kGemvTiles + tl) * p.n * 128 + r * 128 + i];
     start_c = start_next;
   }
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    if (r < p.n) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(acc[r]);
-      Y[static_cast<int64_t>(r) * ldy + col] = *reinterpret_cast<const uint16_t*>(&h);
-    }
-  }
+  const __nv_bfloat16 h = __float2bfloat16_rn(acc);
+  Y[static_cast<int64_t>(r) * ldy + col] = *reinterpret_cast<const uint16_t*>(&h);
 }
 
 }  // namespace rmm

@@ -346,7 +346,8 @@ rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint
   if (e != cudaSuccess) return cuda_fail(e, "decode attribute");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  gemv_fixup_kernel<<<static_cast<unsigned>(ceil_div(m, 128)), 128, 0, s>>>(g, grid, Y, ldy);
+  gemv_fixup_kernel<<<dim3(static_cast<unsigned>(ceil_div(m, 128)), static_cast<unsigned>(n)), 128, 0, s>>>(g, grid, Y,
+                                                                                                           ldy);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode fix-up launch");
   return RMM_OK;

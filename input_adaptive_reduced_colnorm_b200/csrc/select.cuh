@@ -168,21 +168,27 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
-      if (!((valid >> e) & 1u) || (hi[e] & msk_hi) != pre_hi) continue;
-      uint32_t dig;
-      if (shift >= 32) {
-        dig = (hi[e] >> (shift - 32)) & dmask;
-      } else {
-        const uint32_t lo = static_cast<uint32_t>(__double_as_longlong(q[j0 + e]));
-        if ((lo & msk_lo) != pre_lo) continue;
-        if (shift + width > 32) {  // digit straddles the two halves
-          const uint64_t full = (static_cast<uint64_t>(hi[e]) << 32) | lo;
-          dig = static_cast<uint32_t>(full >> shift) & dmask;
+      bool m = ((valid >> e) & 1u) && (hi[e] & msk_hi) == pre_hi;
+      uint32_t dig = 0;
+      if (m) {
+        if (shift >= 32) {
+          dig = (hi[e] >> (shift - 32)) & dmask;
         } else {
-          dig = (lo >> shift) & dmask;
+          const uint32_t lo = static_cast<uint32_t>(__double_as_longlong(q[j0 + e]));
+          m = (lo & msk_lo) == pre_lo;
+          if (shift + width > 32) {  // digit straddles the two halves
+            const uint64_t full = (static_cast<uint64_t>(hi[e]) << 32) | lo;
+            dig = static_cast<uint32_t>(full >> shift) & dmask;
+          } else {
+            dig = (lo >> shift) & dmask;
+          }
         }
       }
-      atomicAdd(&hist[dig], 1u);
+      // lanes with the same digit add once (keys crowd into few bins in the
+      // first pass, and same-address shared atomics serialise)
+      const uint32_t key = m ? dig : (0x10000u + lane);
+      const uint32_t grp = __match_any_sync(0xffffffffu, key);
+      if (m && lane == __ffs(grp) - 1) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(grp)));
     }
     __syncthreads();
     // descending suffix sums: bin b's "above" = count of larger digits
