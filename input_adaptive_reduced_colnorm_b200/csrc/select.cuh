@@ -184,11 +184,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
           }
         }
       }
-      // lanes with the same digit add once (keys crowd into few bins in the
-      // first pass, and same-address shared atomics serialise)
-      const uint32_t key = m ? dig : (0x10000u + lane);
-      const uint32_t grp = __match_any_sync(0xffffffffu, key);
-      if (m && lane == __ffs(grp) - 1) atomicAdd(&hist[dig], static_cast<uint32_t>(__popc(grp)));
+      if (m) atomicAdd(&hist[dig], 1u);
     }
     __syncthreads();
     // descending suffix sums: bin b's "above" = count of larger digits
