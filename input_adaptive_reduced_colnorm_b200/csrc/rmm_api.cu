@@ -89,6 +89,25 @@ rmm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t
   return RMM_OK;
 }
 
+// 3-D output map [batch][rows][cols] for the GEMM's TMA-store epilogue: boxes of
+// 32 rows x 128 bytes (32 fp32 or 64 bf16 columns), 128-byte swizzle; stores are
+// clipped to each batch item's rows and columns.
+rmm_status make_tmap_out(CUtensorMap* tm, const void* base, bool f32, uint64_t cols, uint64_t rows, uint64_t batch,
+                         uint64_t ld, uint64_t bstride) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(RMM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const uint64_t eb = f32 ? 4 : 2;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {ld * eb, (batch > 1 ? bstride : rows * ld) * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RMM_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+  return RMM_OK;
+}
+
 // ---------------------------------------------------------------- workspace carving
 struct Carver {
   uint8_t* base;
@@ -222,13 +241,18 @@ rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
 template <int BN, int BMODE, int EPI, int CAUSAL>
 rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t s) {
   auto kern = rmm_gemm_kernel<BN, BMODE, EPI, CAUSAL>;
+  CUtensorMap to;
+  if (rmm_status st = make_tmap_out(&to, p.out, EPI == kEpiF32, static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.M),
+                                    static_cast<uint64_t>(p.batch), static_cast<uint64_t>(p.ldo),
+                                    static_cast<uint64_t>(p.out_bstride)))
+    return st;
   constexpr int smem = GemmCfg<BN>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "gemm attribute");
   const int64_t tiles = static_cast<int64_t>(p.batch) * p.m_tiles * p.n_tiles;
   if (tiles > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many output tiles");
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
-  kern<<<grid, 192, smem, s>>>(ta, tb, p);
+  kern<<<grid, 192, smem, s>>>(ta, tb, to, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return RMM_OK;
