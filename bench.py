@@ -360,32 +360,67 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
     return out
 
 
+# ------------------------------------------------------------------ ranks
+class Ranks:
+    """Process-group plumbing of the weak-scaled benchmark: one process per GPU,
+    each timing its own replica; the only collectives are the barrier around the
+    timed region and the max over ranks of the measured times (no data-path
+    collective exists).  Works with NCCL on GPUs and with gloo on CPU (tests)."""
+
+    def __init__(self, world, rank, device=None, backend=None):
+        import torch
+        import torch.distributed as dist
+        self.world, self.rank, self.device = world, rank, device
+        self.dist = dist
+        self.on_cuda = device is not None and device.type == "cuda"
+        self.tensor_device = device if self.on_cuda else torch.device("cpu")
+        if world > 1 and not dist.is_initialized():
+            from datetime import timedelta
+            kw = {"device_id": device} if self.on_cuda else {}
+            dist.init_process_group(backend or ("nccl" if self.on_cuda else "gloo"), rank=rank, world_size=world,
+                                    timeout=timedelta(seconds=120), **kw)
+
+    def barrier(self):
+        import torch
+        if self.world > 1:
+            t = torch.zeros(1, device=self.tensor_device)
+            self.dist.all_reduce(t)
+        if self.on_cuda:
+            torch.cuda.synchronize(self.device)
+
+    def max(self, x):
+        """Max over ranks of a per-rank measurement (every rank gets it)."""
+        import torch
+        if self.world == 1:
+            return float(x)
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.tensor_device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1 and self.dist.is_initialized():
+            self.barrier()
+            self.dist.destroy_process_group()
+
+
+def weak_scaled_value(world, flops_per_rank, ms_max):
+    """Whole-job kept-FLOP throughput in TFLOP/s: every rank processed the same
+    per-rank work, divided by the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU leg
 def run_ours(args):
     import torch
-    import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            t = torch.zeros(1, device=dev)
-            dist.all_reduce(t)
-        torch.cuda.synchronize(dev)
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, rank, dev)
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     from input_adaptive_reduced_colnorm_b200 import build as rmm_build
     rmm_build.build()
@@ -502,7 +537,7 @@ def run_ours(args):
     # ---- numbers
     flops = step_flops(RHO_MAIN)
     nbytes = step_bytes(RHO_MAIN)
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = weak_scaled_value(world, flops, ms_step)
     peaks, peak_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
     gate = [i for i, b in enumerate(bufs) if b["name"] == "gate_proj"][0]
@@ -541,9 +576,7 @@ def run_ours(args):
         line["workloads"] = bench_workloads(dev, stream, L)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_rows)
-    if world > 1:
-        barrier()
-        dist.destroy_process_group()
+    ranks.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
