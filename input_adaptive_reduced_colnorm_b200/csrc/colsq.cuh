@@ -27,7 +27,7 @@ struct ColsqParams {
 };
 
 template <int TX, bool CAUSAL>
-__global__ void __launch_bounds__(256) colsq_kernel(const ColsqParams p) {
+__global__ void __launch_bounds__(256, 2) colsq_kernel(const ColsqParams p) {
   constexpr int TY = 256 / TX;
   constexpr int W = TX * 8;  // columns per strip
   __shared__ double red[TY][W + 1];
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) colsq_kernel(const ColsqParams p) {
   if (col0 < p.d) {
     const bool full = (col0 + 8 <= p.d);
     // bursts of U rows: all U 16-byte loads are in flight before any is used
-    constexpr int U = 8;
+    constexpr int U = 16;
     for (int64_t i = r_begin + ty; i < r_end; i += U * TY) {
       uint32_t w[U][4];
 #pragma unroll

@@ -125,12 +125,16 @@ __device__ __forceinline__ void pack_stage_async(uint16_t* buf, const uint16_t* 
   }
 }
 
-// Contiguous row range per CTA, double-buffered rows.  Dynamic shared memory:
-// 16-bit index offsets [k_pad] (0xFFFF marks padding) + two row buffers [d_round].
+// Contiguous row range per CTA; kPackBufs row buffers, so kPackBufs - 1 rows
+// are being copied (cp.async) while the current row is gathered.  Dynamic
+// shared memory: 16-bit index offsets [k_pad] (0xFFFF marks padding) +
+// kPackBufs row buffers [d_round].
+constexpr int kPackBufs = 4;
+
 __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, int64_t d_round, int64_t idx_elems) {
   extern __shared__ __align__(16) uint16_t pk_smem[];
   uint16_t* s_idx = pk_smem;
-  uint16_t* bufs[2] = {pk_smem + idx_elems, pk_smem + idx_elems + d_round};
+  uint16_t* bufs = pk_smem + idx_elems;
   const int64_t total = p.batch * p.rows;
   const int64_t per = (total + gridDim.x - 1) / gridDim.x;
   const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * per;
@@ -138,22 +142,30 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
   if (r_end > total) r_end = total;
   if (r_begin >= r_end) return;
 
-  int64_t b, i;
-  const uint16_t* src = pack_src_row(p, r_begin, b, i);
-  pack_stage_async(bufs[0], src, pack_visible(p, i), p.d);
-  cp_async_commit();
+  // prologue: the first kPackBufs - 1 rows (one commit group each, empty groups past the end)
+#pragma unroll
+  for (int q = 0; q < kPackBufs - 1; ++q) {
+    const int64_t r = r_begin + q;
+    if (r < r_end) {
+      int64_t b, i;
+      const uint16_t* src = pack_src_row(p, r, b, i);
+      pack_stage_async(bufs + q * d_round, src, pack_visible(p, i), p.d);
+    }
+    cp_async_commit();
+  }
   int64_t cur_b = -1;
   for (int64_t r = r_begin; r < r_end; ++r) {
     const int64_t rb = r / p.rows;
     const int64_t ri = r - rb * p.rows;
-    if (r + 1 < r_end) {
-      int64_t nb, ni;
-      const uint16_t* nsrc = pack_src_row(p, r + 1, nb, ni);
-      pack_stage_async(bufs[(r + 1 - r_begin) & 1], nsrc, pack_visible(p, ni), p.d);
+    {  // copy row r + kPackBufs - 1 into the buffer freed by row r - 1
+      const int64_t rn = r + kPackBufs - 1;
+      if (rn < r_end) {
+        int64_t nb, ni;
+        const uint16_t* nsrc = pack_src_row(p, rn, nb, ni);
+        pack_stage_async(bufs + ((rn - r_begin) % kPackBufs) * d_round, nsrc, pack_visible(p, ni), p.d);
+      }
       cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+      cp_async_wait<kPackBufs - 1>();  // row r's group has landed
     }
     if (rb != cur_b) {  // (re)load this batch item's index set as 16-bit offsets
       const int32_t* I = p.idx + rb * p.k;
@@ -173,7 +185,7 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
       cur_b = rb;
     }
     __syncthreads();
-    const uint16_t* row = bufs[(r - r_begin) & 1];
+    const uint16_t* row = bufs + ((r - r_begin) % kPackBufs) * d_round;
     const int64_t lim = pack_visible(p, ri);
     uint16_t* dst = p.dst + r * p.k_pad;
     for (int64_t t0 = static_cast<int64_t>(threadIdx.x) * 8; t0 < p.k_pad; t0 += 8 * blockDim.x) {
@@ -183,7 +195,7 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const uint32_t j0 = iw[h] & 0xFFFFu, j1 = iw[h] >> 16;
-        const uint32_t v0 = (j0 < lim) ? row[j0] : 0u;   // 0xFFFF padding is never < lim (d <= 32768)
+        const uint32_t v0 = (j0 < lim) ? row[j0] : 0u;  // 0xFFFF padding is never < lim (d <= 32768)
         const uint32_t v1 = (j1 < lim) ? row[j1] : 0u;
         w[h] = v0 | (v1 << 16);
       }
@@ -211,45 +223,50 @@ struct RowPackParams {
   int64_t g_outer, g_inner, s_outer, s_inner; // source item of b (as in PackParams)
 };
 
-// 2-D layout: 2^tpr_log2 threads per output row, 256 >> tpr_log2 rows per CTA;
-// each thread copies every (2^tpr_log2)-th 16-byte vector of its row.
+// 2-D layout: 2^tpr_log2 threads per output row, 256 >> tpr_log2 rows per CTA
+// pass, grid-stride over row groups; each thread copies every (2^tpr_log2)-th
+// 16-byte vector of its row, up to eight loads in flight.
 __global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackParams p, int tpr_log2) {
   constexpr int ILP = 8;
   const int tpr = 1 << tpr_log2;
+  const int rpg = 256 >> tpr_log2;
   const int tx = threadIdx.x & (tpr - 1);
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (256 >> tpr_log2) + (threadIdx.x >> tpr_log2);
-  if (row >= p.batch * p.rows_out) return;
-  const int64_t b = row / p.rows_out;
-  const int64_t t = row - b * p.rows_out;
-  uint16_t* dst = p.dst + row * p.dst_ld;
+  const int64_t total = p.batch * p.rows_out;
   const int vpr = static_cast<int>((p.cols + 7) / 8);
-  const uint16_t* src = nullptr;
-  if (t < p.k) {
-    const int64_t j = __ldg(p.idx + b * p.k + t);
-    const int64_t item = (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
-    src = p.src + item + j * p.src_ld;
-  }
   const bool full_tail = (p.cols % 8) == 0;
-  for (int c0 = tx; c0 < vpr; c0 += tpr * ILP) {
-    uint4 v[ILP];
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * rpg + (threadIdx.x >> tpr_log2); row < total;
+       row += static_cast<int64_t>(gridDim.x) * rpg) {
+    const int64_t b = row / p.rows_out;
+    const int64_t t = row - b * p.rows_out;
+    uint16_t* dst = p.dst + row * p.dst_ld;
+    const uint16_t* src = nullptr;
+    if (t < p.k) {
+      const int64_t j = __ldg(p.idx + b * p.k + t);
+      const int64_t item = (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+      src = p.src + item + j * p.src_ld;
+    }
+    for (int c0 = tx; c0 < vpr; c0 += tpr * ILP) {
+      uint4 v[ILP];
 #pragma unroll
-    for (int u = 0; u < ILP; ++u) {
-      const int c = c0 + u * tpr;
-      v[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (src != nullptr && c < vpr) {
-        if (full_tail || c + 1 < vpr) {
-          v[u] = ldg_nc_v4(src + c * 8);
-        } else {
-          uint32_t w[4] = {0u, 0u, 0u, 0u};
-          for (int e = 0; c * 8 + e < p.cols; ++e) w[e >> 1] |= static_cast<uint32_t>(__ldg(src + c * 8 + e)) << (16 * (e & 1));
-          v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int u = 0; u < ILP; ++u) {
+        const int c = c0 + u * tpr;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (src != nullptr && c < vpr) {
+          if (full_tail || c + 1 < vpr) {
+            v[u] = ldg_nc_v4(src + c * 8);
+          } else {
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            for (int e = 0; c * 8 + e < p.cols; ++e)
+              w[e >> 1] |= static_cast<uint32_t>(__ldg(src + c * 8 + e)) << (16 * (e & 1));
+            v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < ILP; ++u) {
-      const int c = c0 + u * tpr;
-      if (c < vpr) *reinterpret_cast<uint4*>(dst + c * 8) = v[u];
+      for (int u = 0; u < ILP; ++u) {
+        const int c = c0 + u * tpr;
+        if (c < vpr) *reinterpret_cast<uint4*>(dst + c * 8) = v[u];
+      }
     }
   }
 }

@@ -126,11 +126,28 @@ struct Carver {
 // ---------------------------------------------------------------- launches
 rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64_t n, int64_t d, int64_t lda,
                         bool causal, int64_t off, double* colsq, cudaStream_t s) {
-  int C = 1;
-  while (C < 8 && n / (2 * C) >= 128) C *= 2;
-  const int64_t target = 2LL * num_sms();
-  int TX = 32;
-  while (TX > 4 && ceil_div(d, TX * 8) * batch * C < target) TX /= 2;
+  // Pick the strip width (TX threads x 8 columns) and the cluster size C (CTAs
+  // splitting a strip's rows) so that the grid fits in one wave of two CTAs per
+  // SM with as many CTAs as possible; larger problems simply take several waves.
+  const int64_t wave = 2LL * num_sms();
+  int C = 0, TX = 0;
+  int64_t best = 0;
+  for (int tx = 32; tx >= 4; tx /= 2) {
+    for (int c = 1; c <= 8; c *= 2) {
+      if (c > 1 && n / c < 64) break;  // keep at least 64 rows per CTA
+      const int64_t ctas = ceil_div(d, tx * 8) * batch * c;
+      if (ctas <= wave && ctas > best) {
+        best = ctas;
+        C = c;
+        TX = tx;
+      }
+    }
+  }
+  if (best == 0) {  // even the smallest grid exceeds one wave: widest strips, full clusters
+    TX = 32;
+    C = 1;
+    while (C < 8 && n / (2 * C) >= 128) C *= 2;
+  }
   const int64_t strips = ceil_div(d, TX * 8);
   if (strips * C > kIntMax || batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "column-norm grid too large");
   ColsqParams p{};
@@ -210,14 +227,14 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
     pack_rows_warp_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round);
   } else {
     const int64_t idx_elems = round_up(p.k_pad, 8);
-    const size_t smem = static_cast<size_t>((idx_elems + 2 * d_round) * 2);
-    if (smem > 48 * 1024) {
-      e = cudaFuncSetAttribute(pack_rows_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-      if (e != cudaSuccess) return cuda_fail(e, "pack attribute");
-    }
-    const int64_t per_sm = std::max<int64_t>(1, std::min<int64_t>(8, (200 * 1024) / static_cast<int64_t>(smem)));
-    const int64_t grid = std::min<int64_t>(rows, per_sm * num_sms());
+    const size_t smem = static_cast<size_t>((idx_elems + kPackBufs * d_round) * 2);
+    if (smem > 227 * 1024) return fail(RMM_ERR_UNSUPPORTED, "row too long for the pack kernel");
+    e = cudaFuncSetAttribute(pack_rows_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "pack attribute");
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_rows_cta_kernel, 256, smem);
+    if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+    const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * num_sms());
     pack_rows_cta_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round, idx_elems);
   }
   e = cudaGetLastError();
@@ -226,12 +243,14 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
 }
 
 rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
+  // threads per row: a power of two with at least 8 vectors per thread where the
+  // rows are long enough, so each thread keeps several 16-byte loads in flight
   const int64_t vpr = (p.cols + 7) / 8;
   int tpr_log2 = 0;
-  while ((1LL << tpr_log2) < vpr && tpr_log2 < 8) ++tpr_log2;
+  while ((1LL << tpr_log2) < 256 && (1LL << (tpr_log2 + 1)) * 8 <= vpr) ++tpr_log2;
   const int64_t rows = p.batch * p.rows_out;
-  const int64_t grid = ceil_div(rows, 256 >> tpr_log2);
-  if (grid > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "row pack grid too large");
+  const int64_t groups = ceil_div(rows, 256 >> tpr_log2);
+  const int64_t grid = std::min<int64_t>(groups, 4LL * num_sms());
   pack_rows_gather_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p, tpr_log2);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "row pack launch");
