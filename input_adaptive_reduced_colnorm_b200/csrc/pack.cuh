@@ -125,12 +125,32 @@ __device__ __forceinline__ void pack_stage_async(uint16_t* buf, const uint16_t* 
   }
 }
 
-// Contiguous row range per CTA; kPackBufs row buffers, so kPackBufs - 1 rows
-// are being copied (cp.async) while the current row is gathered.  Dynamic
-// shared memory: 16-bit index offsets [k_pad] (0xFFFF marks padding) +
-// kPackBufs row buffers [d_round].
-constexpr int kPackBufs = 4;
+// Contiguous row range per CTA; NBUF row buffers, so NBUF - 1 rows are being
+// copied (cp.async) while the current row is gathered.  Dynamic shared memory:
+// 16-bit index offsets [k_pad] (0xFFFF marks padding) + NBUF row buffers
+// [d_round].  The batch item of a row is tracked incrementally (integer
+// divisions only when the item changes).
+struct PackCursor {
+  int64_t b, i;          // batch item, row within it
+  const uint16_t* base;  // source item base
+  __device__ void init(const PackParams& p, int64_t r) {
+    b = r / p.rows;
+    i = r - b * p.rows;
+    set_base(p);
+  }
+  __device__ void set_base(const PackParams& p) {
+    base = p.src + (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+  }
+  __device__ void next(const PackParams& p) {
+    if (++i == p.rows) {
+      i = 0;
+      ++b;
+      set_base(p);
+    }
+  }
+};
 
+template <int NBUF>
 __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, int64_t d_round, int64_t idx_elems) {
   extern __shared__ __align__(16) uint16_t pk_smem[];
   uint16_t* s_idx = pk_smem;
@@ -141,54 +161,56 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
   int64_t r_end = r_begin + per;
   if (r_end > total) r_end = total;
   if (r_begin >= r_end) return;
+  const int nrows = static_cast<int>(r_end - r_begin);
+  const int k_pad = static_cast<int>(p.k_pad);
 
-  // prologue: the first kPackBufs - 1 rows (one commit group each, empty groups past the end)
+  PackCursor stage_at, gather_at;
+  stage_at.init(p, r_begin);
+  gather_at = stage_at;
+  // prologue: the first NBUF - 1 rows (one commit group each, empty groups past the end)
 #pragma unroll
-  for (int q = 0; q < kPackBufs - 1; ++q) {
-    const int64_t r = r_begin + q;
-    if (r < r_end) {
-      int64_t b, i;
-      const uint16_t* src = pack_src_row(p, r, b, i);
-      pack_stage_async(bufs + q * d_round, src, pack_visible(p, i), p.d);
+  for (int q = 0; q < NBUF - 1; ++q) {
+    if (q < nrows) {
+      pack_stage_async(bufs + q * d_round, stage_at.base + stage_at.i * p.src_ld, pack_visible(p, stage_at.i), p.d);
+      stage_at.next(p);
     }
     cp_async_commit();
   }
   int64_t cur_b = -1;
-  for (int64_t r = r_begin; r < r_end; ++r) {
-    const int64_t rb = r / p.rows;
-    const int64_t ri = r - rb * p.rows;
-    {  // copy row r + kPackBufs - 1 into the buffer freed by row r - 1
-      const int64_t rn = r + kPackBufs - 1;
-      if (rn < r_end) {
-        int64_t nb, ni;
-        const uint16_t* nsrc = pack_src_row(p, rn, nb, ni);
-        pack_stage_async(bufs + ((rn - r_begin) % kPackBufs) * d_round, nsrc, pack_visible(p, ni), p.d);
+  for (int q = 0; q < nrows; ++q) {
+    {  // copy row q + NBUF - 1 into the buffer freed by row q - 1
+      const int qn = q + NBUF - 1;
+      if (qn < nrows) {
+        pack_stage_async(bufs + (qn % NBUF) * d_round, stage_at.base + stage_at.i * p.src_ld,
+                         pack_visible(p, stage_at.i), p.d);
+        stage_at.next(p);
       }
       cp_async_commit();
-      cp_async_wait<kPackBufs - 1>();  // row r's group has landed
+      cp_async_wait<NBUF - 1>();  // row q's group has landed
     }
-    if (rb != cur_b) {  // (re)load this batch item's index set as 16-bit offsets
-      const int32_t* I = p.idx + rb * p.k;
-      for (int64_t t0 = threadIdx.x; t0 < p.k_pad; t0 += 8 * static_cast<int64_t>(blockDim.x)) {
+    if (gather_at.b != cur_b) {  // (re)load this batch item's index set as 16-bit offsets
+      const int32_t* I = p.idx + gather_at.b * p.k;
+      const int k = static_cast<int>(p.k);
+      for (int t0 = threadIdx.x; t0 < k_pad; t0 += 8 * blockDim.x) {
         int32_t v[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {  // eight loads in flight per thread
-          const int64_t t = t0 + e * static_cast<int64_t>(blockDim.x);
-          v[e] = (t < p.k) ? __ldg(I + t) : 0xFFFF;
+          const int t = t0 + e * blockDim.x;
+          v[e] = (t < k) ? __ldg(I + t) : 0xFFFF;
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int64_t t = t0 + e * static_cast<int64_t>(blockDim.x);
-          if (t < p.k_pad) s_idx[t] = static_cast<uint16_t>(v[e]);
+          const int t = t0 + e * blockDim.x;
+          if (t < k_pad) s_idx[t] = static_cast<uint16_t>(v[e]);
         }
       }
-      cur_b = rb;
+      cur_b = gather_at.b;
     }
     __syncthreads();
-    const uint16_t* row = bufs + ((r - r_begin) % kPackBufs) * d_round;
-    const int64_t lim = pack_visible(p, ri);
-    uint16_t* dst = p.dst + r * p.k_pad;
-    for (int64_t t0 = static_cast<int64_t>(threadIdx.x) * 8; t0 < p.k_pad; t0 += 8 * blockDim.x) {
+    const uint16_t* row = bufs + (q % NBUF) * d_round;
+    const uint32_t lim = static_cast<uint32_t>(pack_visible(p, gather_at.i));
+    uint16_t* dst = p.dst + (r_begin + q) * p.k_pad;
+    for (int t0 = threadIdx.x * 8; t0 < k_pad; t0 += 8 * blockDim.x) {
       const uint4 iv = *reinterpret_cast<const uint4*>(s_idx + t0);
       const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
       uint32_t w[4];
@@ -201,6 +223,7 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
       }
       *reinterpret_cast<uint4*>(dst + t0) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    gather_at.next(p);
     __syncthreads();
   }
 }

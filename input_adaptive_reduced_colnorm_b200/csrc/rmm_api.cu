@@ -226,16 +226,19 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
     const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), 8LL * num_sms());
     pack_rows_warp_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round);
   } else {
+    // four row buffers for rows up to 8192 columns, two beyond (more CTAs per SM)
     const int64_t idx_elems = round_up(p.k_pad, 8);
-    const size_t smem = static_cast<size_t>((idx_elems + kPackBufs * d_round) * 2);
+    const int nbuf = (d_round <= 8192) ? 4 : 2;
+    const size_t smem = static_cast<size_t>((idx_elems + nbuf * d_round) * 2);
     if (smem > 227 * 1024) return fail(RMM_ERR_UNSUPPORTED, "row too long for the pack kernel");
-    e = cudaFuncSetAttribute(pack_rows_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    auto kern = (nbuf == 4) ? pack_rows_cta_kernel<4> : pack_rows_cta_kernel<2>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e, "pack attribute");
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_rows_cta_kernel, 256, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
     if (e != cudaSuccess || per_sm < 1) per_sm = 1;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * num_sms());
-    pack_rows_cta_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round, idx_elems);
+    kern<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round, idx_elems);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
