@@ -28,6 +28,7 @@ struct ColsqParams {
 
 template <int TX, bool CAUSAL>
 __global__ void __launch_bounds__(256, 2) colsq_kernel(const ColsqParams p) {
+  wait_prior_kernels();
   constexpr int TY = 256 / TX;
   constexpr int W = TX * 8;  // columns per strip
   __shared__ double red[TY][W + 1];

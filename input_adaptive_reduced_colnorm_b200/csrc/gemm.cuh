@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = p.batch * p.m_tiles * p.n_tiles;
+  wait_prior_kernels();  // operands and the output buffer are touched only after this
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

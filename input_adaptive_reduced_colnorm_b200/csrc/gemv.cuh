@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  wait_prior_kernels();  // operands and partials are touched only after this
 
   const int64_t G = gridDim.x;
   const int64_t u_begin = gemv_unit_begin(blockIdx.x, p.units, G);
@@ -314,6 +315,7 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
 // increasing c, of their partial sums ).  One thread per (output column, row r =
 // blockIdx.y); the owning CTAs are found from the same unit split as the kernel.
 __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy) {
+  wait_prior_kernels();
   const int col = blockIdx.x * 128 + threadIdx.x;
   const int r = blockIdx.y;
   if (col >= p.m) return;

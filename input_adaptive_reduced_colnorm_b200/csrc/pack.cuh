@@ -69,6 +69,7 @@ __device__ __forceinline__ void pack_stage(uint16_t* buf, const uint16_t* src, i
 
 // one row per warp; dynamic shared memory: 8 warps x d_round bf16
 __global__ void __launch_bounds__(256) pack_rows_warp_kernel(const PackParams p, int64_t d_round) {
+  wait_prior_kernels();
   extern __shared__ __align__(16) uint16_t pk_smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint16_t* buf = pk_smem + warp * d_round;
@@ -152,6 +153,7 @@ struct PackCursor {
 
 template <int NBUF>
 __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, int64_t d_round, int64_t idx_elems) {
+  wait_prior_kernels();
   extern __shared__ __align__(16) uint16_t pk_smem[];
   uint16_t* s_idx = pk_smem;
   uint16_t* bufs = pk_smem + idx_elems;
@@ -250,6 +252,7 @@ struct RowPackParams {
 // pass, grid-stride over row groups; each thread copies every (2^tpr_log2)-th
 // 16-byte vector of its row, up to eight loads in flight.
 __global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackParams p, int tpr_log2) {
+  wait_prior_kernels();
   constexpr int ILP = 8;
   const int tpr = 1 << tpr_log2;
   const int rpg = 256 >> tpr_log2;

@@ -39,6 +39,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- launch chaining
+// Every kernel of the library is launched with programmatic stream
+// serialisation, so it may start while the previous kernel on the stream is
+// finishing.  It runs only its private prologue (barriers, tensor memory,
+// descriptor prefetch) before this wait, which returns once the previous
+// kernel has completed and its memory operations are visible; as every kernel
+// waits, all earlier kernels on the stream are complete past this point.
+__device__ __forceinline__ void wait_prior_kernels() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

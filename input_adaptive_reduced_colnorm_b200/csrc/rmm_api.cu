@@ -108,6 +108,23 @@ rmm_status make_tmap_out(CUtensorMap* tm, const void* base, bool f32, uint64_t c
   return RMM_OK;
 }
 
+// Launch with programmatic stream serialisation (see wait_prior_kernels()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------- workspace carving
 struct Carver {
   uint8_t* base;
@@ -166,13 +183,15 @@ rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaSuccess;
 #define RMM_COLSQ_CASE(tx)                                                          \
   case tx:                                                                          \
@@ -199,8 +218,7 @@ rmm_status launch_select_t(const SelectParams& p, int64_t batch, cudaStream_t s)
                                                static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_fail(e, "select attribute");
   }
-  select_kernel<KPT, NT><<<static_cast<unsigned>(batch), NT, smem, s>>>(p);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_chained(select_kernel<KPT, NT>, dim3(static_cast<unsigned>(batch)), dim3(NT), smem, s, p);
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   return RMM_OK;
 }
@@ -224,7 +242,8 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
   if (p.d <= 1024) {
     const size_t smem = static_cast<size_t>(8 * d_round * 2);
     const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), 8LL * num_sms());
-    pack_rows_warp_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round);
+    e = launch_chained(pack_rows_warp_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), smem, s, p, d_round);
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
   } else {
     // four row buffers for rows up to 8192 columns, two beyond (more CTAs per SM)
     const int64_t idx_elems = round_up(p.k_pad, 8);
@@ -238,7 +257,8 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
     if (e != cudaSuccess || per_sm < 1) per_sm = 1;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * num_sms());
-    kern<<<static_cast<unsigned>(grid), 256, smem, s>>>(p, d_round, idx_elems);
+    e = launch_chained(kern, dim3(static_cast<unsigned>(grid)), dim3(256), smem, s, p, d_round, idx_elems);
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
@@ -254,8 +274,7 @@ rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
   const int64_t rows = p.batch * p.rows_out;
   const int64_t groups = ceil_div(rows, 256 >> tpr_log2);
   const int64_t grid = std::min<int64_t>(groups, 4LL * num_sms());
-  pack_rows_gather_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(p, tpr_log2);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_chained(pack_rows_gather_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p, tpr_log2);
   if (e != cudaSuccess) return cuda_fail(e, "row pack launch");
   return RMM_OK;
 }
@@ -274,8 +293,7 @@ rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmP
   const int64_t tiles = static_cast<int64_t>(p.batch) * p.m_tiles * p.n_tiles;
   if (tiles > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many output tiles");
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
-  kern<<<grid, 192, smem, s>>>(ta, tb, to, p);
-  e = cudaGetLastError();
+  e = launch_chained(kern, dim3(grid), dim3(192), smem, s, ta, tb, to, p);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return RMM_OK;
 }
@@ -384,17 +402,14 @@ rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint
   cudaError_t e;
   if (N == 16) {
     e = cudaFuncSetAttribute(gemv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) gemv_kernel<16><<<grid, 288, smem, s>>>(tx, g);
+    if (e == cudaSuccess) e = launch_chained(gemv_kernel<16>, dim3(grid), dim3(288), smem, s, tx, g);
   } else {
     e = cudaFuncSetAttribute(gemv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) gemv_kernel<32><<<grid, 288, smem, s>>>(tx, g);
+    if (e == cudaSuccess) e = launch_chained(gemv_kernel<32>, dim3(grid), dim3(288), smem, s, tx, g);
   }
-  if (e != cudaSuccess) return cuda_fail(e, "decode attribute");
-  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  gemv_fixup_kernel<<<dim3(static_cast<unsigned>(ceil_div(m, 128)), static_cast<unsigned>(n)), 128, 0, s>>>(g, grid, Y,
-                                                                                                           ldy);
-  e = cudaGetLastError();
+  e = launch_chained(gemv_fixup_kernel, dim3(static_cast<unsigned>(ceil_div(m, 128)), static_cast<unsigned>(n)),
+                     dim3(128), 0, s, g, grid, Y, ldy);
   if (e != cudaSuccess) return cuda_fail(e, "decode fix-up launch");
   return RMM_OK;
 }
@@ -589,8 +604,7 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
     if (k == d) {
       float* partial = c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
       if (idx_out != nullptr) {
-        iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024)), 256, 0, s>>>(idx_out, 1, d);
-        const cudaError_t e = cudaGetLastError();
+        const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024))), dim3(256), 0, s, idx_out, 1, d);
         if (e != cudaSuccess) return cuda_fail(e, "iota launch");
       }
       return decode_product(A, n, lda, B, d, m, ldb, nullptr, partial, Y, ldy, s);
@@ -609,8 +623,7 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
   if (k == d) {
     // rho = 1: the dense product, I = [0, d)
     if (idx_out != nullptr) {
-      iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024)), 256, 0, s>>>(idx_out, 1, d);
-      const cudaError_t e = cudaGetLastError();
+      const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024))), dim3(256), 0, s, idx_out, 1, d);
       if (e != cudaSuccess) return cuda_fail(e, "iota launch");
     }
     return gemm_packed(A, n, d, lda, B, m, ldb, Y, ldy, s);
@@ -730,9 +743,7 @@ rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch,
     g.b_s_outer = hkv * nk;
     g.b_s_inner = nk;
     if (idx_out != nullptr) {
-      iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(items * dh, 256), 1024)), 256, 0, s>>>(
-          idx_out, items, dh);
-      const cudaError_t e = cudaGetLastError();
+      const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(items * dh, 256), 1024))), dim3(256), 0, s, idx_out, items, dh);
       if (e != cudaSuccess) return cuda_fail(e, "iota launch");
     }
   } else {
@@ -842,9 +853,7 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
     g.num_kb = static_cast<int>(ceil_div(nk, 64));
     g.idx = nullptr;
     if (idx_out != nullptr) {
-      iota_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(items * nk, 256), 4096)), 256, 0, s>>>(
-          idx_out, items, nk);
-      const cudaError_t e = cudaGetLastError();
+      const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(items * nk, 256), 4096))), dim3(256), 0, s, idx_out, items, nk);
       if (e != cudaSuccess) return cuda_fail(e, "iota launch");
     }
   } else {

@@ -79,6 +79,7 @@ __device__ __forceinline__ double block_sum_f64(double v, double* s_buf) {
 // dynamic shared memory: hi32 keys [NT * KPT] (uint32)
 template <int KPT, int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
+  wait_prior_kernels();
   constexpr int NW = NT / 32;
   constexpr int BPT = kSelBins / NT;  // histogram bins scanned per thread
   static_assert(kSelBins % NT == 0, "bins must split evenly");
@@ -280,6 +281,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
 
 // I = [0, d) for the rho = 1 path when the caller asks for the index set.
 __global__ void iota_kernel(int32_t* idx, int64_t batch, int64_t d) {
+  wait_prior_kernels();
   const int64_t total = batch * d;
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x)
