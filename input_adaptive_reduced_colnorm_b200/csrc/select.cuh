@@ -13,8 +13,7 @@
 //   * the low 32 bits are fetched from global memory only for keys that still
 //     tie on the top 32 bits (exact or near-exact ties);
 //   * a pass stops early as soon as the bucket holding the k-th key is taken
-//     whole; once that bucket holds at most kSelCandMax keys (usually after the
-//     first pass) its keys are ranked exactly against each other instead.
+//     whole.
 // The final compaction is two block-wide prefix scans in index order, which
 // gives the lower-index tie rule and the ascending order without any sort.
 // All counts are integers, so the result does not depend on atomic ordering.
@@ -33,8 +32,6 @@ struct SelectParams {
 
 constexpr int kSelBits = 12;
 constexpr int kSelBins = 1 << kSelBits;
-constexpr int kSelCandMax = 512;   // threshold buckets this small are resolved by exact ranks
-constexpr int kSelMaxD = 32768;
 
 template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* s_total) {
@@ -93,10 +90,6 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   __shared__ int s_digit, s_above, s_cnt;
   __shared__ uint32_t s_and[32], s_or[32];
   __shared__ double s_sum[32];
-  __shared__ int s_ncand;
-  __shared__ int s_cand[kSelCandMax];                 // candidate indices (threshold bucket)
-  __shared__ unsigned long long s_ckey[kSelCandMax];  // their full 64-bit keys
-  __shared__ uint32_t s_bits[kSelMaxD / 32];          // chosen candidates, one bit per index
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t b = blockIdx.x;
@@ -167,7 +160,6 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   }
   // bit cursor: position (in the 64-bit key) just above the next digit
   int cursor = 32 + ((msk_hi == 0xffffffffu) ? 0 : (32 - __popc(msk_hi)));
-  bool use_rank = false;
 
   while (!take_bucket && cursor > 0) {
     const int width = cursor >= kSelBits ? kSelBits : cursor;
@@ -229,38 +221,6 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
     msk_lo |= static_cast<uint32_t>(dm);
     if (s_cnt == need) take_bucket = true;
     cursor = shift;
-    if (!take_bucket && s_cnt <= kSelCandMax) use_rank = true;
-    if (threadIdx.x == 0) s_ncand = 0;
-    __syncthreads();
-    if (use_rank) break;
-  }
-
-  if (use_rank) {
-    // The bucket holding the k-th key has at most kSelCandMax keys: collect
-    // them with their full keys, and keep the `need` best by exact rank (key
-    // descending, index ascending -- the lower index wins ties).
-    for (int w = threadIdx.x; w < (d + 31) / 32; w += NT) s_bits[w] = 0u;
-#pragma unroll
-    for (int e = 0; e < KPT; ++e) {
-      if (!((valid >> e) & 1u) || (hi[e] & msk_hi) != pre_hi) continue;
-      const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(q[j0 + e]));
-      if ((static_cast<uint32_t>(key) & msk_lo) != pre_lo) continue;
-      const int slot = atomicAdd(&s_ncand, 1);
-      s_cand[slot] = j0 + e;
-      s_ckey[slot] = key;
-    }
-    __syncthreads();
-    const int c = s_ncand;
-    for (int sl = threadIdx.x; sl < c; sl += NT) {
-      const unsigned long long ks = s_ckey[sl];
-      const int js = s_cand[sl];
-      int r = 0;
-      for (int s2 = 0; s2 < c; ++s2) {
-        const unsigned long long k2 = s_ckey[s2];
-        r += (k2 > ks) || (k2 == ks && s_cand[s2] < js);
-      }
-      if (r < need) atomicOr(&s_bits[js >> 5], 1u << (js & 31));
-    }
     __syncthreads();
   }
 
@@ -285,10 +245,6 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   uint32_t sel = gt;
   if (take_bucket) {
     sel |= eq;
-  } else if (use_rank) {
-#pragma unroll
-    for (int e = 0; e < KPT; ++e)
-      if (((eq >> e) & 1u) && ((s_bits[(j0 + e) >> 5] >> ((j0 + e) & 31)) & 1u)) sel |= 1u << e;
   } else {
     // keep the first `need` bucket members in index order
     const int before = block_exclusive_scan<NT>(__popc(eq), s_warp, &s_total);
