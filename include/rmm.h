@@ -168,6 +168,9 @@ rmm_status rmm_gemm_packed(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t
  *   S  device fp32 [batch][Hq][nq][nk], contiguous.  With causal = 1, entries
  *      with key j > i + (nk - nq) are -inf (bottom-right alignment).
  *   idx_out device int32 [batch][Hq][k] or NULL, k = rmm_k(rho, dh).
+ * The product is bound by writing S, so the dropped head dims are zeroed in a
+ * per-head copy of Q (workspace) and the tensor-core GEMM reads K as it is:
+ * the result is exactly the reduced product.
  * Requires Hq % Hkv == 0, dh % 8 == 0, nk % 4 == 0, dh <= 32768. */
 size_t rmm_qk_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh,
                               double rho);
@@ -183,8 +186,11 @@ rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch,
  *   V  device bf16 [batch][Hkv][nk][dh], contiguous.
  *   O  device bf16 [batch][H][nq][dh], contiguous.
  *   causal = 1 treats P[i, j] with j > i + (nk - nq) as zero: those entries are
- *   neither read for the scores nor multiplied.
+ *   not read for the scores and are zeroed before any product uses them.
  *   idx_out device int32 [batch][H][k] or NULL, k = rmm_k(rho, nk).
+ * The product is bound by reading P, so the V rows of dropped positions are
+ * zeroed in a per-head copy of V (workspace) and P is streamed once by the
+ * tensor-core GEMM: the result is exactly the reduced product.
  * Requires H % Hkv == 0, nk % 8 == 0, dh == 64 or 128, nk <= 32768. */
 size_t rmm_pv_workspace_bytes(int64_t batch, int64_t h, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, double rho);
 rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t batch, int64_t h, int64_t hkv,

@@ -66,6 +66,7 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
   static constexpr int EPI_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 chunks of 32 rows x 128 bytes
   static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + EPI_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(8 * (3 * STAGES + 5) + 8 <= 256, "barrier area");
 };
 
 __device__ __forceinline__ int64_t gemm_b_row_base(const GemmParams& p, int b) {
@@ -99,6 +100,40 @@ __device__ __forceinline__ int gemm_tile_kb(const GemmParams& p, int b, int m0, 
   return p.num_kb;
 }
 
+// Causal PV: does k-block kb of the M tile at m0 hold entries above the
+// diagonal (key j > row i + causal_off) for some row?  Those A tiles are masked
+// in shared memory before the MMA reads them.
+template <int CAUSAL>
+__device__ __forceinline__ bool gemm_diag_block(const GemmParams& p, int m0, int kb) {
+  return CAUSAL == kCausalLimitK &&
+         static_cast<int64_t>(kb) * 64 + 63 > static_cast<int64_t>(m0) + p.causal_off;
+}
+
+// Zero A-tile entries (row r, column c) with 64 kb + c > m0 + r + causal_off;
+// 32 lanes, four rows each, 128-byte-swizzled K-major layout.
+__device__ __forceinline__ void gemm_mask_diag(uint8_t* tileA, const GemmParams& p, int m0, int kb, int lane) {
+  for (int r = lane; r < 128; r += 32) {
+    const int64_t lim = static_cast<int64_t>(m0) + r + p.causal_off - static_cast<int64_t>(kb) * 64;  // last visible column
+    if (lim >= 63) continue;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c_lo = u * 8;
+      if (c_lo + 7 <= lim) continue;
+      uint4* ptr = reinterpret_cast<uint4*>(tileA + r * 128 + ((u ^ (r & 7)) << 4));
+      if (c_lo > lim) {
+        *ptr = make_uint4(0u, 0u, 0u, 0u);
+      } else {
+        uint4 v = *ptr;
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (c_lo + e > lim) w[e >> 1] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+        *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
+
 // Tile order: batch item, then N tile, then M tile fastest, so CTAs running at
 // the same time share B column blocks in L2.
 __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& b, int& m0, int& nt) {
@@ -127,7 +162,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ready = drain + 1;  // [STAGES]: diagonal A tiles masked (causal PV)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -141,6 +177,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[a], 128);
     }
     mbar_init(drain, 1);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&ready[st], 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tmA);
@@ -192,6 +229,20 @@ __global__ void __launch_bounds__(192, 1)
           if (lane == 0) tma_load_2d(dstB, &tmB, &full[stage], kb * 64, static_cast<int32_t>(brow0 + n0));
         }
         __syncwarp();
+        if (gemm_diag_block<CAUSAL>(p, m0, kb)) {
+          // let this stage land, zero its entries above the diagonal, then release it to the MMA
+          int landed = 1;
+          if (lane == 0) landed = mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+          landed = __shfl_sync(0xffffffffu, landed, 0);
+          if (!landed) {
+            ok = false;
+            break;
+          }
+          gemm_mask_diag(sA + stage * C::A_BYTES, p, m0, kb, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ready[stage]);
+        }
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -216,6 +267,7 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t ready_phase = 0;  // one parity bit per stage for the `ready` barriers
       int acc_i = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
@@ -232,7 +284,14 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma)) {
+          bool got;
+          if (gemm_diag_block<CAUSAL>(p, m0, kb)) {
+            got = mbar_wait(&ready[stage], (ready_phase >> stage) & 1u, abort_flag, kDevErrTimeoutMma);
+            ready_phase ^= 1u << stage;
+          } else {
+            got = mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma);
+          }
+          if (!got) {
             ok = false;
             break;
           }

@@ -297,4 +297,70 @@ __global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackPara
   }
 }
 
+// Masked copy: the dropped contraction terms set to zero instead of skipped.
+// For QK^T (keep indexes the columns of Q_h: head-feature dims) and PV (keep
+// indexes the rows of V_g(h): token positions) the product is bound by writing
+// S or reading P, so skipping the dropped terms saves no time; zeroing them
+// gives exactly sum_{j in I} A[:, j] B[j, :] with no packed copies.
+//   dst[b][r, c] = keep_b[by_rows ? r : c] ? src_item(b)[r, c] : 0
+struct MaskParams {
+  const uint16_t* src;
+  uint16_t* dst;
+  int64_t rows, cols;                          // per batch item (cols % 8 == 0)
+  const uint8_t* keep;                         // [batch][by_rows ? rows : cols]
+  int by_rows;
+  int64_t batch;
+  int64_t g_outer, g_inner, s_outer, s_inner;  // source item of b (as in PackParams)
+};
+
+__global__ void __launch_bounds__(256) mask_copy_kernel(const MaskParams p) {
+  wait_prior_kernels();
+  constexpr int ILP = 4;
+  const int64_t vpr = p.cols / 8;
+  const int64_t total = p.batch * p.rows * vpr;
+  const int64_t keep_len = p.by_rows ? p.rows : p.cols;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v0 < total; v0 += ILP * stride) {
+    uint4 val[ILP];
+    int64_t dst_off[ILP];
+#pragma unroll
+    for (int u = 0; u < ILP; ++u) {
+      const int64_t v = v0 + u * stride;
+      dst_off[u] = -1;
+      val[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (v < total) {
+        const int64_t row_g = v / vpr;  // row over all batch items
+        const int64_t c8 = (v - row_g * vpr) * 8;
+        const int64_t b = row_g / p.rows;
+        const int64_t r = row_g - b * p.rows;
+        dst_off[u] = row_g * p.cols + c8;
+        const uint8_t* kb = p.keep + b * keep_len;
+        const uint16_t* src =
+            p.src + (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner + r * p.cols + c8;
+        if (p.by_rows) {
+          if (__ldg(kb + r)) val[u] = ldg_nc_v4(src);
+        } else {
+          const uint2 kk = *reinterpret_cast<const uint2*>(kb + c8);  // eight keep bytes
+          if (kk.x | kk.y) {
+            const uint4 x = ldg_nc_v4(src);
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+            const uint32_t ks[2] = {kk.x, kk.y};
+            uint32_t o[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const uint32_t kw = ks[h >> 1] >> (16 * (h & 1));  // keep bytes of elements 2h, 2h+1
+              const uint32_t m = ((kw & 0xFFu) ? 0x0000FFFFu : 0u) | ((kw & 0xFF00u) ? 0xFFFF0000u : 0u);
+              o[h] = xs[h] & m;
+            }
+            val[u] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < ILP; ++u)
+      if (dst_off[u] >= 0) *reinterpret_cast<uint4*>(p.dst + dst_off[u]) = val[u];
+  }
+}
+
 }  // namespace rmm

@@ -224,8 +224,8 @@ rmm_status launch_select_t(const SelectParams& p, int64_t batch, cudaStream_t s)
 }
 
 rmm_status launch_select(const double* colsq, int64_t batch, int64_t d, int64_t k, int32_t* idx, double* retained,
-                         cudaStream_t s) {
-  SelectParams p{colsq, d, k, idx, retained};
+                         cudaStream_t s, uint8_t* keep = nullptr) {
+  SelectParams p{colsq, d, k, idx, retained, keep};
   if (d <= 128) return launch_select_t<1, 128>(p, batch, s);
   if (d <= 1024) return launch_select_t<1, 1024>(p, batch, s);
   if (d <= 2048) return launch_select_t<2, 1024>(p, batch, s);
@@ -276,6 +276,14 @@ rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
   const int64_t grid = std::min<int64_t>(groups, 4LL * num_sms());
   const cudaError_t e = launch_chained(pack_rows_gather_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p, tpr_log2);
   if (e != cudaSuccess) return cuda_fail(e, "row pack launch");
+  return RMM_OK;
+}
+
+rmm_status launch_mask(const MaskParams& p, cudaStream_t s) {
+  const int64_t total = p.batch * p.rows * (p.cols / 8);
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256 * 4), 8LL * num_sms()));
+  const cudaError_t e = launch_chained(mask_copy_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p);
+  if (e != cudaSuccess) return cuda_fail(e, "mask launch");
   return RMM_OK;
 }
 
@@ -687,16 +695,16 @@ rmm_status rmm_gemm_packed(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t
 size_t rmm_qk_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh,
                               double rho) {
   (void)hkv;
+  (void)nk;
   const int64_t k = rmm_k(rho, dh);
-  if (k < 0 || batch < 1 || hq < 1 || nq < 1 || nk < 1) return 0;
+  if (k < 0 || batch < 1 || hq < 1 || nq < 1) return 0;
   if (k == dh) return 0;
   const int64_t items = batch * hq;
-  const int64_t k_pad = round_up(k, 8);
   Carver c(nullptr);
   c.take<double>(items * dh);
   c.take<int32_t>(items * k);
-  c.take<uint16_t>(items * nq * k_pad);
-  c.take<uint16_t>(items * nk * k_pad);
+  c.take<uint8_t>(items * dh);
+  c.take<uint16_t>(items * nq * dh);
   return c.bytes();
 }
 
@@ -747,49 +755,40 @@ rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch,
       if (e != cudaSuccess) return cuda_fail(e, "iota launch");
     }
   } else {
+    // QK^T is bound by writing S: the dropped head dims of each query head are
+    // zeroed (Q_m) and the dense product with K runs as is -- exactly
+    // sum_{j in I_h} Q_h[:, j] K_g(h)[:, j]^T, without packed Q_I / K_I copies.
     const size_t need = rmm_qk_workspace_bytes(batch, hq, hkv, nq, nk, dh, rho);
     if (ws == nullptr || ws_bytes < need)
       return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
-    const int64_t k_pad = round_up(k, 8);
     Carver c(ws);
     double* colsq = c.take<double>(items * dh);
     int32_t* idx_ws = c.take<int32_t>(items * k);
-    uint16_t* qpack = c.take<uint16_t>(items * nq * k_pad);
-    uint16_t* kpack = c.take<uint16_t>(items * nk * k_pad);
+    uint8_t* keep = c.take<uint8_t>(items * dh);
+    uint16_t* qm = c.take<uint16_t>(items * nq * dh);
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if (rmm_status st = launch_colsq(Q, items, nq * dh, nq, dh, dh, false, 0, colsq, s)) return st;
-    if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s)) return st;
-    PackParams pq{};
-    pq.src = Q;
-    pq.src_ld = dh;
-    pq.rows = nq;
-    pq.d = dh;
-    pq.g_outer = 1;
-    pq.g_inner = 1;
-    pq.s_outer = nq * dh;
-    pq.s_inner = 0;
-    pq.idx = idx;
-    pq.k = k;
-    pq.k_pad = k_pad;
-    pq.dst = qpack;
-    pq.batch = items;
-    if (rmm_status st = launch_pack(pq, s)) return st;
-    PackParams pkk = pq;
-    pkk.src = K;
-    pkk.rows = nk;
-    pkk.g_outer = hq;
-    pkk.g_inner = hq / hkv;
-    pkk.s_outer = hkv * nk * dh;
-    pkk.s_inner = nk * dh;
-    pkk.dst = kpack;
-    if (rmm_status st = launch_pack(pkk, s)) return st;
-    if (rmm_status st = make_tmap(&ta, qpack, k_pad, items * nq, k_pad * 2, 64, 128)) return st;
-    if (rmm_status st = make_tmap(&tb, kpack, k_pad, items * nk, k_pad * 2, 64, 256)) return st;
-    g.k = static_cast<int>(k);
-    g.num_kb = static_cast<int>(ceil_div(k, 64));
-    g.b_g_outer = 1;
-    g.b_g_inner = 1;
-    g.b_s_outer = nk;
+    if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s, keep)) return st;
+    MaskParams mp{};
+    mp.src = Q;
+    mp.dst = qm;
+    mp.rows = nq;
+    mp.cols = dh;
+    mp.keep = keep;
+    mp.by_rows = 0;
+    mp.batch = items;
+    mp.g_outer = 1;
+    mp.g_inner = 1;
+    mp.s_outer = nq * dh;
+    if (rmm_status st = launch_mask(mp, s)) return st;
+    if (rmm_status st = make_tmap(&ta, qm, dh, items * nq, dh * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, K, dh, batch * hkv * nk, dh * 2, 64, 256)) return st;
+    g.k = static_cast<int>(dh);
+    g.num_kb = static_cast<int>(ceil_div(dh, 64));
+    g.b_g_outer = static_cast<int>(hq);
+    g.b_g_inner = static_cast<int>(hq / hkv);
+    g.b_s_outer = hkv * nk;
+    g.b_s_inner = nk;
   }
   if (causal) return launch_gemm<256, kBTileK, kEpiF32, kCausalMaskScores>(ta, tb, g, s);
   return launch_gemm<256, kBTileK, kEpiF32, kCausalNone>(ta, tb, g, s);
@@ -798,15 +797,16 @@ rmm_status rmm_qk(const rmm_bf16* Q, const rmm_bf16* K, float* S, int64_t batch,
 // ---------------------------------------------------------------- PV
 size_t rmm_pv_workspace_bytes(int64_t batch, int64_t h, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, double rho) {
   (void)hkv;
+  (void)nq;
   const int64_t k = rmm_k(rho, nk);
-  if (k < 0 || batch < 1 || h < 1 || nq < 1) return 0;
+  if (k < 0 || batch < 1 || h < 1 || dh < 1) return 0;
   if (k == nk) return 0;
   const int64_t items = batch * h;
   Carver c(nullptr);
   c.take<double>(items * nk);
   c.take<int32_t>(items * k);
-  c.take<uint16_t>(items * nq * round_up(k, 8));
-  c.take<uint16_t>(items * round_up(k, 64) * dh);
+  c.take<uint8_t>(items * nk);
+  c.take<uint16_t>(items * nk * dh);
   return c.bytes();
 }
 
@@ -857,60 +857,42 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
       if (e != cudaSuccess) return cuda_fail(e, "iota launch");
     }
   } else {
+    // PV is bound by reading P: the V rows of dropped key positions are zeroed
+    // (V_m, per query head) and the product streams P once -- exactly
+    // sum_{j in I_h} P_h[:, j] V_g(h)[j, :], without a packed P_I.  With
+    // causal = 1 the entries above the diagonal are masked in shared memory.
     const size_t need = rmm_pv_workspace_bytes(batch, h, hkv, nq, nk, dh, rho);
     if (ws == nullptr || ws_bytes < need)
       return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
-    const int64_t k_pad = round_up(k, 8);
     Carver c(ws);
     double* colsq = c.take<double>(items * nk);
     int32_t* idx_ws = c.take<int32_t>(items * k);
-    uint16_t* ppack = c.take<uint16_t>(items * nq * k_pad);
-    const int64_t k_rows = round_up(k, 64);
-    uint16_t* vpack = c.take<uint16_t>(items * k_rows * dh);
+    uint8_t* keep = c.take<uint8_t>(items * nk);
+    uint16_t* vm = c.take<uint16_t>(items * nk * dh);
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if (rmm_status st = launch_colsq(P, items, nq * nk, nq, nk, nk, causal != 0, off, colsq, s)) return st;
-    if (rmm_status st = launch_select(colsq, items, nk, k, idx, nullptr, s)) return st;
-    PackParams pp{};
-    pp.src = P;
-    pp.src_ld = nk;
-    pp.rows = nq;
-    pp.d = nk;
-    pp.g_outer = 1;
-    pp.g_inner = 1;
-    pp.s_outer = nq * nk;
-    pp.idx = idx;
-    pp.k = k;
-    pp.k_pad = k_pad;
-    pp.dst = ppack;
-    pp.batch = items;
-    pp.causal = causal;
-    pp.causal_off = off;
-    if (rmm_status st = launch_pack(pp, s)) return st;
-    // V_pack[b][t, :] = V_g(b)[I_b[t], :], zero rows up to a multiple of 64
-    RowPackParams rp{};
-    rp.src = V;
-    rp.src_ld = dh;
-    rp.cols = dh;
-    rp.idx = idx;
-    rp.k = k;
-    rp.rows_out = k_rows;
-    rp.dst = vpack;
-    rp.dst_ld = dh;
-    rp.batch = items;
-    rp.g_outer = h;
-    rp.g_inner = h / hkv;
-    rp.s_outer = hkv * nk * dh;
-    rp.s_inner = nk * dh;
-    if (rmm_status st = launch_rowpack(rp, s)) return st;
-    if (rmm_status st = make_tmap(&ta, ppack, k_pad, items * nq, k_pad * 2, 64, 128)) return st;
-    if (rmm_status st = make_tmap(&tb, vpack, dh, items * k_rows, dh * 2, 64, 64)) return st;
-    g.k = static_cast<int>(k);
-    g.num_kb = static_cast<int>(ceil_div(k, 64));
-    g.idx = idx;
-    g.idx_bstride = k;
+    if (rmm_status st = launch_select(colsq, items, nk, k, idx, nullptr, s, keep)) return st;
+    MaskParams mp{};
+    mp.src = V;
+    mp.dst = vm;
+    mp.rows = nk;
+    mp.cols = dh;
+    mp.keep = keep;
+    mp.by_rows = 1;
+    mp.batch = items;
+    mp.g_outer = h;
+    mp.g_inner = h / hkv;
+    mp.s_outer = hkv * nk * dh;
+    mp.s_inner = nk * dh;
+    if (rmm_status st = launch_mask(mp, s)) return st;
+    if (rmm_status st = make_tmap(&ta, P, nk, items * nq, nk * 2, 64, 128)) return st;
+    if (rmm_status st = make_tmap(&tb, vm, dh, items * nk, dh * 2, 64, 64)) return st;
+    g.k = static_cast<int>(nk);
+    g.num_kb = static_cast<int>(ceil_div(nk, 64));
+    g.idx = nullptr;
     g.b_g_outer = 1;
     g.b_g_inner = 1;
-    g.b_s_outer = k_rows;
+    g.b_s_outer = nk;
     g.b_s_inner = 0;
   }
   if (dh == 128)

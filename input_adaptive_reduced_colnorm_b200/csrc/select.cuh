@@ -28,6 +28,7 @@ struct SelectParams {
   int64_t k;
   int32_t* idx;         // [batch][k]
   double* retained;     // [batch] or nullptr: sum_{j in I} q_j / sum_j q_j
+  uint8_t* keep;        // [batch][d] or nullptr: 1 where j is in I, else 0
 };
 
 constexpr int kSelBits = 12;
@@ -262,6 +263,12 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
 #pragma unroll
   for (int e = 0; e < KPT; ++e) {
     if ((sel >> e) & 1u) out[pos++] = j0 + e;
+  }
+  if (p.keep != nullptr) {
+    uint8_t* kp = p.keep + b * p.d;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e)
+      if ((valid >> e) & 1u) kp[j0 + e] = static_cast<uint8_t>((sel >> e) & 1u);
   }
   if (p.retained != nullptr) {
     double kept = 0.0, all = 0.0;

@@ -123,7 +123,7 @@ def test_workspace_queries(L):
     assert a >= 4096 * 2048 * 2
     assert L.rmm_qk_workspace_bytes(1, 32, 8, 4096, 4096, 128, 1.0) == 0
     assert L.rmm_qk_workspace_bytes(1, 32, 8, 4096, 4096, 128, 0.5) >= 2 * 32 * 4096 * 64 * 2
-    assert L.rmm_pv_workspace_bytes(1, 32, 32, 1024, 1024, 128, 0.5) >= 32 * 1024 * 512 * 2
+    assert L.rmm_pv_workspace_bytes(1, 32, 32, 1024, 1024, 128, 0.5) >= 32 * 1024 * 128 * 2
     assert L.rmm_select_workspace_bytes(3, 10, 100) >= 3 * 100 * 8
 
 

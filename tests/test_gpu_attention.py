@@ -131,6 +131,24 @@ def test_pv_entry_point_with_junk_above_diagonal():
         check_close(synthetic.widen(O.cpu()), ref["O"], "pv entry point")
 
 
+@pytest.mark.parametrize("rho", [1.0, 0.8])
+def test_pv_dense_and_reduced_ignore_entries_above_the_diagonal(rho):
+    """Causal PV treats P[i, j] with j > i + (nk - nq) as zero on every path."""
+    P, V = synthetic.pv_inputs(heads=2, n=328)
+    junk = torch.triu(torch.full((328, 328), 5.0), 1).to(torch.bfloat16)
+    Pj = P + junk
+    O, idx = rmm.pv(Pj.cuda(), V.cuda(), rho, causal=True, return_idx=True)
+    torch.cuda.synchronize()
+    for h in range(2):
+        q = oracle.column_sq_norms(synthetic.widen(Pj[0, h]), causal=True)
+        I = idx[0, h].cpu().numpy().astype(np.int64)
+        check_index_set(I, q, oracle.retention_count(rho, 328))
+        Ph = synthetic.widen(Pj[0, h])
+        Pr = Ph[:, I].copy()
+        Pr[I[None, :] > np.arange(328)[:, None]] = 0.0
+        check_close(synthetic.widen(O[0, h].cpu()), Pr @ synthetic.widen(V[0, h])[I, :], f"pv junk head {h}")
+
+
 @pytest.mark.parametrize("rho", [0.5, 0.8])
 def test_pv_seq16384_sampled(rho):
     """Long-context PV: 32 heads x 16384 x 16384 causal softmax probabilities drawn on
