@@ -126,3 +126,197 @@ __global__ void __launch_bounds__(256, 2) colsq_kernel(const ColsqParams p) {
 }
 
 }  // namespace rmm
+
+namespace rmm {
+
+// ---------------------------------------------------------------- TMA-staged variant
+// Same sums, for matrices with at least a few dozen rows.  A strip of W columns
+// is streamed through shared memory in 16 KB tiles of R = 8192 / W rows by one
+// producer thread issuing 3-D TMA loads (x = column, y = row, z = batch item)
+// into a ring of kColsqStages buffers; eight consumer warps square and sum each
+// tile straight out of shared memory.  Keeping ~96 KB of loads in flight per
+// CTA costs no registers, so the kernel holds HBM busy with two CTAs per SM.
+//
+// Work split: the CTAs of a cluster share one strip.  With CAUSAL the rows of
+// a strip that see none of its columns are skipped first and only the visible
+// rows are dealt out in whole tiles, so every CTA of the cluster has the same
+// amount of work (the triangle of a causal matrix no longer leaves half of
+// each cluster idle at the cluster barrier).  Rows past n and columns past d
+// are outside the tensor map and arrive as zeros.
+//
+// Summation order per column: each thread adds 4 rows in fp32 (exact bf16
+// squares, ~1e-7 relative rounding), folds them into fp64, then the warps'
+// partials are added in a fixed order and the cluster's CTAs in rank order.
+// Deterministic.
+constexpr int kColsqStages = 6;
+constexpr uint32_t kColsqTileBytes = 16384;
+constexpr int kColsqThreads = 288;  // 8 consumer warps + 1 producer warp
+
+struct ColsqTmaParams {
+  int64_t n, d;
+  int64_t causal_off;  // with CAUSAL: element (i, j) counts iff j <= i + causal_off
+  double* colsq;       // [batch][d]
+  int csize;           // CTAs of a cluster sharing one strip (1, 2, 4 or 8)
+};
+
+template <int W>
+struct ColsqShape {
+  static constexpr int TX = W / 8;                          // threads across a row (8 columns each)
+  static constexpr int TY = 256 / TX;                       // rows covered by one pass of the consumers
+  static constexpr int R = kColsqTileBytes / (2 * W);       // rows per tile
+  static constexpr int RPT = R / TY;                        // rows per thread per tile
+  static_assert(RPT == 4, "each thread adds four rows of a tile in fp32");
+};
+
+template <int W, bool CAUSAL>
+__global__ void __launch_bounds__(kColsqThreads, 2)
+    colsq_tma_kernel(const __grid_constant__ CUtensorMap tmA, const ColsqTmaParams p) {
+  using S = ColsqShape<W>;
+  extern __shared__ __align__(128) uint8_t smem[];  // kColsqStages tiles, reused for the final reduction
+  __shared__ uint64_t full[kColsqStages], empty[kColsqStages];
+  __shared__ double part[W];
+  __shared__ int abort_word;
+  volatile int* abort_flag = &abort_word;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int C = p.csize;
+  const uint32_t rank = (C > 1) ? cluster_ctarank() : 0u;
+  const int64_t strip = blockIdx.x / C;
+  const int b = blockIdx.y;
+  const int64_t c0 = strip * W;
+
+  // the strip's visible rows, in whole tiles, split evenly over the cluster
+  int64_t first = 0;
+  if (CAUSAL) {
+    first = c0 - p.causal_off;
+    if (first < 0) first = 0;
+    first = first / S::R * S::R;
+  }
+  const int64_t tiles = first < p.n ? (p.n - first + S::R - 1) / S::R : 0;
+  const int64_t per = (tiles + C - 1) / C;
+  const int64_t t_begin = static_cast<int64_t>(rank) * per;
+  const int64_t t_end = t_begin + per < tiles ? t_begin + per : tiles;
+  const int nt = t_end > t_begin ? static_cast<int>(t_end - t_begin) : 0;
+  const int64_t row0 = first + t_begin * S::R;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kColsqStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 8);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8 && lane == 0) prefetch_tensormap(&tmA);
+  __syncthreads();
+  wait_prior_kernels();
+
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  const int tx = threadIdx.x % S::TX;
+  const int ty = threadIdx.x / S::TX;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int t = 0; t < nt; ++t) {
+        const int stage = t % kColsqStages;
+        const int use = t / kColsqStages;
+        if (use > 0 && !mbar_wait(&empty[stage], (use - 1) & 1, abort_flag, kDevErrTimeoutProducer)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], kColsqTileBytes);
+        tma_load_3d(smem + stage * kColsqTileBytes, &tmA, &full[stage], static_cast<int32_t>(c0),
+                    static_cast<int32_t>(row0 + static_cast<int64_t>(t) * S::R), b);
+        ++issued;
+      }
+      if (!ok) {
+        // wait (bounded) for the loads already issued so none lands after exit
+        for (int s = 0; s < kColsqStages; ++s) {
+          const uint32_t uses = (issued + kColsqStages - 1 - s) / kColsqStages;
+          if (uses == 0) continue;
+          const uint32_t a = smem_u32(&full[s]);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(a, (uses - 1) & 1u) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const uint32_t base = smem_u32(smem) + static_cast<uint32_t>((ty * W + tx * 8) * 2);
+    for (int t = 0; t < nt; ++t) {
+      const int stage = t % kColsqStages;
+      if (!mbar_wait(&full[stage], (t / kColsqStages) & 1, abort_flag, kDevErrTimeoutEpilogue)) break;
+      uint4 v[S::RPT];
+#pragma unroll
+      for (int u = 0; u < S::RPT; ++u) v[u] = lds_v4(base + stage * kColsqTileBytes + u * S::TY * W * 2);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
+      float a32[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a32[e] = 0.f;
+      const int64_t r = row0 + static_cast<int64_t>(t) * S::R;
+      if (CAUSAL && c0 + W - 1 > r + p.causal_off) {
+        // this tile crosses the diagonal: drop (i, j) with j > i + off
+#pragma unroll
+        for (int u = 0; u < S::RPT; ++u) {
+          const int64_t lim = r + ty + u * S::TY + p.causal_off - (c0 + tx * 8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float x = (e & 1) ? bf16hi(w[u * 4 + (e >> 1)]) : bf16lo(w[u * 4 + (e >> 1)]);
+            if (e > lim) x = 0.f;
+            a32[e] = fmaf(x, x, a32[e]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < S::RPT; ++u) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = (e & 1) ? bf16hi(w[u * 4 + (e >> 1)]) : bf16lo(w[u * 4 + (e >> 1)]);
+            a32[e] = fmaf(x, x, a32[e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
+    }
+  }
+
+  // ------------------------------------------------------------ reduction
+  __syncthreads();  // every tile consumed (or abandoned): the ring can hold the partials
+  double* red = reinterpret_cast<double*>(smem);  // [TY][W]
+  if (warp < 8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[ty * W + tx * 8 + e] = acc[e];
+  }
+  __syncthreads();
+  if (threadIdx.x < W) {
+    double s = 0.0;
+    for (int y = 0; y < S::TY; ++y) s += red[y * W + threadIdx.x];
+    part[threadIdx.x] = s;
+  }
+  if (C > 1) {
+    cluster_sync();
+    if (rank == 0 && threadIdx.x < W) {
+      const int64_t col = c0 + threadIdx.x;
+      const uint32_t a = smem_u32(&part[threadIdx.x]);
+      double s = 0.0;
+      for (int q = 0; q < C; ++q) s += ld_shared_cluster_f64(map_shared_rank(a, static_cast<uint32_t>(q)));
+      if (col < p.d) p.colsq[static_cast<int64_t>(b) * p.d + col] = s;
+    }
+    cluster_sync();
+  } else if (threadIdx.x < W) {
+    const int64_t col = c0 + threadIdx.x;
+    if (col < p.d) p.colsq[static_cast<int64_t>(b) * p.d + col] = part[threadIdx.x];
+  }
+}
+
+}  // namespace rmm

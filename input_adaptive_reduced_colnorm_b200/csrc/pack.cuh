@@ -313,36 +313,40 @@ struct MaskParams {
   int64_t g_outer, g_inner, s_outer, s_inner;  // source item of b (as in PackParams)
 };
 
+// One batch item per blockIdx.y; inside an item each thread walks the 16-byte
+// vectors v, v + stride, ... with an incremental (row, column) cursor, so the
+// loop carries no divisions.
 __global__ void __launch_bounds__(256) mask_copy_kernel(const MaskParams p) {
   wait_prior_kernels();
   constexpr int ILP = 4;
+  const int64_t b = blockIdx.y;
   const int64_t vpr = p.cols / 8;
-  const int64_t total = p.batch * p.rows * vpr;
-  const int64_t keep_len = p.by_rows ? p.rows : p.cols;
+  const int64_t per_item = p.rows * vpr;
+  const uint8_t* kb = p.keep + b * (p.by_rows ? p.rows : p.cols);
+  const uint16_t* src = p.src + (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+  uint16_t* dst = p.dst + b * per_item * 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v0 < total; v0 += ILP * stride) {
+  const int64_t srow = stride / vpr;
+  const int64_t scol = stride - srow * vpr;
+  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  int64_t row = v / vpr;
+  int64_t col = v - row * vpr;
+  while (v < per_item) {
     uint4 val[ILP];
-    int64_t dst_off[ILP];
+    int64_t off[ILP];
 #pragma unroll
     for (int u = 0; u < ILP; ++u) {
-      const int64_t v = v0 + u * stride;
-      dst_off[u] = -1;
+      off[u] = -1;
       val[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (v < total) {
-        const int64_t row_g = v / vpr;  // row over all batch items
-        const int64_t c8 = (v - row_g * vpr) * 8;
-        const int64_t b = row_g / p.rows;
-        const int64_t r = row_g - b * p.rows;
-        dst_off[u] = row_g * p.cols + c8;
-        const uint8_t* kb = p.keep + b * keep_len;
-        const uint16_t* src =
-            p.src + (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner + r * p.cols + c8;
+      if (v < per_item) {
+        off[u] = v * 8;
+        const uint16_t* sp = src + row * p.cols + col * 8;
         if (p.by_rows) {
-          if (__ldg(kb + r)) val[u] = ldg_nc_v4(src);
+          if (__ldg(kb + row)) val[u] = ldg_nc_v4(sp);
         } else {
-          const uint2 kk = *reinterpret_cast<const uint2*>(kb + c8);  // eight keep bytes
+          const uint2 kk = *reinterpret_cast<const uint2*>(kb + col * 8);  // eight keep bytes
           if (kk.x | kk.y) {
-            const uint4 x = ldg_nc_v4(src);
+            const uint4 x = ldg_nc_v4(sp);
             const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
             const uint32_t ks[2] = {kk.x, kk.y};
             uint32_t o[4];
@@ -356,10 +360,17 @@ __global__ void __launch_bounds__(256) mask_copy_kernel(const MaskParams p) {
           }
         }
       }
+      v += stride;
+      row += srow;
+      col += scol;
+      if (col >= vpr) {
+        col -= vpr;
+        ++row;
+      }
     }
 #pragma unroll
     for (int u = 0; u < ILP; ++u)
-      if (dst_off[u] >= 0) *reinterpret_cast<uint4*>(p.dst + dst_off[u]) = val[u];
+      if (off[u] >= 0) *reinterpret_cast<uint4*>(dst + off[u]) = val[u];
   }
 }
 

@@ -141,11 +141,116 @@ struct Carver {
 };
 
 // ---------------------------------------------------------------- launches
+// Cluster launch with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, int csize, cudaStream_t s,
+                           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Column sums of squares through shared-memory tiles (colsq_tma_kernel).  The
+// strip width W and the cluster size C are chosen so that one wave of two CTAs
+// per SM holds as many CTAs as possible while every CTA keeps at least two
+// tiles; problems larger than a wave take W = 256 and C up to 8 (at least four
+// tiles per CTA) so that no single CTA is long enough to leave a tail.
+template <int W, bool CAUSAL>
+rmm_status launch_colsq_tma_t(const CUtensorMap& tm, const ColsqTmaParams& p, int64_t strips, int64_t batch,
+                              cudaStream_t s) {
+  constexpr size_t smem = static_cast<size_t>(kColsqStages) * kColsqTileBytes;
+  cudaError_t e = cudaFuncSetAttribute(colsq_tma_kernel<W, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e, "column-norm attribute");
+  e = launch_cluster(colsq_tma_kernel<W, CAUSAL>, dim3(static_cast<unsigned>(strips * p.csize), static_cast<unsigned>(batch)),
+                     dim3(kColsqThreads), smem, p.csize, s, tm, p);
+  if (e != cudaSuccess) return cuda_fail(e, "column-norm launch");
+  return RMM_OK;
+}
+
+rmm_status launch_colsq_tma(const uint16_t* A, int64_t batch, int64_t bstride, int64_t n, int64_t d, int64_t lda,
+                            bool causal, int64_t off, double* colsq, cudaStream_t s) {
+  const int64_t wave = 2LL * num_sms();
+  int W = 0, C = 0;
+  int64_t best = 0;
+  for (int w = 256; w >= 64; w /= 2) {
+    const int64_t R = kColsqTileBytes / (2 * w);
+    for (int c = 1; c <= 8; c *= 2) {
+      if (c > 1 && n < c * 2 * R) break;
+      const int64_t ctas = ceil_div(d, w) * batch * c;
+      if (ctas <= wave && ctas > best) {
+        best = ctas;
+        W = w;
+        C = c;
+      }
+    }
+  }
+  if (best == 0) {
+    W = 256;
+    const int64_t R = kColsqTileBytes / (2 * W);
+    C = 1;
+    while (C < 8 && n >= 2 * C * 4 * R) C *= 2;
+  }
+  const int64_t strips = ceil_div(d, W);
+  if (strips * C > kIntMax || batch > 65535 || n > kIntMax || d > kIntMax)
+    return fail(RMM_ERR_UNSUPPORTED, "column-norm grid too large");
+
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(RMM_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  CUtensorMap tm;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(lda) * 2,
+                           static_cast<cuuint64_t>(batch > 1 ? bstride : n * lda) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(W), static_cast<cuuint32_t>(kColsqTileBytes / (2 * W)), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(A), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RMM_ERR_CUDA, "cuTensorMapEncodeTiled (column norms) failed (%d)", static_cast<int>(r));
+
+  ColsqTmaParams p{};
+  p.n = n;
+  p.d = d;
+  p.causal_off = off;
+  p.colsq = colsq;
+  p.csize = C;
+#define RMM_COLSQ_TMA_CASE(w)                                                          \
+  case w:                                                                              \
+    return causal ? launch_colsq_tma_t<w, true>(tm, p, strips, batch, s)               \
+                  : launch_colsq_tma_t<w, false>(tm, p, strips, batch, s);
+  switch (W) {
+    RMM_COLSQ_TMA_CASE(256)
+    RMM_COLSQ_TMA_CASE(128)
+    RMM_COLSQ_TMA_CASE(64)
+  }
+#undef RMM_COLSQ_TMA_CASE
+  return fail(RMM_ERR_UNSUPPORTED, "column-norm strip width");
+}
+
+// Column sums of squares.  Matrices of 64 rows or more whose batch items start
+// on 16-byte boundaries stream through shared memory with TMA
+// (colsq_tma_kernel); short ones (decode rows) and oddly strided batches use
+// the register kernel, whose 16-row bursts of direct loads finish a few rows in
+// one round trip.
 rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64_t n, int64_t d, int64_t lda,
                         bool causal, int64_t off, double* colsq, cudaStream_t s) {
-  // Pick the strip width (TX threads x 8 columns) and the cluster size C (CTAs
-  // splitting a strip's rows) so that the grid fits in one wave of two CTAs per
-  // SM with as many CTAs as possible; larger problems simply take several waves.
+  if (n >= 64 && (batch == 1 || bstride % 8 == 0)) return launch_colsq_tma(A, batch, bstride, n, d, lda, causal, off, colsq, s);
+  // Register kernel: pick the strip width (TX threads x 8 columns) and the
+  // cluster size C (CTAs splitting a strip's rows) so that the grid fits in one
+  // wave of two CTAs per SM with as many CTAs as possible; larger problems
+  // simply take several waves.
   const int64_t wave = 2LL * num_sms();
   int C = 0, TX = 0;
   int64_t best = 0;
@@ -177,26 +282,12 @@ rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64
   p.colsq = colsq;
   p.rows_per_cta = ceil_div(n, C);
   p.csize = C;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(strips * C), static_cast<unsigned>(batch), 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  const dim3 grid(static_cast<unsigned>(strips * C), static_cast<unsigned>(batch), 1);
   cudaError_t e = cudaSuccess;
-#define RMM_COLSQ_CASE(tx)                                                          \
-  case tx:                                                                          \
-    e = causal ? cudaLaunchKernelEx(&cfg, colsq_kernel<tx, true>, p)               \
-               : cudaLaunchKernelEx(&cfg, colsq_kernel<tx, false>, p);             \
+#define RMM_COLSQ_CASE(tx)                                                                                  \
+  case tx:                                                                                                  \
+    e = causal ? launch_cluster(colsq_kernel<tx, true>, grid, dim3(256), 0, C, s, p)                        \
+               : launch_cluster(colsq_kernel<tx, false>, grid, dim3(256), 0, C, s, p);                      \
     break;
   switch (TX) {
     RMM_COLSQ_CASE(32)
@@ -280,9 +371,12 @@ rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
 }
 
 rmm_status launch_mask(const MaskParams& p, cudaStream_t s) {
-  const int64_t total = p.batch * p.rows * (p.cols / 8);
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256 * 4), 8LL * num_sms()));
-  const cudaError_t e = launch_chained(mask_copy_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p);
+  const int64_t per_item = p.rows * (p.cols / 8);
+  if (p.batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "too many batch items for the mask copy");
+  const int64_t cap = std::max<int64_t>(1, 8LL * num_sms() / p.batch);
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(per_item, 256 * 4), cap));
+  const cudaError_t e = launch_chained(mask_copy_kernel, dim3(static_cast<unsigned>(grid), static_cast<unsigned>(p.batch)),
+                                       dim3(256), 0, s, p);
   if (e != cudaSuccess) return cuda_fail(e, "mask launch");
   return RMM_OK;
 }
