@@ -230,6 +230,115 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
   }
 }
 
+// Same pack, with each source row staged by one 1-D bulk copy (TMA) instead
+// of 16-byte cp.async by every thread.  Thread 0 keeps NBUF - 1 rows in
+// flight; the CTA gathers one staged row per step with a single barrier.
+// Each thread produces column PAIRS: lanes read consecutive entries of the
+// index set, so the 32 gathers of one warp instruction fall within a few
+// hundred bytes of the row (no 8-way bank conflicts) and the warp writes 128
+// contiguous bytes.  Dynamic shared memory: NBUF row buffers of ``buf_bytes``,
+// then the index set as 16-bit offsets [k_pad] (0xFFFF marks padding).
+// Requires 16-byte aligned source rows and an even k_pad.
+template <int NBUF>
+__global__ void __launch_bounds__(256) pack_rows_bulk_kernel(const PackParams p, uint32_t buf_bytes) {
+  extern __shared__ __align__(128) uint8_t pk_bulk_smem[];
+  __shared__ uint64_t full[NBUF];
+  __shared__ int abort_word;
+  volatile int* abort_flag = &abort_word;
+  uint8_t* bufs = pk_bulk_smem;
+  uint16_t* s_idx = reinterpret_cast<uint16_t*>(pk_bulk_smem + static_cast<size_t>(NBUF) * buf_bytes);
+
+  const int64_t total = p.batch * p.rows;
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * per;
+  int64_t r_end = r_begin + per;
+  if (r_end > total) r_end = total;
+  if (r_begin >= r_end) return;  // uniform over the CTA
+  const int nrows = static_cast<int>(r_end - r_begin);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NBUF; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  wait_prior_kernels();
+
+  PackCursor stage_at, gather_at;
+  stage_at.init(p, r_begin);
+  gather_at = stage_at;
+  uint32_t issued = 0;
+  auto issue_next = [&]() {  // thread 0: stage row `issued` into buffer issued % NBUF
+    const int64_t lim = pack_visible(p, stage_at.i);
+    const uint32_t bytes = static_cast<uint32_t>((lim + 7) / 8 * 16);
+    uint64_t* bar = &full[issued % NBUF];
+    if (bytes > 0) {
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_load_1d(bufs + (issued % NBUF) * buf_bytes, stage_at.base + stage_at.i * p.src_ld, bytes, bar);
+    } else {
+      mbar_arrive(bar);  // nothing visible in this row
+    }
+    stage_at.next(p);
+    ++issued;
+  };
+  if (threadIdx.x == 0)
+    while (issued < static_cast<uint32_t>(NBUF - 1) && issued < static_cast<uint32_t>(nrows)) issue_next();
+
+  const int pairs = static_cast<int>(p.k_pad / 2);
+  const uint32_t* idx2 = reinterpret_cast<const uint32_t*>(s_idx);
+  int64_t cur_b = -1;
+  for (int q = 0; q < nrows; ++q) {
+    if (gather_at.b != cur_b) {  // (re)load this batch item's index set
+      __syncthreads();
+      const int32_t* I = p.idx + gather_at.b * p.k;
+      const int k = static_cast<int>(p.k);
+      const int k_pad = static_cast<int>(p.k_pad);
+      for (int t0 = threadIdx.x; t0 < k_pad; t0 += 8 * blockDim.x) {
+        int32_t v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int t = t0 + e * blockDim.x;
+          v[e] = (t < k) ? __ldg(I + t) : 0xFFFF;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int t = t0 + e * blockDim.x;
+          if (t < k_pad) s_idx[t] = static_cast<uint16_t>(v[e]);
+        }
+      }
+      cur_b = gather_at.b;
+    }
+    const bool got = mbar_wait(&full[q % NBUF], (q / NBUF) & 1, abort_flag, kDevErrTimeoutProducer);
+    // row q has landed everywhere and every thread is done with row q - 1
+    if (!__syncthreads_and(got)) break;
+    if (threadIdx.x == 0 && issued < static_cast<uint32_t>(nrows)) issue_next();  // into row q - 1's buffer
+
+    const uint16_t* row = reinterpret_cast<const uint16_t*>(bufs + (q % NBUF) * buf_bytes);
+    const uint32_t lim = static_cast<uint32_t>(pack_visible(p, gather_at.i));
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.dst + (r_begin + q) * p.k_pad);
+#pragma unroll 4
+    for (int t = threadIdx.x; t < pairs; t += 256) {
+      const uint32_t w = idx2[t];
+      const uint32_t j0 = w & 0xFFFFu, j1 = w >> 16;
+      const uint32_t v0 = (j0 < lim) ? row[j0] : 0u;  // 0xFFFF padding is never < lim (d <= 32768)
+      const uint32_t v1 = (j1 < lim) ? row[j1] : 0u;
+      dst[t] = v0 | (v1 << 16);
+    }
+    gather_at.next(p);
+  }
+  if (threadIdx.x == 0 && *abort_flag) {
+    // wait (bounded) for the copies already issued so none lands after exit
+    for (int s = 0; s < NBUF; ++s) {
+      const uint32_t uses = (issued + NBUF - 1 - s) / NBUF;
+      if (uses == 0) continue;
+      const uint32_t a = smem_u32(&full[s]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, (uses - 1) & 1u) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+  }
+}
+
 // Row pack of the kept contraction rows of the second operand:
 // dst[b][t, :] = src_item(b)[I_b[t], :] for t < k, zero rows for k <= t < rows_out
 // ("Algorithm Deep-Dive: RMM", Core Approach: B[I, :]).  Whole rows are
@@ -292,6 +401,103 @@ __global__ void __launch_bounds__(256) pack_rows_gather_kernel(const RowPackPara
       for (int u = 0; u < ILP; ++u) {
         const int c = c0 + u * tpr;
         if (c < vpr) *reinterpret_cast<uint4*>(dst + c * 8) = v[u];
+      }
+    }
+  }
+}
+
+// Row pack by bulk copies: rows of 16-byte multiples, every row kept
+// (rows_out == k).  Each CTA owns a contiguous range of at most
+// kRowpackMaxRows packed rows and copies them in chunks of at most
+// kRowpackChunk bytes: a 1-D bulk load into a ring slot of shared memory, then
+// a 1-D bulk store from that slot to the packed matrix, kRowpackStages - 1
+// loads in flight while the stores drain.  The CTA's row indices are staged in
+// shared memory first and one thread walks the chunks with an incremental
+// cursor, so issuing a copy costs a few instructions and no memory round trip.
+constexpr int kRowpackStages = 6;
+constexpr uint32_t kRowpackChunk = 16384;
+constexpr int64_t kRowpackMaxRows = 2048;
+
+struct RowpackCursor {
+  int64_t local;   // packed row within this CTA's range
+  int64_t b, t;    // batch item, row within it
+  int c;           // chunk within the row
+  const uint16_t* item;
+  __device__ void set_item(const RowPackParams& p) {
+    item = p.src + (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+  }
+  __device__ void next(const RowPackParams& p, int chunks) {
+    if (++c < chunks) return;
+    c = 0;
+    ++local;
+    if (++t == p.k) {
+      t = 0;
+      ++b;
+      set_item(p);
+    }
+  }
+};
+
+__global__ void __launch_bounds__(32) pack_rows_bulk_copy_kernel(const RowPackParams p, int chunks) {
+  extern __shared__ __align__(128) uint8_t rp_smem[];
+  __shared__ uint64_t full[kRowpackStages];
+  __shared__ int abort_word;
+  volatile int* abort_flag = &abort_word;
+  int32_t* s_rows = reinterpret_cast<int32_t*>(rp_smem + kRowpackStages * kRowpackChunk);
+  const int64_t total = p.batch * p.k;
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * per;
+  int64_t r1 = r0 + per;
+  if (r1 > total) r1 = total;
+  if (r0 >= r1) return;  // uniform over the CTA
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRowpackStages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  wait_prior_kernels();
+  for (int64_t r = threadIdx.x; r < r1 - r0; r += 32) s_rows[r] = __ldg(p.idx + r0 + r);
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+
+  const int64_t n = (r1 - r0) * chunks;
+  const int64_t chunk_elems = kRowpackChunk / 2;
+  const uint32_t last_bytes = static_cast<uint32_t>(p.cols * 2 - static_cast<int64_t>(chunks - 1) * kRowpackChunk);
+  RowpackCursor ld{0, r0 / p.k, r0 % p.k, 0, nullptr};
+  ld.set_item(p);
+  RowpackCursor st = ld;
+  auto load = [&](int64_t q) {
+    const uint32_t bytes = (ld.c == chunks - 1) ? last_bytes : kRowpackChunk;
+    const uint16_t* src = ld.item + static_cast<int64_t>(s_rows[ld.local]) * p.src_ld + ld.c * chunk_elems;
+    uint64_t* bar = &full[q % kRowpackStages];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load_1d(rp_smem + (q % kRowpackStages) * kRowpackChunk, src, bytes, bar);
+    ld.next(p, chunks);
+  };
+  int64_t loaded = 0;
+  while (loaded < kRowpackStages && loaded < n) load(loaded++);
+  for (int64_t q = 0; q < n; ++q) {
+    const int s = static_cast<int>(q % kRowpackStages);
+    if (!mbar_wait(&full[s], static_cast<uint32_t>((q / kRowpackStages) & 1), abort_flag, kDevErrTimeoutProducer)) break;
+    const uint32_t bytes = (st.c == chunks - 1) ? last_bytes : kRowpackChunk;
+    uint16_t* dst = p.dst + (st.b * p.rows_out + st.t) * p.dst_ld + st.c * chunk_elems;
+    bulk_store_1d(dst, rp_smem + s * kRowpackChunk, bytes);
+    bulk_commit_group();
+    st.next(p, chunks);
+    if (q >= 1 && loaded < n) {
+      bulk_wait_group_read<1>();  // the store of chunk q - 1 has left its slot
+      load(loaded++);             // chunk q - 1 + kRowpackStages into that slot
+    }
+  }
+  bulk_wait_group<0>();
+  if (*abort_flag) {
+    // wait (bounded) for the loads already issued so none lands after exit
+    for (int s = 0; s < kRowpackStages; ++s) {
+      const int64_t uses = (loaded + kRowpackStages - 1 - s) / kRowpackStages;
+      if (uses == 0) continue;
+      const uint32_t a = smem_u32(&full[s]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, static_cast<uint32_t>((uses - 1) & 1)) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
   }

@@ -335,6 +335,24 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
     const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), 8LL * num_sms());
     e = launch_chained(pack_rows_warp_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), smem, s, p, d_round);
     if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  } else if (p.k_pad % 2 == 0 && (p.batch == 1 || (p.s_outer % 8 == 0 && p.s_inner % 8 == 0))) {
+    // rows staged by bulk copies: as many row buffers (2 to 4) as fit in
+    // ~110 KB, so that two CTAs share an SM even for the longest rows
+    const uint32_t buf_bytes = static_cast<uint32_t>(round_up(d_round * 2, 128));
+    const size_t idx_bytes = static_cast<size_t>(round_up(p.k_pad * 2, 16));
+    int nbuf = 4;
+    while (nbuf > 2 && nbuf * static_cast<size_t>(buf_bytes) + idx_bytes > 110 * 1024) --nbuf;
+    const size_t smem = nbuf * static_cast<size_t>(buf_bytes) + idx_bytes;
+    if (smem > 220 * 1024) return fail(RMM_ERR_UNSUPPORTED, "row too long for the pack kernel");
+    auto kern = (nbuf == 4) ? pack_rows_bulk_kernel<4> : (nbuf == 3) ? pack_rows_bulk_kernel<3> : pack_rows_bulk_kernel<2>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "pack attribute");
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+    const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * num_sms());
+    e = launch_chained(kern, dim3(static_cast<unsigned>(grid)), dim3(256), smem, s, p, buf_bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
   } else {
     // four row buffers for rows up to 8192 columns, two beyond (more CTAs per SM)
     const int64_t idx_elems = round_up(p.k_pad, 8);
@@ -357,6 +375,22 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
 }
 
 rmm_status launch_rowpack(const RowPackParams& p, cudaStream_t s) {
+  if (p.rows_out == p.k && p.k > 0 && p.cols % 8 == 0 && p.src_ld % 8 == 0 && p.dst_ld % 8 == 0 &&
+      (p.batch == 1 || (p.s_outer % 8 == 0 && p.s_inner % 8 == 0))) {
+    // whole rows by bulk copies: two CTAs per SM, at most kRowpackMaxRows rows each
+    const int64_t chunks = ceil_div(p.cols * 2, kRowpackChunk);
+    const int64_t rows = p.batch * p.k;
+    if (chunks > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "rows too long for the row pack");
+    const int64_t grid = std::min<int64_t>(rows, std::max<int64_t>(2LL * num_sms(), ceil_div(rows, kRowpackMaxRows)));
+    const size_t smem = static_cast<size_t>(kRowpackStages) * kRowpackChunk + kRowpackMaxRows * sizeof(int32_t);
+    cudaError_t e = cudaFuncSetAttribute(pack_rows_bulk_copy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail(e, "row pack attribute");
+    e = launch_chained(pack_rows_bulk_copy_kernel, dim3(static_cast<unsigned>(grid)), dim3(32), smem, s, p,
+                       static_cast<int>(chunks));
+    if (e != cudaSuccess) return cuda_fail(e, "row pack launch");
+    return RMM_OK;
+  }
   // threads per row: a power of two with at least 8 vectors per thread where the
   // rows are long enough, so each thread keeps several 16-byte loads in flight
   const int64_t vpr = (p.cols + 7) / 8;

@@ -137,6 +137,45 @@ def test_stage_entry_points_compose_to_rmm_linear():
     assert torch.equal(bp.cpu()[:, :520], B.cpu()[I, :])
 
 
+def _bf16_rows(g, rows, cols):
+    return synthetic.to_bf16(g.standard_normal((rows, cols), dtype=np.float32))
+
+
+def test_gather_rows_long_rows_unsorted_indices():
+    """Rows of 8200 columns (two bulk chunks, the second 16 bytes), indices in any
+    order with repeats; the packed rows are exact copies."""
+    g = synthetic.rng(32)
+    B = _bf16_rows(g, 3000, 8200).cuda()
+    idx = torch.as_tensor(g.integers(0, 3000, size=1700), dtype=torch.int32).cuda()
+    bp = rmm.gather_rows(B, idx)
+    torch.cuda.synchronize()
+    assert torch.equal(bp[:, :8200], B[idx.long()])
+
+
+def test_gather_rows_more_rows_than_one_wave_holds():
+    """650000 kept rows of 16 bytes: more than two CTAs per SM x 2048 rows, so the
+    grid grows past two CTAs per SM."""
+    g = synthetic.rng(33)
+    B = _bf16_rows(g, 700000, 8).cuda()
+    idx = torch.as_tensor(np.sort(g.choice(700000, size=650000, replace=False)), dtype=torch.int32).cuda()
+    bp = rmm.gather_rows(B, idx)
+    torch.cuda.synchronize()
+    assert torch.equal(bp, B[idx.long()])
+
+
+def test_gather_columns_long_strided_rows():
+    """Rows of 14336 columns inside a wider allocation (lda 14400), 7000 kept
+    columns padded to 7040."""
+    g = synthetic.rng(34)
+    full = _bf16_rows(g, 37, 14400).cuda()
+    A = full[:, :14336]
+    idx = torch.as_tensor(np.sort(g.choice(14336, size=7000, replace=False)), dtype=torch.int32).cuda()
+    ap = rmm.gather_columns(A, idx, ld_pack=7040)
+    torch.cuda.synchronize()
+    assert torch.equal(ap[:, :7000], A[:, idx.long()])
+    assert not ap[:, 7000:].any()
+
+
 _DECODE_W = {}
 
 
