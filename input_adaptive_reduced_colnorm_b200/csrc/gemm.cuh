@@ -21,6 +21,13 @@
 //               alternating) -> one TMA tensor store per chunk, clipped to the
 //               batch item's rows and columns.  (Stores from registers, one row
 //               per lane, left the fp32 score writes at ~26% of HBM bandwidth.)
+// Work split: tiles are dealt to the CTAs round-robin.  When the tile count is
+// not a multiple of the grid, the last wave holds fewer tiles than there are
+// CTAs and most SMs would idle for a whole tile time; instead each of those
+// tail_tiles trailing tiles is cut along N into tail_split pieces of BN /
+// tail_split columns (a narrower UMMA, N = 128 or 64), one piece per CTA, so
+// the last wave takes about 1 / tail_split of a tile time.  Nothing is added
+// across CTAs: every output element is still produced by one accumulator.
 // Every wait is bounded (about one second); on a timeout the CTA records an
 // error code, drains its own copies in flight, frees its TMEM and returns.
 // There is no cluster multicast anywhere: each CTA fetches its own tiles and
@@ -55,6 +62,9 @@ struct GemmParams {
   int64_t out_bstride;   // elements between batch items
   float scale;
   int64_t causal_off;    // key/position j is visible to row i iff j <= i + causal_off
+  // narrow last wave (MN-major B only): the last tail_tiles tiles are cut into
+  // tail_split pieces of BN / tail_split (>= 64) columns; 0 / 1 = no cut
+  int tail_tiles, tail_split;
 };
 
 template <int BN>
@@ -144,6 +154,34 @@ __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, 
   m0 = (r - nt * p.m_tiles) * 128;
 }
 
+// One unit of a CTA's work: output columns [nt * BN + n_off, + w) of one tile.
+struct GemmWork {
+  int tile, n_off, w;
+};
+
+// The it-th work unit of this CTA, or false when it has none left: whole tiles
+// blockIdx.x, + P, ... first, then at most one piece of the narrow last wave.
+template <int BN>
+__device__ __forceinline__ bool gemm_work(const GemmParams& p, int total_tiles, int it, GemmWork& wk) {
+  const int P = gridDim.x;
+  const int bx = blockIdx.x;
+  const int whole = total_tiles - p.tail_tiles;
+  const int n_whole = whole > bx ? (whole - bx + P - 1) / P : 0;
+  if (it < n_whole) {
+    wk.tile = bx + it * P;
+    wk.n_off = 0;
+    wk.w = BN;
+    return true;
+  }
+  if (p.tail_tiles == 0) return false;
+  const int q = bx + (it - n_whole) * P;  // piece of the last wave
+  if (q >= p.tail_tiles * p.tail_split) return false;
+  wk.tile = whole + q / p.tail_split;
+  wk.w = BN / p.tail_split;
+  wk.n_off = (q % p.tail_split) * wk.w;
+  return true;
+}
+
 template <int BN, int BMODE, int EPI, int CAUSAL>
 __global__ void __launch_bounds__(192, 1)
     rmm_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -201,11 +239,13 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t phase = 0;
     uint32_t issued = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    GemmWork wk;
+    for (int it = 0; ok && gemm_work<BN>(p, total_tiles, it, wk); ++it) {
       int b, m0, nt;
-      gemm_tile_coords(p, tile, b, m0, nt);
-      const int n0 = nt * BN;
-      const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, n0);
+      gemm_tile_coords(p, wk.tile, b, m0, nt);
+      const int n0 = nt * BN + wk.n_off;
+      const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, nt * BN);
+      const uint32_t b_bytes = static_cast<uint32_t>(wk.w) * 64 * 2;
       const int a_row = b * p.a_rows_per_batch + m0;
       const int64_t brow0 = gemm_b_row_base(p, b);
       for (int kb = 0; kb < nkb; ++kb) {
@@ -217,13 +257,13 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
+          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + b_bytes);
           tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * 64, a_row);
         }
         __syncwarp();
         uint8_t* dstB = sB + stage * C::B_BYTES;
         if (BMODE == kBTileMN) {
-          if (lane < BN / 64)
+          if (lane < wk.w / 64)
             tma_load_2d(dstB + lane * 8192, &tmB, &full[stage], n0 + lane * 64, static_cast<int32_t>(brow0 + kb * 64));
         } else {
           if (lane == 0) tma_load_2d(dstB, &tmB, &full[stage], kb * 64, static_cast<int32_t>(brow0 + n0));
@@ -270,11 +310,13 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t ready_phase = 0;  // one parity bit per stage for the `ready` barriers
       int acc_i = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      GemmWork wk;
+      for (int it = 0; ok && gemm_work<BN>(p, total_tiles, it, wk); ++it) {
         int b, m0, nt;
-        gemm_tile_coords(p, tile, b, m0, nt);
+        gemm_tile_coords(p, wk.tile, b, m0, nt);
         const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, nt * BN);
         if (nkb == 0) continue;
+        const uint32_t idesc = (wk.w == BN) ? IDESC : make_idesc_bf16(128, wk.w, 0, (BMODE == kBTileK) ? 0 : 1);
         const int acc = acc_i & 1;
         const uint32_t acc_par = (acc_i >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, kDevErrTimeoutMma)) {
@@ -303,7 +345,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t ad = make_sw128_desc(a0 + kk * 32, 16, 1024);
             const uint64_t bd = (BMODE == kBTileK) ? make_sw128_desc(b0 + kk * 32, 16, 1024)
                                                    : make_sw128_desc(b0 + kk * 2048, 8192, 1024);
-            umma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -330,11 +372,12 @@ __global__ void __launch_bounds__(192, 1)
     constexpr int CW = (EPI == kEpiF32) ? 32 : 64;  // columns per 128-byte chunk row
     int acc_i = 0;
     int seq = 0;  // chunks staged by this warp so far (buffer alternation)
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    GemmWork wk;
+    for (int it = 0; gemm_work<BN>(p, total_tiles, it, wk); ++it) {
       int b, m0, nt;
-      gemm_tile_coords(p, tile, b, m0, nt);
-      const int n0 = nt * BN;
-      const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, n0);
+      gemm_tile_coords(p, wk.tile, b, m0, nt);
+      const int n0 = nt * BN + wk.n_off;
+      const int nkb = gemm_tile_kb<BN, CAUSAL>(p, b, m0, nt * BN);
       const int row0 = m0 + quarter * 32;  // this warp's 32-row slab
       const int row = row0 + lane;
       if (nkb > 0) {
@@ -343,7 +386,7 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&tfull[acc], acc_par, abort_flag, kDevErrTimeoutEpilogue, 64)) break;
         tc_fence_after();
       }
-      for (int c = 0; c < BN / CW; ++c) {
+      for (int c = 0; c < wk.w / CW; ++c) {
         float v[CW];
         if (nkb > 0) {
           uint32_t r[32];

@@ -428,7 +428,8 @@ rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmP
   if (e != cudaSuccess) return cuda_fail(e, "gemm attribute");
   const int64_t tiles = static_cast<int64_t>(p.batch) * p.m_tiles * p.n_tiles;
   if (tiles > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many output tiles");
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  const int64_t units = tiles - p.tail_tiles + static_cast<int64_t>(p.tail_tiles) * std::max(p.tail_split, 1);
+  const int grid = static_cast<int>(std::min<int64_t>(units, num_sms()));
   e = launch_chained(kern, dim3(grid), dim3(192), smem, s, ta, tb, to, p);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return RMM_OK;
@@ -502,6 +503,17 @@ rmm_status gemm_packed(const uint16_t* A, int64_t n, int64_t k, int64_t lda, con
   g.n_tiles = static_cast<int>(ceil_div(m, 256));
   g.k = static_cast<int>(k);
   g.num_kb = static_cast<int>(ceil_div(k, 64));
+  // narrow last wave: cut the tiles of a partial last wave into 2 or 4 pieces
+  // along N when that many pieces still fit one per SM
+  const int64_t tiles = static_cast<int64_t>(g.m_tiles) * g.n_tiles;
+  const int64_t P = num_sms();
+  const int64_t R = tiles > P ? tiles % P : tiles;
+  int split = 4;
+  while (split > 1 && R * split > P) split /= 2;
+  if (R > 0 && split > 1) {
+    g.tail_tiles = static_cast<int>(R);
+    g.tail_split = split;
+  }
   return launch_gemm<256, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, s);
 }
 

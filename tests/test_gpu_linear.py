@@ -176,6 +176,30 @@ def test_gather_columns_long_strided_rows():
     assert not ap[:, 7000:].any()
 
 
+@pytest.mark.parametrize("n,k,m", [(4096, 1024, 4736), (4000, 1000, 4696), (19072, 576, 256), (256, 200, 512),
+                                   (4096, 2048, 14336)])
+def test_gemm_packed_narrow_last_wave(n, k, m):
+    """Products whose last wave of 128 x 256 output tiles is partial (or that have
+    fewer tiles than SMs): those tiles are computed as 2 or 4 narrower pieces along
+    N.  Every shape here has such a tail on a 148-SM B200; the product must match
+    the fp32 reference within the parity tolerance and repeat bit for bit."""
+    g = synthetic.rng(35)
+    ldp = (k + 7) // 8 * 8
+    A = torch.zeros((n, ldp), dtype=torch.bfloat16)
+    A[:, :k] = synthetic.to_bf16(g.standard_normal((n, k), dtype=np.float32))
+    B = synthetic.to_bf16(g.standard_normal((k, m), dtype=np.float32) / np.float32(np.sqrt(k)))
+    A, B = A.cuda(), B.cuda()
+    Y1 = rmm.gemm_packed(A, k, B, m)
+    Y2 = rmm.gemm_packed(A, k, B, m)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)
+    ref = (A[:, :k].float() @ B.float()).cpu().numpy()
+    check_close(Y1.float().cpu().numpy(), ref, "narrow-last-wave product")
+    # every column block of the tail tiles, element by element against the reference
+    tail = Y1[-128:, -512:].float().cpu().numpy()
+    assert np.abs(tail - ref[-128:, -512:]).max() <= 3e-2 * np.abs(ref).max()
+
+
 _DECODE_W = {}
 
 
