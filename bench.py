@@ -33,7 +33,8 @@ PROJ = ["q_proj", "gate_proj", "up_proj", "down_proj"]
 N_TOKENS = 4096
 RHO_MAIN = 0.5
 RHO_SWEEP = (0.9, 0.7)
-GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm.cuh", "input_adaptive_reduced_colnorm_b200/csrc/ptx.cuh"]
+GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm_pair.cuh", "input_adaptive_reduced_colnorm_b200/csrc/gemm.cuh",
+                "input_adaptive_reduced_colnorm_b200/csrc/ptx.cuh"]
 TRAFFIC_PROFILE = "profiles/gemm_packed_llama8b_gate.md"
 
 
@@ -563,7 +564,7 @@ def run_ours(args):
         "rmm_linear_ms_per_step_rho0.5": ms_linear_main,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(),
-                     "kernel": "rmm_gemm_kernel<256, MN tile> on packed gate_proj operands (4096 x 14336, k=2048)",
+                     "kernel": "rmm_gemm_pair_kernel (CTA pairs, 256 x 256 tiles) on packed gate_proj operands (4096 x 14336, k=2048)",
                      "peak_source": f"bf16_tflops_sustained of {peak_src}",
                      "all_gemm_launches_tflops": all_gemm},
         "gemm_ms_per_launch": {x["name"]: gemm_ms[i] for i, x in enumerate(bufs)},

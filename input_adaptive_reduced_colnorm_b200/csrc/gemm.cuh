@@ -161,10 +161,14 @@ struct GemmWork {
 
 // The it-th work unit of this CTA, or false when it has none left: whole tiles
 // blockIdx.x, + P, ... first, then at most one piece of the narrow last wave.
+// (P workers, this one is bx: CTAs, or CTA pairs in the pair kernel)
 template <int BN>
-__device__ __forceinline__ bool gemm_work(const GemmParams& p, int total_tiles, int it, GemmWork& wk) {
-  const int P = gridDim.x;
-  const int bx = blockIdx.x;
+__device__ __forceinline__ bool gemm_work(const GemmParams& p, int total_tiles, int it, GemmWork& wk, int P = -1,
+                                          int bx = -1) {
+  if (P < 0) {
+    P = gridDim.x;
+    bx = blockIdx.x;
+  }
   const int whole = total_tiles - p.tail_tiles;
   const int n_whole = whole > bx ? (whole - bx + P - 1) / P : 0;
   if (it < n_whole) {

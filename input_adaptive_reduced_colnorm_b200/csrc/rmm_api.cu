@@ -17,6 +17,7 @@
 #include "select.cuh"
 #include "pack.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "gemv.cuh"
 
 using namespace rmm;
@@ -435,6 +436,33 @@ rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmP
   return RMM_OK;
 }
 
+// Linear-path product on CTA pairs (256 x 256 tiles, see gemm_pair.cuh).
+rmm_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s) {
+  CUtensorMap to;
+  if (rmm_status st = make_tmap_out(&to, p.out, false, static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.M),
+                                    static_cast<uint64_t>(p.batch), static_cast<uint64_t>(p.ldo),
+                                    static_cast<uint64_t>(p.out_bstride)))
+    return st;
+  constexpr int smem = PairCfg::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(rmm_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm attribute");
+  const int64_t tiles = static_cast<int64_t>(p.batch) * p.m_tiles * p.n_tiles;
+  if (tiles > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many output tiles");
+  // a partial last wave of pair tiles is cut into 256 x 128 pieces when twice
+  // its tiles still fit one per pair
+  const int64_t P = std::max(1, num_sms() / 2);
+  const int64_t R = tiles > P ? tiles % P : tiles;
+  if (R > 0 && 2 * R <= P) {
+    p.tail_tiles = static_cast<int>(R);
+    p.tail_split = 2;
+  }
+  const int64_t units = tiles - p.tail_tiles + static_cast<int64_t>(p.tail_tiles) * std::max(p.tail_split, 1);
+  const int pairs = static_cast<int>(std::min<int64_t>(units, P));
+  e = launch_cluster(rmm_gemm_pair_kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(192), smem, 2, s, ta, tb, to, p);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return RMM_OK;
+}
+
 GemmParams gemm_defaults() {
   GemmParams p{};
   p.batch = 1;
@@ -503,6 +531,10 @@ rmm_status gemm_packed(const uint16_t* A, int64_t n, int64_t k, int64_t lda, con
   g.n_tiles = static_cast<int>(ceil_div(m, 256));
   g.k = static_cast<int>(k);
   g.num_kb = static_cast<int>(ceil_div(k, 64));
+  if (n > 128) {
+    g.m_tiles = static_cast<int>(ceil_div(n, 256));
+    return launch_gemm_pair(ta, tb, g, s);
+  }
   // narrow last wave: cut the tiles of a partial last wave into 2 or 4 pieces
   // along N when that many pieces still fit one per SM
   const int64_t tiles = static_cast<int64_t>(g.m_tiles) * g.n_tiles;
