@@ -23,6 +23,12 @@ Readings where the pages are silent (each is also pinned by a test):
     query i iff j <= i + (nk - nq).  Masked scores are -inf; masked entries of
     P are treated as zero (they are neither read for the norms nor multiplied).
   * GQA: query head h reads key/value head h // (Hq // Hkv).
+  * Decode attention (one query row per head, keys and values in a cache): the
+    G = Hq / Hkv query rows that share a key/value head are the rows of A, so
+    each key/value head gets ONE index set, chosen on the column norms of its
+    group's rows, and its cache is read once for the whole group.  (Per-head
+    sets would make the G heads of a group read G different subsets of the same
+    cache.)  For Hq = Hkv this is per head.
 
 Parity: every function here is pinned by tests/test_oracle.py against
 hand-derived fixtures, closed forms, brute force or invariants; none is
@@ -38,7 +44,7 @@ __all__ = [
     "retention_count", "column_sq_norms", "column_norms", "topk_ascending",
     "retained_energy", "select", "reduced_product", "error_bound", "rmm_linear",
     "rmm_linear_rows", "kv_head", "rmm_qk", "rmm_qk_rows", "rmm_pv", "rmm_pv_rows",
-    "near_tie_band",
+    "near_tie_band", "rmm_decode_qk", "rmm_decode_pv",
 ]
 
 
@@ -260,3 +266,68 @@ def rmm_pv(P: np.ndarray, V: np.ndarray, rho: float, causal: bool = True):
 def rmm_pv_rows(Ph: np.ndarray, Vg: np.ndarray, rho: float, rows, causal=True):
     """Rows ``rows`` of one head's reduced PV output.  Returns (O_rows, I, q)."""
     return _pv_head(np.asarray(Ph, dtype=np.float64), np.asarray(Vg, dtype=np.float64), rho, causal, rows)
+
+
+def _group(hq: int, hkv: int) -> int:
+    if hq % hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return hq // hkv
+
+
+def rmm_decode_qk(Q: np.ndarray, Kt: np.ndarray, rho: float, scale: float = 1.0, nk=None):
+    """Decode scores against a key cache: per key/value group g of batch item b,
+    A = Q[b, g G:(g+1) G, :] (the group's G query rows, [G, dh]), I_g = TopK of the
+    column norms of A over the head-feature dims, and
+        S[b, h, j] = scale * sum_{t in I_g} Q[b, h, t] * Kt[b, g, t, j],   j < nk.
+
+    [DD] "Component mapping" (QK^T selects along the head feature dim by the Q
+    column norm; K gathers those dims) and "Engineering Notes" (decode prunes
+    attention); [KB] "计算 attention score 时".  The key cache is dim-major
+    (Kt [B, Hkv, dh, L], tokens along the last axis), so the kept dims are whole
+    rows of it.  Q [B, Hq, dh] -> S [B, Hq, nk], I [B, Hkv, k].
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    Kt = np.asarray(Kt, dtype=np.float64)
+    Bsz, hq, dh = Q.shape
+    hkv, L = Kt.shape[1], Kt.shape[3]
+    nk = L if nk is None else int(nk)
+    G = _group(hq, hkv)
+    k = retention_count(rho, dh)
+    S = np.empty((Bsz, hq, nk))
+    I = np.empty((Bsz, hkv, k), dtype=np.int64)
+    for b in range(Bsz):
+        for g in range(hkv):
+            A = Q[b, g * G:(g + 1) * G]
+            Ig = topk_ascending(column_norms(A), k)
+            S[b, g * G:(g + 1) * G] = scale * reduced_product(A, Kt[b, g][:, :nk], Ig)
+            I[b, g] = Ig
+    return {"S": S, "I": I}
+
+
+def rmm_decode_pv(P: np.ndarray, V: np.ndarray, rho: float, nk=None):
+    """Decode attention output against a value cache: per key/value group g of
+    batch item b, A = P[b, g G:(g+1) G, :nk] (the group's G probability rows),
+    I_g = TopK of the column norms of A over the token positions, and
+        O[b, h, :] = sum_{j in I_g} P[b, h, j] * V[b, g, j, :].
+
+    [DD] "Component mapping" (PV selects along token positions) and "Engineering
+    Notes" (decode prunes attention); [KB] "计算 attention output 时": only the
+    positions where P has the larger norm let their V rows take part.
+    P [B, Hq, L] (first nk valid), V [B, Hkv, L, dh] -> O [B, Hq, dh], I [B, Hkv, k].
+    """
+    P = np.asarray(P, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    Bsz, hq, L = P.shape
+    hkv, dh = V.shape[1], V.shape[3]
+    nk = L if nk is None else int(nk)
+    G = _group(hq, hkv)
+    k = retention_count(rho, nk)
+    O = np.empty((Bsz, hq, dh))
+    I = np.empty((Bsz, hkv, k), dtype=np.int64)
+    for b in range(Bsz):
+        for g in range(hkv):
+            A = P[b, g * G:(g + 1) * G, :nk]
+            Ig = topk_ascending(column_norms(A), k)
+            O[b, g * G:(g + 1) * G] = reduced_product(A, V[b, g, :nk], Ig)
+            I[b, g] = Ig
+    return {"O": O, "I": I}

@@ -261,3 +261,90 @@ def test_synthetic_generators_are_seeded_and_shaped():
     Pw = synthetic.widen(P)
     assert np.allclose(Pw.sum(axis=-1), 1.0, atol=2e-2)
     assert np.all(np.triu(Pw[0, 0], 1) == 0)
+
+
+# ----------------------------------------------------------------- decode attention
+def test_decode_qk_hand_fixture_group_selection():
+    fx = load("decode_hand.json")["qk"]
+    Q = np.array(fx["Q"], dtype=np.float64)
+    Kt = np.array(fx["Kt_dim_major"], dtype=np.float64)
+    r = oracle.rmm_decode_qk(Q, Kt, fx["rho"])
+    assert np.array_equal(r["I"], np.array(fx["I"]))
+    assert np.allclose(r["S"], np.array(fx["S"]), rtol=0, atol=1e-12)
+    dense = oracle.rmm_decode_qk(Q, Kt, 1.0)
+    assert np.allclose(dense["S"], np.array(fx["S_dense"]), rtol=0, atol=1e-12)
+    # a per-head selection (each head alone) gives other scores: the grouped reading is what is pinned
+    per_head = oracle.rmm_decode_qk(Q.reshape(1, 2, 1, 4)[:, :, 0], np.repeat(Kt, 2, axis=1), fx["rho"])
+    assert not np.allclose(per_head["S"], r["S"])
+
+
+def test_decode_pv_hand_fixture_and_bound():
+    fx = load("decode_hand.json")["pv"]
+    P = np.array(fx["P"], dtype=np.float64)
+    V = np.array(fx["V"], dtype=np.float64)
+    r = oracle.rmm_decode_pv(P, V, fx["rho"])
+    assert np.array_equal(r["I"], np.array(fx["I"]))
+    assert np.allclose(r["O"], np.array(fx["O"]), rtol=0, atol=1e-12)
+    dense = oracle.rmm_decode_pv(P, V, 1.0)
+    assert np.allclose(dense["O"], np.array(fx["O_dense"]), rtol=0, atol=1e-12)
+    err = np.linalg.norm(dense["O"] - r["O"])
+    assert abs(err - fx["error"]) < 1e-3 and err <= fx["bound"]
+    assert abs(oracle.error_bound(P[0], V[0, 0], r["I"][0, 0]) - fx["bound"]) < 1e-3
+
+
+def test_decode_rho_one_is_the_dense_product_bruteforce():
+    g = np.random.default_rng(7)
+    B, hq, hkv, dh, L, nk = 2, 4, 2, 6, 9, 7
+    Q = g.standard_normal((B, hq, dh))
+    Kt = g.standard_normal((B, hkv, dh, L))
+    P = g.random((B, hq, L))
+    V = g.standard_normal((B, hkv, L, dh))
+    S = oracle.rmm_decode_qk(Q, Kt, 1.0, scale=0.5, nk=nk)["S"]
+    O = oracle.rmm_decode_pv(P, V, 1.0, nk=nk)["O"]
+    for b in range(B):
+        for h in range(hq):
+            g_ = h // (hq // hkv)
+            for j in range(nk):
+                acc = 0.0
+                for t in range(dh):
+                    acc += Q[b, h, t] * Kt[b, g_, t, j]
+                assert abs(S[b, h, j] - 0.5 * acc) < 1e-12
+            for c in range(dh):
+                acc = 0.0
+                for j in range(nk):  # tokens at and beyond nk are not part of the cache
+                    acc += P[b, h, j] * V[b, g_, j, c]
+                assert abs(O[b, h, c] - acc) < 1e-12
+
+
+def test_decode_group_of_one_keeps_the_largest_magnitudes():
+    """Hq = Hkv: the column norm of a single row is |x_j|, so the kept set is the k
+    largest |p_j| (QK: |q_t|), lower index first on ties."""
+    g = np.random.default_rng(8)
+    P = np.round(g.standard_normal((1, 3, 40)), 1)  # rounding makes ties
+    V = g.standard_normal((1, 3, 40, 4))
+    k = oracle.retention_count(0.3, 40)
+    I = oracle.rmm_decode_pv(P, V, 0.3)["I"]
+    for h in range(3):
+        order = sorted(range(40), key=lambda j: (-abs(P[0, h, j]), j))
+        assert list(I[0, h]) == sorted(order[:k])
+    Q = np.round(g.standard_normal((1, 2, 16)), 1)
+    Kt = g.standard_normal((1, 2, 16, 5))
+    kq = oracle.retention_count(0.5, 16)
+    Iq = oracle.rmm_decode_qk(Q, Kt, 0.5)["I"]
+    for h in range(2):
+        order = sorted(range(16), key=lambda t: (-abs(Q[0, h, t]), t))
+        assert list(Iq[0, h]) == sorted(order[:kq])
+
+
+def test_decode_error_bound_and_head_order_invariance():
+    g = np.random.default_rng(9)
+    for _ in range(20):
+        Q = g.standard_normal((1, 4, 8)) * np.exp(g.standard_normal(8))
+        Kt = g.standard_normal((1, 1, 8, 11))
+        red = oracle.rmm_decode_qk(Q, Kt, 0.5)
+        dense = oracle.rmm_decode_qk(Q, Kt, 1.0)["S"]
+        I = red["I"][0, 0]
+        # the pages' bound with A = the group's query rows and B = the kept cache rows
+        assert np.linalg.norm(dense - red["S"]) <= oracle.error_bound(Q[0], Kt[0, 0], I) + 1e-9
+        perm = g.permutation(4)
+        assert np.array_equal(oracle.rmm_decode_qk(Q[:, perm], Kt, 0.5)["I"], red["I"])
