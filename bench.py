@@ -358,6 +358,42 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
     out["pv_seq16384"] = pv
     del P, V, O, ws
     torch.cuda.empty_cache()
+
+    # decode attention (one query row per head) against a 32768-token cache:
+    # 8 sequences, 32 query / 8 key-value heads, head dim 128; one index set per
+    # key/value group.  Algorithmic bytes: QK^T reads the kept dim-rows of the
+    # key cache and writes S (plus Q); PV reads P (scores, rho < 1), the kept V
+    # rows and their P entries, and writes O.
+    Q, Kt, P, V = synthetic.decode_attention_inputs_device(dev)
+    b_, hq, dh = Q.shape
+    hkv, nk = Kt.shape[1], Kt.shape[3]
+    G = hq // hkv
+    S = torch.empty((b_, hq, nk), dtype=torch.float32, device=dev)
+    O = torch.empty((b_, hq, dh), dtype=torch.bfloat16, device=dev)
+    da = {}
+    for rho in (1.0, 0.7, 0.5):
+        kq, kp = k_of(rho, dh), k_of(rho, nk)
+        wq = torch.empty(max(L.rmm_decode_qk_workspace_bytes(b_, hq, hkv, dh, rho), 256), dtype=torch.uint8,
+                         device=dev)
+        wp = torch.empty(max(L.rmm_decode_pv_workspace_bytes(b_, hq, hkv, nk, dh, rho), 256), dtype=torch.uint8,
+                         device=dev)
+        ms_qk = timed_call(lambda: ok(L.rmm_decode_qk(Q.data_ptr(), Kt.data_ptr(), S.data_ptr(), b_, hq, hkv, dh, nk,
+                                                      nk, nk, 0.088, rho, None, wq.data_ptr(), wq.numel(), sptr)))
+        ms_pv = timed_call(lambda: ok(L.rmm_decode_pv(P.data_ptr(), V.data_ptr(), O.data_ptr(), b_, hq, hkv, nk, nk, nk,
+                                                      dh, rho, None, wp.data_ptr(), wp.numel(), sptr)))
+        groups = b_ * hkv
+        bq = groups * kq * nk * 2 + b_ * hq * nk * 4 + b_ * hq * dh * 2
+        bp = groups * kp * dh * 2 + b_ * hq * kp * 2 + b_ * hq * dh * 2 + (b_ * hq * nk * 2 if kp < nk else 0)
+        da[str(rho)] = {"k_qk": kq, "k_pv": kp, "qk_ms": ms_qk, "pv_ms": ms_pv,
+                        "qk_gbs": bq / (ms_qk * 1e-3) / 1e9, "pv_gbs": bp / (ms_pv * 1e-3) / 1e9,
+                        "qk_hbm_frac": bq / (ms_qk * 1e-3) / 1e9 / hbm, "pv_hbm_frac": bp / (ms_pv * 1e-3) / 1e9 / hbm}
+        del wq, wp
+    for r in da:
+        da[r]["qk_speedup_vs_rho1"] = da["1.0"]["qk_ms"] / da[r]["qk_ms"]
+        da[r]["pv_speedup_vs_rho1"] = da["1.0"]["pv_ms"] / da[r]["pv_ms"]
+    out["decode_attention_llama8b_ctx32768"] = da
+    del Q, Kt, P, V, S, O
+    torch.cuda.empty_cache()
     return out
 
 

@@ -197,6 +197,45 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
                   int64_t nq, int64_t nk, int64_t dh, int causal, double rho, int32_t* idx_out, void* ws,
                   size_t ws_bytes, rmm_stream stream);
 
+/* ---------------------------------------------------------------- decode attention
+ * One query row per head against a key/value cache ("Algorithm Deep-Dive: RMM",
+ * Component mapping and Engineering Notes: decode prunes attention).  The
+ * G = hq / hkv query rows that share a key/value head are the rows of A, so each
+ * (batch item, key/value head) group gets ONE index set, chosen on the column
+ * norms of its G rows, and its cache rows are read once for the whole group.
+ * Query head h of batch item b belongs to group b * hkv + h / G.
+ *
+ * rmm_decode_qk: I_g = TopK of the column norms of Q_g over the dh head dims,
+ *   S[b][h][j] = scale * sum_{t in I_g} Q[b][h][t] * Kt[b][g][t][j], j < nk.
+ *   Q   device bf16 [batch][hq][dh], contiguous.
+ *   Kt  device bf16 [batch][hkv][dh][ldk]: the key cache stored dim-major
+ *       (token j of dim t at Kt[..][t][j]) so that a kept dim is one contiguous
+ *       row; tokens j < nk are valid, ldk >= nk and a multiple of 8 (columns up
+ *       to the next multiple of 8 past nk are read, and ignored).
+ *   S   device fp32 [batch][hq][lds], lds >= nk and a multiple of 4.
+ *   idx_out device int32 [batch][hkv][k] or NULL, k = rmm_k(rho, dh).
+ *   Requires dh % 8 == 0, dh <= 512, hq / hkv in {1, 2, 4, 8}.
+ * rmm_decode_pv: I_g = TopK of the column norms of P_g over the nk positions,
+ *   O[b][h][:] = sum_{j in I_g} P[b][h][j] * V[b][g][j][:].
+ *   P   device bf16 [batch][hq][ldp] (softmax probabilities of the one query
+ *       row), ldp >= nk and a multiple of 8.
+ *   V   device bf16 [batch][hkv][cap][dh]: the value cache, token-major, cap >= nk.
+ *   O   device bf16 [batch][hq][dh], contiguous.
+ *   idx_out device int32 [batch][hkv][k] or NULL, k = rmm_k(rho, nk).
+ *   Requires dh in {64, 128, 256}, hq / hkv in {1, 2, 4, 8}, (hq / hkv) * dh
+ *   <= 1024, nk <= 32768.
+ * rho = 1 reads the whole cache (no scores, no selection).  Workspaces: the
+ * scores and index sets (rho < 1) and, for PV, fp32 partial sums of the token
+ * chunks that a fix-up kernel adds in a fixed order (deterministic). */
+size_t rmm_decode_qk_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t dh, double rho);
+rmm_status rmm_decode_qk(const rmm_bf16* Q, const rmm_bf16* Kt, float* S, int64_t batch, int64_t hq, int64_t hkv,
+                         int64_t dh, int64_t nk, int64_t ldk, int64_t lds, float scale, double rho, int32_t* idx_out,
+                         void* ws, size_t ws_bytes, rmm_stream stream);
+size_t rmm_decode_pv_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nk, int64_t dh, double rho);
+rmm_status rmm_decode_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t batch, int64_t hq, int64_t hkv,
+                         int64_t nk, int64_t ldp, int64_t cap, int64_t dh, double rho, int32_t* idx_out, void* ws,
+                         size_t ws_bytes, rmm_stream stream);
+
 /* ---------------------------------------------------------------- diagnostics */
 const char* rmm_status_string(rmm_status s);
 /* Message of the most recent failure on the calling thread ("" if none). */

@@ -53,6 +53,12 @@ _SIGNATURES = {
     "rmm_pv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_pv": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_dbl, _c_p, _c_p,
                         _c_size, _c_p]),
+    "rmm_decode_qk_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_decode_qk": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64,
+                               ctypes.c_float, _c_dbl, _c_p, _c_p, _c_size, _c_p]),
+    "rmm_decode_pv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_decode_pv": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl,
+                               _c_p, _c_p, _c_size, _c_p]),
     "rmm_status_string": (ctypes.c_char_p, [_c_int]),
     "rmm_last_error": (ctypes.c_char_p, []),
     "rmm_device_error": (_c_int, [ctypes.POINTER(ctypes.c_int32)]),
@@ -260,6 +266,59 @@ def pv(P, V, rho: float, *, causal: bool = True, out=None, return_idx: bool = Fa
     ws = _workspace(L.rmm_pv_workspace_bytes(b, h, hkv, nq, nk, dh, float(rho)), dev, workspace)
     _check(L.rmm_pv(_ptr(P), _ptr(V), _ptr(out), b, h, hkv, nq, nk, dh, int(causal), float(rho), _ptr(idx),
                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def decode_qk(Q, Kt, rho: float, *, nk=None, scale: float = 1.0, out=None, return_idx: bool = False,
+              workspace=None):
+    """Decode scores against a dim-major key cache.  Q [B, Hq, dh], Kt [B, Hkv, dh, L]
+    (tokens along the last axis, the first nk valid; L a multiple of 8) -> S [B, Hq, nk]
+    fp32.  One index set per key/value group, chosen on the group's query rows."""
+    import torch
+    _require(Q, "Q", torch.bfloat16, 3)
+    _require(Kt, "Kt", torch.bfloat16, 4)
+    if not (Q.is_contiguous() and Kt.is_contiguous()):
+        raise ValueError("Q and Kt must be contiguous")
+    b, hq, dh = Q.shape
+    b2, hkv, dh2, L = Kt.shape
+    if b2 != b or dh2 != dh:
+        raise ValueError("Q / Kt shape mismatch")
+    nk = L if nk is None else int(nk)
+    dev = Q.device
+    if out is None:
+        out = torch.empty((b, hq, (nk + 3) // 4 * 4), dtype=torch.float32, device=dev)[:, :, :nk]
+    k = rmm_k(rho, dh)
+    idx = torch.empty((b, hkv, max(k, 0)), dtype=torch.int32, device=dev) if return_idx else None
+    Lb = lib()
+    ws = _workspace(Lb.rmm_decode_qk_workspace_bytes(b, hq, hkv, dh, float(rho)), dev, workspace)
+    _check(Lb.rmm_decode_qk(_ptr(Q), _ptr(Kt), _ptr(out), b, hq, hkv, dh, nk, L, out.stride(1), float(scale),
+                            float(rho), _ptr(idx), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def decode_pv(P, V, rho: float, *, nk=None, out=None, return_idx: bool = False, workspace=None):
+    """Decode attention output against a token-major value cache.  P [B, Hq, L]
+    (probabilities of the one query row, the first nk valid; L a multiple of 8),
+    V [B, Hkv, cap, dh] -> O [B, Hq, dh] bf16.  One index set per key/value group."""
+    import torch
+    _require(P, "P", torch.bfloat16, 3)
+    _require(V, "V", torch.bfloat16, 4)
+    if not (P.is_contiguous() and V.is_contiguous()):
+        raise ValueError("P and V must be contiguous")
+    b, hq, L = P.shape
+    b2, hkv, cap, dh = V.shape
+    if b2 != b:
+        raise ValueError("P / V shape mismatch")
+    nk = min(L, cap) if nk is None else int(nk)
+    dev = P.device
+    if out is None:
+        out = torch.empty((b, hq, dh), dtype=torch.bfloat16, device=dev)
+    k = rmm_k(rho, nk)
+    idx = torch.empty((b, hkv, max(k, 0)), dtype=torch.int32, device=dev) if return_idx else None
+    Lb = lib()
+    ws = _workspace(Lb.rmm_decode_pv_workspace_bytes(b, hq, hkv, nk, dh, float(rho)), dev, workspace)
+    _check(Lb.rmm_decode_pv(_ptr(P), _ptr(V), _ptr(out), b, hq, hkv, nk, L, cap, dh, float(rho), _ptr(idx),
+                            _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
     return (out, idx) if return_idx else out
 
 

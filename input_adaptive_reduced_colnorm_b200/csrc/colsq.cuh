@@ -320,3 +320,68 @@ __global__ void __launch_bounds__(kColsqThreads, 2)
 }
 
 }  // namespace rmm
+
+namespace rmm {
+
+// ---------------------------------------------------------------- short matrices
+// Column sums of squares of a matrix of at most 32 rows (decode activations,
+// the query rows of one key/value group): one thread per 8 columns reads all n
+// rows of its columns, so no reduction between threads is needed and a grid of
+// ceil(d / 1024) x batch CTAs of 128 threads covers the matrix once.  Rows are
+// summed 4 at a time in fp32 (exact bf16 squares) and folded into fp64, in row
+// order.  Non-causal only.
+constexpr int kColsqShortMaxRows = 32;
+
+__global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {
+  wait_prior_kernels();
+  const int64_t b = blockIdx.y;
+  const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (col0 >= p.d) return;
+  const uint16_t* A = p.A + b * p.batch_stride + col0;
+  const bool full = col0 + 8 <= p.d;
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  for (int64_t r0 = 0; r0 < p.n; r0 += 8) {
+    uint32_t w[8][4];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      w[u][0] = w[u][1] = w[u][2] = w[u][3] = 0u;
+      if (r0 + u < p.n) {
+        const uint16_t* src = A + (r0 + u) * p.lda;
+        if (full) {
+          const uint4 v = ldg_nc_v4(src);
+          w[u][0] = v.x;
+          w[u][1] = v.y;
+          w[u][2] = v.z;
+          w[u][3] = v.w;
+        } else {
+          for (int e = 0; e < 8; ++e)
+            if (col0 + e < p.d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < 8; g += 4) {
+      float a32[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a32[e] = 0.f;
+#pragma unroll
+      for (int u = g; u < g + 4; ++u) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = (e & 1) ? bf16hi(w[u][e >> 1]) : bf16lo(w[u][e >> 1]);
+          a32[e] = fmaf(x, x, a32[e]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
+    }
+  }
+  double* out = p.colsq + b * p.d + col0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    if (col0 + e < p.d) out[e] = acc[e];
+}
+
+}  // namespace rmm

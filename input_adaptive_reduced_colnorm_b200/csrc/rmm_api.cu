@@ -19,6 +19,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "gemv.cuh"
+#include "decode_attn.cuh"
 
 using namespace rmm;
 
@@ -248,6 +249,20 @@ rmm_status launch_colsq_tma(const uint16_t* A, int64_t batch, int64_t bstride, i
 rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64_t n, int64_t d, int64_t lda,
                         bool causal, int64_t off, double* colsq, cudaStream_t s) {
   if (n >= 64 && (batch == 1 || bstride % 8 == 0)) return launch_colsq_tma(A, batch, bstride, n, d, lda, causal, off, colsq, s);
+  if (!causal && n <= kColsqShortMaxRows) {
+    if (batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "column-norm grid too large");
+    ColsqParams p{};
+    p.A = A;
+    p.batch_stride = bstride;
+    p.n = n;
+    p.d = d;
+    p.lda = lda;
+    p.colsq = colsq;
+    const dim3 grid(static_cast<unsigned>(ceil_div(d, 1024)), static_cast<unsigned>(batch));
+    const cudaError_t e = launch_chained(colsq_short_kernel, grid, dim3(128), 0, s, p);
+    if (e != cudaSuccess) return cuda_fail(e, "column-norm launch");
+    return RMM_OK;
+  }
   // Register kernel: pick the strip width (TX threads x 8 columns) and the
   // cluster size C (CTAs splitting a strip's rows) so that the grid fits in one
   // wave of two CTAs per SM with as many CTAs as possible; larger problems
@@ -304,7 +319,7 @@ rmm_status launch_colsq(const uint16_t* A, int64_t batch, int64_t bstride, int64
 template <int KPT, int NT>
 rmm_status launch_select_t(const SelectParams& p, int64_t batch, cudaStream_t s) {
   // dynamic keys plus ~17 KB of static histogram and scan space can pass 48 KB
-  const size_t smem = static_cast<size_t>(NT) * KPT * sizeof(uint32_t);
+  const size_t smem = static_cast<size_t>(NT) * KPT * sizeof(uint32_t) * 33 / 32 + sizeof(uint32_t);
   {
     const cudaError_t e = cudaFuncSetAttribute(select_kernel<KPT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
@@ -606,6 +621,187 @@ int64_t rmm_k(double rho, int64_t d) {
   if (k < 1) k = 1;
   if (k > d) k = d;
   return k;
+}
+
+// ---------------------------------------------------------------- decode attention
+}  // extern "C"
+
+namespace {
+bool decode_group_ok(int64_t g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+// Kept positions per PV CTA: enough CTAs for about four per SM over all groups.
+void decode_pv_plan(int64_t groups, int64_t k, int* chunk, int* splits) {
+  const int64_t want = 4LL * num_sms();
+  int64_t c = ceil_div(groups * k, want);
+  c = round_up(std::max<int64_t>(c, 32), 32);
+  if (c > kDecodePvMaxChunk) c = kDecodePvMaxChunk;
+  *chunk = static_cast<int>(c);
+  *splits = static_cast<int>(ceil_div(k, c));
+}
+
+template <int G>
+cudaError_t launch_decode_qk_t(const DecodeQkParams& p, int64_t groups, cudaStream_t s) {
+  constexpr size_t smem = static_cast<size_t>(kDqkStages) * kDqkStageBytes;
+  const cudaError_t e = cudaFuncSetAttribute(decode_qk_staged_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(ceil_div(p.nk, kDqkTokens)), static_cast<unsigned>(groups));
+  return launch_chained(decode_qk_staged_kernel<G>, grid, dim3(288), smem, s, p);
+}
+
+template <int G, int DH>
+cudaError_t launch_decode_pv_t(const DecodePvParams& p, int64_t groups, cudaStream_t s) {
+  constexpr size_t smem = static_cast<size_t>(256 / (DH / 8)) * G * DH * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(decode_pv_kernel<G, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(p.splits), static_cast<unsigned>(groups));
+  return launch_chained(decode_pv_kernel<G, DH>, grid, dim3(256), smem, s, p);
+}
+}  // namespace
+
+extern "C" {
+
+size_t rmm_decode_qk_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t dh, double rho) {
+  const int64_t k = rmm_k(rho, dh);
+  if (k < 0 || batch < 1 || hq < 1 || hkv < 1 || k == dh) return 0;
+  const int64_t groups = batch * hkv;
+  Carver c(nullptr);
+  c.take<double>(groups * dh);
+  c.take<int32_t>(groups * k);
+  return c.bytes();
+}
+
+rmm_status rmm_decode_qk(const rmm_bf16* Q, const rmm_bf16* Kt, float* S, int64_t batch, int64_t hq, int64_t hkv,
+                         int64_t dh, int64_t nk, int64_t ldk, int64_t lds, float scale, double rho, int32_t* idx_out,
+                         void* ws, size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (Q == nullptr || Kt == nullptr || S == nullptr) return fail(RMM_ERR_INVALID_ARG, "Q, Kt and S are required");
+  if (batch < 1 || hq < 1 || hkv < 1 || dh < 1 || nk < 1 || ldk < nk || lds < nk)
+    return fail(RMM_ERR_INVALID_ARG, "need batch, hq, hkv, dh, nk >= 1, ldk >= nk and lds >= nk");
+  if (hq % hkv) return fail(RMM_ERR_INVALID_ARG, "hq must be a multiple of hkv");
+  if (!std::isfinite(scale)) return fail(RMM_ERR_INVALID_ARG, "scale must be finite");
+  const int64_t G = hq / hkv;
+  if (!decode_group_ok(G)) return fail(RMM_ERR_UNSUPPORTED, "hq / hkv must be 1, 2, 4 or 8");
+  if (dh % 8 || dh > kDecodeQkMaxK) return fail(RMM_ERR_UNSUPPORTED, "dh must be a multiple of 8 and at most 512");
+  if (!aligned16(Q) || !aligned16(Kt) || !aligned16(S) || (ldk % 8) || (lds % 4))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned, ldk a multiple of 8 and lds of 4");
+  const int64_t groups = batch * hkv;
+  if (groups > 65535 || nk > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many groups or tokens");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t k = rmm_k(rho, dh);
+  DecodeQkParams p{};
+  p.Q = Q;
+  p.Kt = Kt;
+  p.S = S;
+  p.nk = nk;
+  p.ldk = ldk;
+  p.lds = lds;
+  p.dh = static_cast<int>(dh);
+  p.k = static_cast<int>(k);
+  p.scale = scale;
+  if (k < dh) {
+    const size_t need = rmm_decode_qk_workspace_bytes(batch, hq, hkv, dh, rho);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+    Carver c(ws);
+    double* colsq = c.take<double>(groups * dh);
+    int32_t* idx_ws = c.take<int32_t>(groups * k);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(Q, groups, G * dh, G, dh, dh, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, groups, dh, k, idx, nullptr, s)) return st;
+    p.idx = idx;
+  } else if (idx_out != nullptr) {
+    const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(groups * dh, 256), 1024))),
+                                         dim3(256), 0, s, idx_out, groups, dh);
+    if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+  }
+  cudaError_t e = cudaSuccess;
+  switch (G) {
+    case 1: e = launch_decode_qk_t<1>(p, groups, s); break;
+    case 2: e = launch_decode_qk_t<2>(p, groups, s); break;
+    case 4: e = launch_decode_qk_t<4>(p, groups, s); break;
+    default: e = launch_decode_qk_t<8>(p, groups, s); break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode QK launch");
+  return RMM_OK;
+}
+
+size_t rmm_decode_pv_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nk, int64_t dh, double rho) {
+  const int64_t k = rmm_k(rho, nk);
+  if (k < 0 || batch < 1 || hq < 1 || hkv < 1 || dh < 1 || hq % hkv) return 0;
+  const int64_t groups = batch * hkv;
+  int chunk = 0, splits = 0;
+  decode_pv_plan(groups, k, &chunk, &splits);
+  Carver c(nullptr);
+  if (k < nk) {
+    c.take<double>(groups * nk);
+    c.take<int32_t>(groups * k);
+  }
+  c.take<float>(groups * splits * (hq / hkv) * dh);
+  return c.bytes();
+}
+
+rmm_status rmm_decode_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t batch, int64_t hq, int64_t hkv,
+                         int64_t nk, int64_t ldp, int64_t cap, int64_t dh, double rho, int32_t* idx_out, void* ws,
+                         size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (P == nullptr || V == nullptr || O == nullptr) return fail(RMM_ERR_INVALID_ARG, "P, V and O are required");
+  if (batch < 1 || hq < 1 || hkv < 1 || dh < 1 || nk < 1 || ldp < nk || cap < nk)
+    return fail(RMM_ERR_INVALID_ARG, "need batch, hq, hkv, dh, nk >= 1, ldp >= nk and cap >= nk");
+  if (hq % hkv) return fail(RMM_ERR_INVALID_ARG, "hq must be a multiple of hkv");
+  const int64_t G = hq / hkv;
+  if (!decode_group_ok(G)) return fail(RMM_ERR_UNSUPPORTED, "hq / hkv must be 1, 2, 4 or 8");
+  if (dh != 64 && dh != 128 && dh != 256) return fail(RMM_ERR_UNSUPPORTED, "dh must be 64, 128 or 256");
+  if (G * dh > 1024) return fail(RMM_ERR_UNSUPPORTED, "hq / hkv times dh must be at most 1024");
+  if (!aligned16(P) || !aligned16(V) || !aligned16(O) || (ldp % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and ldp a multiple of 8");
+  if (nk > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "nk above the selection limit (32768)");
+  const int64_t groups = batch * hkv;
+  if (groups > 65535) return fail(RMM_ERR_UNSUPPORTED, "too many groups");
+  const size_t need = rmm_decode_pv_workspace_bytes(batch, hq, hkv, nk, dh, rho);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t k = rmm_k(rho, nk);
+  int chunk = 0, splits = 0;
+  decode_pv_plan(groups, k, &chunk, &splits);
+  Carver c(ws);
+  DecodePvParams p{};
+  if (k < nk) {
+    double* colsq = c.take<double>(groups * nk);
+    int32_t* idx_ws = c.take<int32_t>(groups * k);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(P, groups, G * ldp, G, nk, ldp, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, groups, nk, k, idx, nullptr, s)) return st;
+    p.idx = idx;
+  } else if (idx_out != nullptr) {
+    const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(groups * nk, 256), 1024))),
+                                         dim3(256), 0, s, idx_out, groups, nk);
+    if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+  }
+  float* partial = c.take<float>(groups * splits * G * dh);
+  p.P = P;
+  p.V = V;
+  p.partial = partial;
+  p.ldp = ldp;
+  p.cap = cap;
+  p.k = static_cast<int>(k);
+  p.chunk = chunk;
+  p.splits = splits;
+  cudaError_t e = cudaSuccess;
+#define RMM_DPV(g, d) \
+  if (G == g && dh == d) e = launch_decode_pv_t<g, d>(p, groups, s);
+  RMM_DPV(1, 64) RMM_DPV(1, 128) RMM_DPV(1, 256) RMM_DPV(2, 64) RMM_DPV(2, 128) RMM_DPV(2, 256)
+  RMM_DPV(4, 64) RMM_DPV(4, 128) RMM_DPV(4, 256) RMM_DPV(8, 64) RMM_DPV(8, 128)
+#undef RMM_DPV
+  if (e != cudaSuccess) return cuda_fail(e, "decode PV launch");
+  e = launch_chained(decode_pv_fixup_kernel, dim3(static_cast<unsigned>(groups)), dim3(static_cast<unsigned>(G * dh)), 0, s,
+                     static_cast<const float*>(partial), reinterpret_cast<uint16_t*>(O), splits, static_cast<int>(G * dh));
+  if (e != cudaSuccess) return cuda_fail(e, "decode PV fix-up launch");
+  return RMM_OK;
 }
 
 const char* rmm_status_string(rmm_status s) {

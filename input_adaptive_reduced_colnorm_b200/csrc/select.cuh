@@ -77,13 +77,19 @@ __device__ __forceinline__ double block_sum_f64(double v, double* s_buf) {
   return t;  // valid in thread 0 only
 }
 
-// dynamic shared memory: hi32 keys [NT * KPT] (uint32)
+// Shared-memory slot of key j in the staging array: one padding word per 32
+// keys, so that thread t reading its KPT contiguous keys (t * KPT + e) hits 32
+// different banks for every power-of-two KPT <= 32.
+__device__ __forceinline__ int sel_slot(int j) { return j + (j >> 5); }
+
+// dynamic shared memory: hi32 keys [NT * KPT + NT * KPT / 32] (uint32, padded)
 template <int KPT, int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   wait_prior_kernels();
   constexpr int NW = NT / 32;
   constexpr int BPT = kSelBins / NT;  // histogram bins scanned per thread
   static_assert(kSelBins % NT == 0, "bins must split evenly");
+  static_assert(KPT <= 32 && (KPT & (KPT - 1)) == 0, "a thread's keys must lie in one padded block of 32");
   extern __shared__ __align__(16) uint32_t s_keys[];
   __shared__ uint32_t hist[kSelBins];
   __shared__ int s_warp[32];
@@ -99,33 +105,35 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   const int d = static_cast<int>(p.d);
   const int j0 = threadIdx.x * KPT;
 
-  // coalesced staging of the top 32 bits of every key: all KPT loads of a
-  // thread are in flight before the first store
-  {
-    uint32_t v[KPT];
+  // coalesced staging of the top 32 bits of every key, eight loads in flight
+  // per thread before the first store
+  for (int e0 = 0; e0 < KPT; e0 += 8) {
+    constexpr int B = KPT < 8 ? KPT : 8;
+    uint32_t v[B];
 #pragma unroll
-    for (int e = 0; e < KPT; ++e) {
-      const int j = e * NT + threadIdx.x;
+    for (int e = 0; e < B; ++e) {
+      const int j = (e0 + e) * NT + threadIdx.x;
       v[e] = (j < d) ? static_cast<uint32_t>(static_cast<uint64_t>(__double_as_longlong(__ldg(q + j))) >> 32) : 0u;
     }
 #pragma unroll
-    for (int e = 0; e < KPT; ++e) {
-      const int j = e * NT + threadIdx.x;
-      if (j < d) s_keys[j] = v[e];
+    for (int e = 0; e < B; ++e) {
+      const int j = (e0 + e) * NT + threadIdx.x;
+      if (j < d) s_keys[sel_slot(j)] = v[e];
     }
   }
   __syncthreads();
-  uint32_t hi[KPT];
+  // this thread's keys stay in shared memory (conflict-free by the padding) and
+  // are re-read by each pass instead of being held in registers
+  const uint32_t* my_keys = s_keys + sel_slot(j0);
   uint32_t valid = 0;
   uint32_t kand = 0xffffffffu, kor = 0u;
 #pragma unroll
   for (int e = 0; e < KPT; ++e) {
-    hi[e] = 0u;
     if (j0 + e < d) {
-      hi[e] = s_keys[j0 + e];
+      const uint32_t h = my_keys[e];
       valid |= 1u << e;
-      kand &= hi[e];
-      kor |= hi[e];
+      kand &= h;
+      kor |= h;
     }
   }
   // bits on which all keys agree need no pass
@@ -170,16 +178,16 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < KPT; ++e) {
-      bool m = ((valid >> e) & 1u) && (hi[e] & msk_hi) == pre_hi;
+      bool m = ((valid >> e) & 1u) && (my_keys[e] & msk_hi) == pre_hi;
       uint32_t dig = 0;
       if (m) {
         if (shift >= 32) {
-          dig = (hi[e] >> (shift - 32)) & dmask;
+          dig = (my_keys[e] >> (shift - 32)) & dmask;
         } else {
           const uint32_t lo = static_cast<uint32_t>(__double_as_longlong(q[j0 + e]));
           m = (lo & msk_lo) == pre_lo;
           if (shift + width > 32) {  // digit straddles the two halves
-            const uint64_t full = (static_cast<uint64_t>(hi[e]) << 32) | lo;
+            const uint64_t full = (static_cast<uint64_t>(my_keys[e]) << 32) | lo;
             dig = static_cast<uint32_t>(full >> shift) & dmask;
           } else {
             dig = (lo >> shift) & dmask;
@@ -230,7 +238,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
 #pragma unroll
   for (int e = 0; e < KPT; ++e) {
     if (!((valid >> e) & 1u)) continue;
-    const uint32_t h = hi[e] & msk_hi;
+    const uint32_t h = my_keys[e] & msk_hi;
     if (h > pre_hi) {
       gt |= 1u << e;
     } else if (h == pre_hi) {

@@ -245,3 +245,54 @@ def pv_inputs_device(device, seed: int | None = None, batch: int = 1, heads: int
             V[b, h] = torch.randn((n, dh), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
     del upper
     return P, V
+
+
+# ------------------------------------------------------------------ decode attention
+DECODE_ATTN_SEED = 6  # workload number of the decode-attention inputs
+
+
+def decode_attention_inputs(seed: int | None = None, batch: int = 2, hq: int = 8, hkv: int = 2, dh: int = 128,
+                            nk: int = 1000, L: int | None = None):
+    """Decode-attention operands on the host (small sizes): one query row per head.
+
+    Q  [batch, hq, dh]       N(0,1) times a per-head LogNormal(0,1) scale per head dim
+    Kt [batch, hkv, dh, L]   the key cache stored dim-major, N(0,1)
+    P  [batch, hq, L]        softmax over the first nk positions of 2 N(0,1) logits
+                             (float32, then bfloat16), zero past nk
+    V  [batch, hkv, L, dh]   the value cache, token-major, N(0,1)
+    L defaults to nk rounded up to a multiple of 8 (cache capacity).  bfloat16 CPU tensors."""
+    base = seed_for(DECODE_ATTN_SEED) if seed is None else seed
+    L = (nk + 7) // 8 * 8 if L is None else L
+    Q = np.empty((batch, hq, dh), dtype=np.float32)
+    Kt = np.zeros((batch, hkv, dh, L), dtype=np.float32)
+    P = np.zeros((batch, hq, L), dtype=np.float32)
+    V = np.zeros((batch, hkv, L, dh), dtype=np.float32)
+    for b in range(batch):
+        for h in range(hq):
+            g = rng(head_seed(base, b * 4096 + h))
+            Q[b, h] = g.standard_normal(dh, dtype=np.float32) * np.exp(g.standard_normal(dh)).astype(np.float32)
+            x = 2.0 * g.standard_normal(nk, dtype=np.float32)
+            e = np.exp(x - x.max(), dtype=np.float32)
+            P[b, h, :nk] = e / e.sum(dtype=np.float32)
+        for h in range(hkv):
+            g = rng(head_seed(base, b * 4096 + 2048 + h))
+            Kt[b, h, :, :nk] = g.standard_normal((dh, nk), dtype=np.float32)
+            V[b, h, :nk] = g.standard_normal((nk, dh), dtype=np.float32)
+    return to_bf16(Q), to_bf16(Kt), to_bf16(P), to_bf16(V)
+
+
+def decode_attention_inputs_device(device, seed: int | None = None, batch: int = 8, hq: int = 32, hkv: int = 8,
+                                   dh: int = 128, nk: int = 32768):
+    """Full-size decode-attention operands drawn on the device with torch's seeded
+    generator, same recipe as ``decode_attention_inputs`` (cache capacity = nk)."""
+    base = seed_for(DECODE_ATTN_SEED) if seed is None else seed
+    gen = torch.Generator(device=device)
+    gen.manual_seed(base)
+    f32 = torch.float32
+    Q = (torch.randn((batch, hq, dh), generator=gen, device=device, dtype=f32)
+         * torch.randn((batch, hq, dh), generator=gen, device=device, dtype=f32).exp()).to(torch.bfloat16)
+    Kt = torch.randn((batch, hkv, dh, nk), generator=gen, device=device, dtype=f32).to(torch.bfloat16)
+    P = torch.softmax(2.0 * torch.randn((batch, hq, nk), generator=gen, device=device, dtype=f32), dim=-1)
+    P = P.to(torch.bfloat16)
+    V = torch.randn((batch, hkv, nk, dh), generator=gen, device=device, dtype=f32).to(torch.bfloat16)
+    return Q, Kt, P, V

@@ -133,3 +133,28 @@ def test_binding_refuses_cpu_tensors():
     B = torch.zeros((16, 8), dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         rmm.linear(A, B, 0.5)
+
+
+def test_decode_attention_argument_errors(L):
+    def dqk(Q=P16, Kt=P16, S=P16, b=1, hq=8, hkv=2, dh=128, nk=100, ldk=104, lds=100, scale=1.0, rho=0.5, ws=None,
+            wsb=0):
+        return L.rmm_decode_qk(Q, Kt, S, b, hq, hkv, dh, nk, ldk, lds, scale, rho, None, ws, wsb, None)
+    assert dqk(hkv=3) == INVALID             # hq % hkv
+    assert dqk(ldk=96) == INVALID            # ldk < nk
+    assert dqk(scale=float("inf")) == INVALID
+    assert dqk(hq=24, hkv=2) == UNSUPPORTED  # group of 12
+    assert dqk(dh=100) == UNSUPPORTED
+    assert dqk(ldk=108) == UNSUPPORTED       # not a multiple of 8
+    assert dqk(lds=102) == UNSUPPORTED       # not a multiple of 4
+    assert dqk() == WORKSPACE
+    assert L.rmm_decode_qk_workspace_bytes(1, 8, 2, 128, 1.0) == 0
+
+    def dpv(P=P16, V=P16, O=P16, b=1, hq=8, hkv=2, nk=100, ldp=104, cap=100, dh=128, rho=0.5, ws=None, wsb=0):
+        return L.rmm_decode_pv(P, V, O, b, hq, hkv, nk, ldp, cap, dh, rho, None, ws, wsb, None)
+    assert dpv(cap=99) == INVALID
+    assert dpv(dh=96) == UNSUPPORTED
+    assert dpv(hq=16, hkv=2, dh=256) == UNSUPPORTED  # 8 x 256 > 1024
+    assert dpv(ldp=100) == UNSUPPORTED
+    assert dpv(nk=40000, ldp=40000, cap=40000) == UNSUPPORTED
+    assert dpv() == WORKSPACE
+    assert L.rmm_decode_pv_workspace_bytes(1, 8, 2, 100, 128, 1.0) > 0  # partial sums even at rho = 1
