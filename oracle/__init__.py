@@ -44,7 +44,7 @@ __all__ = [
     "retention_count", "column_sq_norms", "column_norms", "topk_ascending",
     "retained_energy", "select", "reduced_product", "error_bound", "rmm_linear",
     "rmm_linear_rows", "kv_head", "rmm_qk", "rmm_qk_rows", "rmm_pv", "rmm_pv_rows",
-    "near_tie_band", "rmm_decode_qk", "rmm_decode_pv",
+    "near_tie_band", "rmm_decode_qk", "rmm_decode_pv", "silu", "rmm_mlp_gate_up", "rmm_mlp",
 ]
 
 
@@ -331,3 +331,32 @@ def rmm_decode_pv(P: np.ndarray, V: np.ndarray, rho: float, nk=None):
             O[b, g * G:(g + 1) * G] = reduced_product(A, V[b, g, :nk], Ig)
             I[b, g] = Ig
     return {"O": O, "I": I}
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """SiLU(x) = x / (1 + exp(-x)) in float64 (the gate nonlinearity of the MLP block)."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def rmm_mlp_gate_up(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, rho: float):
+    """Gate and up projections of the MLP block with ONE index set I chosen on X
+    (both contract the same input X), then H = SiLU(X_I Wg[I, :]) * (X_I Wu[I, :]).
+
+    [DD] "Attention vs MLP: structural asymmetry" (MLP Up / Down / whole MLP reduced
+    separately) and "Engineering Notes" (conservative MLP rho); [KB] the MLP Up / Gate /
+    Down component analysis.  Returns dict(H, I, G, U).
+    """
+    I, _, _ = select(X, rho)
+    G = reduced_product(X, Wg, I)
+    U = reduced_product(X, Wu, I)
+    return {"H": silu(G) * U, "I": I, "G": G, "U": U}
+
+
+def rmm_mlp(X, Wg, Wu, Wd, rho_gu: float, rho_down: float):
+    """The whole MLP block: H from ``rmm_mlp_gate_up`` (one selection on X), then the
+    down projection Y = H[:, J] Wd[J, :] with its own rho and J chosen on H's column
+    norms (the down input is SiLU(gate) * up).  Returns dict(H, I_gu, Y, I_down)."""
+    gu = rmm_mlp_gate_up(X, Wg, Wu, rho_gu)
+    down = rmm_linear(gu["H"], Wd, rho_down)
+    return {"H": gu["H"], "I_gu": gu["I"], "Y": down["Y"], "I_down": down["I"]}

@@ -348,3 +348,55 @@ def test_decode_error_bound_and_head_order_invariance():
         assert np.linalg.norm(dense - red["S"]) <= oracle.error_bound(Q[0], Kt[0, 0], I) + 1e-9
         perm = g.permutation(4)
         assert np.array_equal(oracle.rmm_decode_qk(Q[:, perm], Kt, 0.5)["I"], red["I"])
+
+
+# ----------------------------------------------------------------- MLP block
+def test_mlp_hand_fixture():
+    fx = load("mlp_hand.json")
+    X, Wg, Wu, Wd = (np.array(fx[n], dtype=np.float64) for n in ("X", "Wg", "Wu", "Wd"))
+    r = oracle.rmm_mlp(X, Wg, Wu, Wd, fx["rho_gu"], fx["rho_down"])
+    assert list(r["I_gu"]) == fx["I_gu"] and list(r["I_down"]) == fx["I_down"]
+    assert np.allclose(r["H"], np.array(fx["H"]), rtol=0, atol=1e-12)
+    assert np.allclose(r["Y"], np.array(fx["Y"]), rtol=0, atol=1e-12)
+    dense = oracle.rmm_mlp(X, Wg, Wu, Wd, 1.0, 1.0)
+    assert np.allclose(dense["H"][1], np.array(fx["H_dense_row1"]), rtol=0, atol=1e-9)
+
+
+def test_mlp_rho_one_is_the_dense_block_bruteforce():
+    g = np.random.default_rng(10)
+    n, d, f, m = 3, 5, 4, 3
+    X, Wg, Wu, Wd = g.standard_normal((n, d)), g.standard_normal((d, f)), g.standard_normal((d, f)), g.standard_normal((f, m))
+    r = oracle.rmm_mlp(X, Wg, Wu, Wd, 1.0, 1.0)
+    for i in range(n):
+        h = []
+        for c in range(f):
+            gs = sum(X[i, j] * Wg[j, c] for j in range(d))
+            us = sum(X[i, j] * Wu[j, c] for j in range(d))
+            h.append(gs / (1.0 + math.exp(-gs)) * us)
+            assert abs(r["H"][i, c] - h[-1]) < 1e-12
+        for c in range(m):
+            assert abs(r["Y"][i, c] - sum(h[j] * Wd[j, c] for j in range(f))) < 1e-12
+
+
+def test_mlp_gate_and_up_use_the_same_columns():
+    """With identity gate and up weights, G = U = X with the dropped columns zeroed,
+    so H = SiLU(x) x exactly on the kept columns of X and 0 on the others."""
+    g = np.random.default_rng(11)
+    X = g.standard_normal((4, 9)) * np.exp(g.standard_normal(9))
+    r = oracle.rmm_mlp_gate_up(X, np.eye(9), np.eye(9), 0.5)
+    I, _, _ = oracle.select(X, 0.5)
+    assert np.array_equal(r["I"], I)
+    keep = np.zeros(9, dtype=bool)
+    keep[I] = True
+    assert np.allclose(r["H"][:, keep], X[:, keep] ** 2 / (1.0 + np.exp(-X[:, keep])), rtol=1e-14, atol=0)
+    assert not r["H"][:, ~keep].any()
+
+
+def test_mlp_down_bound_and_silu_values():
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert abs(oracle.silu(np.array([40.0]))[0] - 40.0) < 1e-12 and abs(oracle.silu(np.array([-40.0]))[0]) < 1e-15
+    g = np.random.default_rng(12)
+    for _ in range(10):
+        X, Wg, Wu, Wd = g.standard_normal((5, 8)), g.standard_normal((8, 6)), g.standard_normal((8, 6)), g.standard_normal((6, 4))
+        r = oracle.rmm_mlp(X, Wg, Wu, Wd, 0.7, 0.5)
+        assert np.linalg.norm(r["H"] @ Wd - r["Y"]) <= oracle.error_bound(r["H"], Wd, r["I_down"]) + 1e-9
