@@ -359,6 +359,31 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
     del P, V, O, ws
     torch.cuda.empty_cache()
 
+    # gated MLP block, Llama-3.1-8B at n = 4096 tokens (d = 4096, f = 14336): one
+    # selection on X for gate and up, fused SiLU(gate) * up, then the down
+    # projection with its own rho.  Kept FLOPs: 2 n k_gu f (gate) + the same (up)
+    # + 2 n k_down m (down).
+    X, Wg, Wu, Wd = (t.to(dev) for t in synthetic.mlp_block())
+    n_, d_ = X.shape
+    f_, m_ = Wg.shape[1], Wd.shape[1]
+    Hb = torch.empty((n_, f_), dtype=torch.bfloat16, device=dev)
+    Yb = torch.empty((n_, m_), dtype=torch.bfloat16, device=dev)
+    mb = {}
+    for rg, rd in ((1.0, 1.0), (0.9, 0.9), (0.7, 0.7), (0.5, 0.5), (0.8, 0.5)):
+        wsm = torch.empty(max(L.rmm_mlp_workspace_bytes(n_, d_, f_, m_, rg, rd), 256), dtype=torch.uint8, device=dev)
+        ms = timed_call(lambda: ok(L.rmm_mlp(X.data_ptr(), n_, d_, d_, Wg.data_ptr(), Wu.data_ptr(), f_, f_,
+                                             Wd.data_ptr(), m_, m_, Hb.data_ptr(), f_, Yb.data_ptr(), m_, rg, rd, None,
+                                             None, wsm.data_ptr(), wsm.numel(), sptr)))
+        kg, kd = k_of(rg, d_), k_of(rd, f_)
+        flops = 4.0 * n_ * kg * f_ + 2.0 * n_ * kd * m_
+        mb[f"{rg}/{rd}"] = {"k_gu": kg, "k_down": kd, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
+        del wsm
+    for r in mb:
+        mb[r]["speedup_vs_rho1"] = mb["1.0/1.0"]["ms"] / mb[r]["ms"]
+    out["mlp_block_llama8b_n4096"] = mb
+    del X, Wg, Wu, Wd, Hb, Yb
+    torch.cuda.empty_cache()
+
     # decode attention (one query row per head) against a 32768-token cache:
     # 8 sequences, 32 query / 8 key-value heads, head dim 128; one index set per
     # key/value group.  Algorithmic bytes: QK^T reads the kept dim-rows of the

@@ -197,6 +197,30 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
                   int64_t nq, int64_t nk, int64_t dh, int causal, double rho, int32_t* idx_out, void* ws,
                   size_t ws_bytes, rmm_stream stream);
 
+/* ---------------------------------------------------------------- MLP block
+ * The gate / up / down projections of a gated MLP ("Algorithm Deep-Dive: RMM",
+ * Attention vs MLP: structural asymmetry, and Engineering Notes: conservative
+ * MLP rho, Down can be lower).  Gate and up contract the same input X, so ONE
+ * index set I (TopK of X's column norms, rho_gu) serves both, and one fused
+ * tensor-core product on CTA pairs writes
+ *   H = SiLU(X[:, I] Wg[I, :]) * (X[:, I] Wu[I, :]),   SiLU(x) = x / (1 + e^-x);
+ * then Y = RMM_rho_down(H, Wd) exactly as rmm_linear (its own selection on H).
+ *   X   device bf16 [n][ldx], n x d.
+ *   Wg, Wu device bf16 [d][ldw], d x f (contraction index as the row).
+ *   Wd  device bf16 [f][ldwd], f x m.
+ *   H   device bf16 [n][ldh], written (the down projection's input).
+ *   Y   device bf16 [n][ldy].
+ *   idx_gu_out  device int32 [rmm_k(rho_gu, d)] or NULL; idx_down_out device
+ *   int32 [rmm_k(rho_down, f)] or NULL.
+ *   ws  rmm_mlp_workspace_bytes(n, d, f, m, rho_gu, rho_down) bytes (0 at
+ *   rho_gu = rho_down = 1 with n > 32: NULL allowed).
+ * Limits: d, f <= 32768; leading dims multiples of 8, pointers 16-byte aligned. */
+size_t rmm_mlp_workspace_bytes(int64_t n, int64_t d, int64_t f, int64_t m, double rho_gu, double rho_down);
+rmm_status rmm_mlp(const rmm_bf16* X, int64_t n, int64_t d, int64_t ldx, const rmm_bf16* Wg, const rmm_bf16* Wu,
+                   int64_t f, int64_t ldw, const rmm_bf16* Wd, int64_t m, int64_t ldwd, rmm_bf16* H, int64_t ldh,
+                   rmm_bf16* Y, int64_t ldy, double rho_gu, double rho_down, int32_t* idx_gu_out,
+                   int32_t* idx_down_out, void* ws, size_t ws_bytes, rmm_stream stream);
+
 /* ---------------------------------------------------------------- decode attention
  * One query row per head against a key/value cache ("Algorithm Deep-Dive: RMM",
  * Component mapping and Engineering Notes: decode prunes attention).  The

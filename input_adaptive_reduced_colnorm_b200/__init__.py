@@ -53,6 +53,9 @@ _SIGNATURES = {
     "rmm_pv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_pv": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_dbl, _c_p, _c_p,
                         _c_size, _c_p]),
+    "rmm_mlp_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_dbl, _c_dbl]),
+    "rmm_mlp": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64,
+                         _c_p, _c_i64, _c_dbl, _c_dbl, _c_p, _c_p, _c_p, _c_size, _c_p]),
     "rmm_decode_qk_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_decode_qk": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64,
                                ctypes.c_float, _c_dbl, _c_p, _c_p, _c_size, _c_p]),
@@ -267,6 +270,36 @@ def pv(P, V, rho: float, *, causal: bool = True, out=None, return_idx: bool = Fa
     _check(L.rmm_pv(_ptr(P), _ptr(V), _ptr(out), b, h, hkv, nq, nk, dh, int(causal), float(rho), _ptr(idx),
                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
     return (out, idx) if return_idx else out
+
+
+def mlp(X, Wg, Wu, Wd, rho_gu: float, rho_down: float, *, H=None, out=None, return_idx: bool = False,
+        workspace=None):
+    """Gated MLP block: H = SiLU(X_I Wg[I]) * (X_I Wu[I]) with one index set I on X for
+    gate and up, then Y = RMM(H, Wd) with its own selection.  X [n, d], Wg / Wu [d, f],
+    Wd [f, m] bf16 CUDA.  Returns Y (and H, idx_gu, idx_down if asked)."""
+    import torch
+    for t, nm in ((X, "X"), (Wg, "Wg"), (Wu, "Wu"), (Wd, "Wd")):
+        _require(t, nm, torch.bfloat16, 2)
+    n, d = X.shape
+    d2, f = Wg.shape
+    if Wu.shape != Wg.shape or d2 != d or Wd.shape[0] != f:
+        raise ValueError("MLP shape mismatch")
+    if Wg.stride(0) != Wu.stride(0):
+        raise ValueError("Wg and Wu must share a row stride")
+    m = Wd.shape[1]
+    dev = X.device
+    if H is None:
+        H = torch.empty((n, f), dtype=torch.bfloat16, device=dev)
+    if out is None:
+        out = torch.empty((n, m), dtype=torch.bfloat16, device=dev)
+    Lb = lib()
+    i1 = torch.empty((max(rmm_k(rho_gu, d), 0),), dtype=torch.int32, device=dev) if return_idx else None
+    i2 = torch.empty((max(rmm_k(rho_down, f), 0),), dtype=torch.int32, device=dev) if return_idx else None
+    ws = _workspace(Lb.rmm_mlp_workspace_bytes(n, d, f, m, float(rho_gu), float(rho_down)), dev, workspace)
+    _check(Lb.rmm_mlp(_ptr(X), n, d, X.stride(0), _ptr(Wg), _ptr(Wu), f, Wg.stride(0), _ptr(Wd), m, Wd.stride(0),
+                      _ptr(H), H.stride(0), _ptr(out), out.stride(0), float(rho_gu), float(rho_down), _ptr(i1),
+                      _ptr(i2), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, H, i1, i2) if return_idx else out
 
 
 def decode_qk(Q, Kt, rho: float, *, nk=None, scale: float = 1.0, out=None, return_idx: bool = False,

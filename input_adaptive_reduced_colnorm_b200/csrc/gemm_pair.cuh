@@ -21,6 +21,13 @@
 //   warps 2..5  epilogue on this CTA's 128 rows (as in the one-CTA kernel);
 //               when an accumulator is drained each warp arrives on the even
 //               CTA's accumulator-empty barrier (8 arrivals per use).
+// SWIGLU (the gate and up projections of an MLP block, "Algorithm Deep-Dive:
+// RMM", Attention vs MLP): the two B halves of a pair tile come from two
+// tensor maps, the even CTA loading gate columns [c, c+128) and the odd CTA up
+// columns [c, c+128) of the same output columns, so each CTA's accumulator holds
+// gate (columns 0-127) and up (128-255) for its rows; the epilogue writes
+// H = SiLU(gate) * up (128 columns per 256-wide tile, bf16).  A narrow piece of
+// width w holds gate in columns [0, w/2) and up in [w/2, w).
 // Work split as in the one-CTA kernel, with pairs as the workers: whole tiles
 // round-robin, then the tiles of a partial last wave cut into two 256 x 128
 // pieces.  Every wait is bounded; the CTAs meet at a cluster barrier before
@@ -50,9 +57,11 @@ __device__ __forceinline__ void pair_tile_coords(const GemmParams& p, int tile, 
   m0 = (r - nt * p.m_tiles) * 256;
 }
 
+template <bool SWIGLU>
 __global__ void __launch_bounds__(192, 1)
     rmm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                         const __grid_constant__ CUtensorMap tmO, const GemmParams p) {
+                         const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmO,
+                         const GemmParams p) {
   using C = PairCfg;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t pair_smem_raw[];
@@ -86,6 +95,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_barrier_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    if (SWIGLU) prefetch_tensormap(&tmB2);
     prefetch_tensormap(&tmO);
   }
   if (warp == 1) {
@@ -114,7 +124,10 @@ __global__ void __launch_bounds__(192, 1)
         pair_tile_coords(p, wk.tile, b, m0, nt);
         const int half = wk.w / 2;
         const int a_row = b * p.a_rows_per_batch + m0 + static_cast<int>(rank) * 128;
-        const int nb = nt * 256 + wk.n_off + static_cast<int>(rank) * half;
+        // B columns of this CTA's half: its 128 of the 256 columns, or (SWIGLU)
+        // the same output columns of gate (even CTA) or up (odd CTA)
+        const int nb = SWIGLU ? nt * 128 + wk.n_off / 2 : nt * 256 + wk.n_off + static_cast<int>(rank) * half;
+        const CUtensorMap* tb = (SWIGLU && rank == 1) ? &tmB2 : &tmB;
         const int64_t brow0 = gemm_b_row_base(p, b);
         const uint32_t pair_bytes = 2u * static_cast<uint32_t>(C::A_BYTES + half * 64 * 2);
         for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -126,7 +139,7 @@ __global__ void __launch_bounds__(192, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], pair_bytes);
           tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * 64, a_row);
           for (int j = 0; j < half / 64; ++j)
-            tma_load_2d_pair(sB + stage * C::B_BYTES + j * 8192, &tmB, bar, nb + j * 64,
+            tma_load_2d_pair(sB + stage * C::B_BYTES + j * 8192, tb, bar, nb + j * 64,
                              static_cast<int32_t>(brow0 + kb * 64));
           ++issued;
           if (++stage == STAGES) {
@@ -207,20 +220,30 @@ __global__ void __launch_bounds__(192, 1)
     for (int it = 0; gemm_work<256>(p, total_tiles, it, wk, npairs, pair); ++it) {
       int b, m0, nt;
       pair_tile_coords(p, wk.tile, b, m0, nt);
-      const int n0 = nt * 256 + wk.n_off;
+      const int n0 = SWIGLU ? nt * 128 + wk.n_off / 2 : nt * 256 + wk.n_off;
       const int row0 = m0 + static_cast<int>(rank) * 128 + quarter * 32;
+      const int out_w = SWIGLU ? wk.w / 2 : wk.w;  // output columns of this unit
       const int acc = acc_i & 1;
       if (!mbar_wait(&tfull[acc], (acc_i >> 1) & 1, abort_flag, kDevErrTimeoutEpilogue, 64)) break;
       tc_fence_after();
-      for (int c = 0; c < wk.w / 64; ++c) {
+      for (int c = 0; c < out_w / 64; ++c) {
         uint32_t w[32];
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t r[32];
-          tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                        static_cast<uint32_t>(acc * 256 + c * 64 + h * 32),
-                    r);
+          tmem_ld32(lane_base + static_cast<uint32_t>(acc * 256 + c * 64 + h * 32), r);
           tmem_ld_wait();
+          if (SWIGLU) {
+            uint32_t u[32];
+            tmem_ld32(lane_base + static_cast<uint32_t>(acc * 256 + out_w + c * 64 + h * 32), u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float g = __uint_as_float(r[e]);
+              r[e] = __float_as_uint(g / (1.f + __expf(-g)) * __uint_as_float(u[e]));
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));

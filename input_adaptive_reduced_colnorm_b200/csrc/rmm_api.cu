@@ -451,15 +451,19 @@ rmm_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmP
   return RMM_OK;
 }
 
-// Linear-path product on CTA pairs (256 x 256 tiles, see gemm_pair.cuh).
-rmm_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s) {
+// Linear-path product on CTA pairs (256 x 256 tiles, see gemm_pair.cuh).  With
+// tb2 != nullptr the gate / up variant: B halves from tb (gate) and tb2 (up),
+// output H = SiLU(gate) * up with 128 output columns per tile.
+rmm_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, GemmParams p, cudaStream_t s,
+                            const CUtensorMap* tb2 = nullptr) {
   CUtensorMap to;
   if (rmm_status st = make_tmap_out(&to, p.out, false, static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.M),
                                     static_cast<uint64_t>(p.batch), static_cast<uint64_t>(p.ldo),
                                     static_cast<uint64_t>(p.out_bstride)))
     return st;
   constexpr int smem = PairCfg::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(rmm_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = tb2 ? rmm_gemm_pair_kernel<true> : rmm_gemm_pair_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "gemm attribute");
   const int64_t tiles = static_cast<int64_t>(p.batch) * p.m_tiles * p.n_tiles;
   if (tiles > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "too many output tiles");
@@ -473,7 +477,7 @@ rmm_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, GemmPa
   }
   const int64_t units = tiles - p.tail_tiles + static_cast<int64_t>(p.tail_tiles) * std::max(p.tail_split, 1);
   const int pairs = static_cast<int>(std::min<int64_t>(units, P));
-  e = launch_cluster(rmm_gemm_pair_kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(192), smem, 2, s, ta, tb, to, p);
+  e = launch_cluster(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(192), smem, 2, s, ta, tb, tb2 ? *tb2 : tb, to, p);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return RMM_OK;
 }
@@ -621,6 +625,108 @@ int64_t rmm_k(double rho, int64_t d) {
   if (k < 1) k = 1;
   if (k > d) k = d;
   return k;
+}
+
+// ---------------------------------------------------------------- MLP block
+}  // extern "C"
+
+namespace {
+// Workspace of the gate / up half of rmm_mlp (rho_gu < 1): scores, index set,
+// X[:, I] and the kept rows of both weights.
+size_t mlp_gate_up_bytes(int64_t n, int64_t d, int64_t f, int64_t k) {
+  if (k == d) return 0;
+  Carver c(nullptr);
+  c.take<double>(d);
+  c.take<int32_t>(k);
+  c.take<uint16_t>(n * round_up(k, 8));
+  c.take<uint16_t>(k * round_up(f, 8));
+  c.take<uint16_t>(k * round_up(f, 8));
+  return c.bytes();
+}
+}  // namespace
+
+extern "C" {
+
+size_t rmm_mlp_workspace_bytes(int64_t n, int64_t d, int64_t f, int64_t m, double rho_gu, double rho_down) {
+  const int64_t k = rmm_k(rho_gu, d);
+  if (k < 0 || n < 1 || f < 1 || m < 1 || rmm_k(rho_down, f) < 0) return 0;
+  return mlp_gate_up_bytes(n, d, f, k) + rmm_linear_workspace_bytes(n, f, m, rho_down);
+}
+
+rmm_status rmm_mlp(const rmm_bf16* X, int64_t n, int64_t d, int64_t ldx, const rmm_bf16* Wg, const rmm_bf16* Wu,
+                   int64_t f, int64_t ldw, const rmm_bf16* Wd, int64_t m, int64_t ldwd, rmm_bf16* H, int64_t ldh,
+                   rmm_bf16* Y, int64_t ldy, double rho_gu, double rho_down, int32_t* idx_gu_out,
+                   int32_t* idx_down_out, void* ws, size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho_gu)) return st;
+  if (rmm_status st = check_rho(rho_down)) return st;
+  if (X == nullptr || Wg == nullptr || Wu == nullptr || Wd == nullptr || H == nullptr || Y == nullptr)
+    return fail(RMM_ERR_INVALID_ARG, "X, Wg, Wu, Wd, H and Y are required");
+  if (n < 1 || d < 1 || f < 1 || m < 1) return fail(RMM_ERR_INVALID_ARG, "n, d, f and m must be >= 1");
+  if (ldx < d || ldw < f || ldwd < m || ldh < f || ldy < m) return fail(RMM_ERR_INVALID_ARG, "leading dimension too small");
+  if (!aligned16(X) || !aligned16(Wg) || !aligned16(Wu) || !aligned16(Wd) || !aligned16(H) || !aligned16(Y) ||
+      (ws != nullptr && !aligned16(ws)) || (ldx % 8) || (ldw % 8) || (ldwd % 8) || (ldh % 8) || (ldy % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
+  if (d > kMaxSelectD || f > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "d and f must be at most 32768");
+  if (n > kIntMax - 256 || f > kIntMax - 256 || m > kIntMax - 256) return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  const int64_t k = rmm_k(rho_gu, d);
+  const size_t gu_bytes = mlp_gate_up_bytes(n, d, f, k);
+  const size_t need = gu_bytes + rmm_linear_workspace_bytes(n, f, m, rho_down);  // both parts 256-byte multiples
+  if ((need > 0 && ws == nullptr) || ws_bytes < need)
+    return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // gate and up: one selection on X, one fused product writing H = SiLU(gate) * up
+  const uint16_t* A = X;
+  int64_t K = d, lda = ldx;
+  const uint16_t* Bg = Wg;
+  const uint16_t* Bu = Wu;
+  int64_t ldb = ldw;
+  if (k < d) {
+    Carver c(ws);
+    double* colsq = c.take<double>(d);
+    int32_t* idx_ws = c.take<int32_t>(k);
+    const int64_t k_pad = round_up(k, 8), f_pad = round_up(f, 8);
+    uint16_t* xpack = c.take<uint16_t>(n * k_pad);
+    uint16_t* gpack = c.take<uint16_t>(k * f_pad);
+    uint16_t* upack = c.take<uint16_t>(k * f_pad);
+    int32_t* idx = idx_gu_out ? idx_gu_out : idx_ws;
+    if (rmm_status st = launch_colsq(X, 1, 0, n, d, ldx, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
+    if (rmm_status st = pack_columns(X, n, d, ldx, idx, k, xpack, k_pad, s)) return st;
+    if (rmm_status st = gather_rows(Wg, f, ldw, idx, k, gpack, f_pad, s)) return st;
+    if (rmm_status st = gather_rows(Wu, f, ldw, idx, k, upack, f_pad, s)) return st;
+    A = xpack;
+    K = k;
+    lda = k_pad;
+    Bg = gpack;
+    Bu = upack;
+    ldb = f_pad;
+  } else if (idx_gu_out != nullptr) {
+    const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024))),
+                                         dim3(256), 0, s, idx_gu_out, 1, d);
+    if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+  }
+  CUtensorMap ta, tg, tu;
+  if (rmm_status st = make_tmap(&ta, A, K, n, lda * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tg, Bg, f, K, ldb * 2, 64, 64)) return st;
+  if (rmm_status st = make_tmap(&tu, Bu, f, K, ldb * 2, 64, 64)) return st;
+  GemmParams g = gemm_defaults();
+  g.M = static_cast<int>(n);
+  g.N = static_cast<int>(f);
+  g.out = H;
+  g.ldo = ldh;
+  g.m_tiles = static_cast<int>(ceil_div(n, 256));
+  g.n_tiles = static_cast<int>(ceil_div(f, 128));
+  g.k = static_cast<int>(K);
+  g.num_kb = static_cast<int>(ceil_div(K, 64));
+  if (rmm_status st = launch_gemm_pair(ta, tg, g, s, &tu)) return st;
+
+  // down: RMM on H with its own rho and selection
+  uint8_t* ws_down = ws ? static_cast<uint8_t*>(ws) + gu_bytes : nullptr;
+  const size_t down_bytes = ws ? ws_bytes - gu_bytes : 0;
+  return rmm_linear(H, n, f, ldh, Wd, m, ldwd, Y, ldy, rho_down, idx_down_out, down_bytes ? ws_down : nullptr,
+                    down_bytes, stream);
 }
 
 // ---------------------------------------------------------------- decode attention

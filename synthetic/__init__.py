@@ -296,3 +296,21 @@ def decode_attention_inputs_device(device, seed: int | None = None, batch: int =
     P = P.to(torch.bfloat16)
     V = torch.randn((batch, hkv, nk, dh), generator=gen, device=device, dtype=f32).to(torch.bfloat16)
     return Q, Kt, P, V
+
+
+# ------------------------------------------------------------------ MLP block
+MLP_SEED = 7  # workload number of the MLP-block inputs
+
+
+def mlp_block(seed: int | None = None, n: int = 4096, d: int = 4096, f: int = 14336, m: int | None = None):
+    """Gated-MLP operands (Llama-3.1-8B shape by default): X [n, d] with N(0,1) entries
+    times LogNormal(0, 1.5) column scales; Wg, Wu [d, f] ~ N(0, 1/d); Wd [f, m] ~ N(0, 1/f)
+    with m = d.  bfloat16 CPU tensors."""
+    base = seed_for(MLP_SEED) if seed is None else seed
+    m = d if m is None else m
+    g = rng(base)
+    X = outlier_activations(g, n, d, 1.5)
+    Wg = gaussian_weight(g, d, f)
+    Wu = gaussian_weight(g, d, f)
+    Wd = gaussian_weight(g, f, m)
+    return to_bf16(X), to_bf16(Wg), to_bf16(Wu), to_bf16(Wd)

@@ -158,3 +158,19 @@ def test_decode_attention_argument_errors(L):
     assert dpv(nk=40000, ldp=40000, cap=40000) == UNSUPPORTED
     assert dpv() == WORKSPACE
     assert L.rmm_decode_pv_workspace_bytes(1, 8, 2, 100, 128, 1.0) > 0  # partial sums even at rho = 1
+
+
+def test_mlp_argument_errors(L):
+    def mlp(X=P16, n=300, d=512, ldx=512, Wg=P16, Wu=P16, f=1024, ldw=1024, Wd=P16, m=512, ldwd=512, H=P16,
+            ldh=1024, Y=P16, ldy=512, rg=0.5, rd=0.5, ws=None, wsb=0):
+        return L.rmm_mlp(X, n, d, ldx, Wg, Wu, f, ldw, Wd, m, ldwd, H, ldh, Y, ldy, rg, rd, None, None, ws, wsb, None)
+    assert mlp(rg=0.0) == INVALID
+    assert mlp(rd=1.5) == INVALID
+    assert mlp(H=None) == INVALID
+    assert mlp(ldh=1000) == INVALID          # ldh < f
+    assert mlp(ldw=1028) == UNSUPPORTED
+    assert mlp(d=40000, ldx=40000) == UNSUPPORTED
+    assert mlp() == WORKSPACE
+    a = L.rmm_mlp_workspace_bytes(300, 512, 1024, 512, 0.5, 0.5)
+    assert a >= L.rmm_linear_workspace_bytes(300, 1024, 512, 0.5) + 300 * 256 * 2 + 2 * 256 * 1024 * 2
+    assert L.rmm_mlp_workspace_bytes(300, 512, 1024, 512, 1.0, 1.0) == 0
