@@ -45,6 +45,7 @@ __all__ = [
     "retained_energy", "select", "reduced_product", "error_bound", "rmm_linear",
     "rmm_linear_rows", "kv_head", "rmm_qk", "rmm_qk_rows", "rmm_pv", "rmm_pv_rows",
     "near_tie_band", "rmm_decode_qk", "rmm_decode_pv", "silu", "rmm_mlp_gate_up", "rmm_mlp",
+    "rmm_linear_int8",
 ]
 
 
@@ -360,3 +361,20 @@ def rmm_mlp(X, Wg, Wu, Wd, rho_gu: float, rho_down: float):
     gu = rmm_mlp_gate_up(X, Wg, Wu, rho_gu)
     down = rmm_linear(gu["H"], Wd, rho_down)
     return {"H": gu["H"], "I_gu": gu["I"], "Y": down["Y"], "I_down": down["I"]}
+
+
+def rmm_linear_int8(A: np.ndarray, Wq: np.ndarray, scale: np.ndarray, rho: float):
+    """Reduced projection with int8 weights: W = Wq * scale[None, :] (one scale per
+    output column), I chosen on A as in ``rmm_linear``, and
+        Y = (A[:, I] . Wq[I, :]) * scale[None, :].
+
+    [GS] "Compatibility" (the method works with INT8 weight quantization) and [DD]
+    "Compatibility & generalization" (INT8 + RMM: lower precision and fewer FLOPs
+    stack): the selection and the kept rows are those of the bf16 case; only the
+    stored weights are int8.  Returns dict(Y, I).
+    """
+    A = np.asarray(A, dtype=np.float64)
+    Wq = np.asarray(Wq, dtype=np.float64)
+    scale = np.asarray(scale, dtype=np.float64)
+    I, _, _ = select(A, rho)
+    return {"Y": (A[:, I] @ Wq[I, :]) * scale[None, :], "I": I}

@@ -400,3 +400,39 @@ def test_mlp_down_bound_and_silu_values():
         X, Wg, Wu, Wd = g.standard_normal((5, 8)), g.standard_normal((8, 6)), g.standard_normal((8, 6)), g.standard_normal((6, 4))
         r = oracle.rmm_mlp(X, Wg, Wu, Wd, 0.7, 0.5)
         assert np.linalg.norm(r["H"] @ Wd - r["Y"]) <= oracle.error_bound(r["H"], Wd, r["I_down"]) + 1e-9
+
+
+# ----------------------------------------------------------------- int8 weights
+def test_int8_hand_fixture():
+    fx = load("int8_hand.json")
+    r = oracle.rmm_linear_int8(np.array(fx["A"], float), np.array(fx["Wq"], float), np.array(fx["scale"]), fx["rho"])
+    assert list(r["I"]) == fx["I"]
+    assert np.allclose(r["Y"], np.array(fx["Y"]), rtol=0, atol=1e-12)
+
+
+def test_int8_rho_one_bruteforce_and_scale_per_column():
+    g = np.random.default_rng(13)
+    A = g.integers(-4, 5, size=(3, 6)).astype(float)
+    Wq = g.integers(-127, 128, size=(6, 5)).astype(float)
+    s = g.random(5) + 0.1
+    Y = oracle.rmm_linear_int8(A, Wq, s, 1.0)["Y"]
+    for i in range(3):
+        for c in range(5):
+            assert abs(Y[i, c] - s[c] * sum(A[i, j] * Wq[j, c] for j in range(6))) < 1e-9
+    # doubling one column's scale doubles that output column only
+    s2 = s.copy()
+    s2[2] *= 2.0
+    Y2 = oracle.rmm_linear_int8(A, Wq, s2, 1.0)["Y"]
+    assert np.allclose(Y2[:, 2], 2.0 * Y[:, 2]) and np.allclose(np.delete(Y2, 2, 1), np.delete(Y, 2, 1))
+
+
+def test_int8_keeps_the_bf16_selection():
+    """The index set depends on A only: the same I as the bf16 projection for any weights."""
+    g = np.random.default_rng(14)
+    A = g.standard_normal((4, 20)) * np.exp(g.standard_normal(20))
+    Wq = g.integers(-127, 128, size=(20, 7)).astype(float)
+    r = oracle.rmm_linear_int8(A, Wq, np.ones(7), 0.4)
+    assert np.array_equal(r["I"], oracle.select(A, 0.4)[0])
+    keep = np.zeros(20, bool)
+    keep[r["I"]] = True
+    assert np.allclose(r["Y"], A[:, keep] @ Wq[keep], rtol=1e-12, atol=1e-9)
