@@ -309,7 +309,36 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
             row[r]["speedup_vs_rho1"] = row["1.0"]["ms"] / row[r]["ms"]
         dec[f"n={n}"] = row
     out["decode_70b_mlp_up"] = dec
+
+    # the same decode shape with int8 weights (one fp32 scale per output column):
+    # algorithmic bytes = kept int8 rows k*m + scores n*d*2 (rho < 1) + x n*k*2 + Y n*m*2
+    Wq, sc = synthetic.int8_weight(synthetic.rng(synthetic.seed_for(3) + 100), 8192, 28672)
+    Wq, sc = Wq.to(dev), sc.to(dev)
     del W
+    torch.cuda.empty_cache()
+    dq = {}
+    for n in (1, 8):
+        x, _ = synthetic.decode_gemv(n, weight=False)
+        x = x.to(dev)
+        d, m = 8192, 28672
+        Y = torch.empty((n, m), dtype=torch.bfloat16, device=dev)
+        row = {}
+        for r in (1.0, 0.9, 0.7, 0.5):
+            ws = torch.empty(max(L.rmm_linear_int8_workspace_bytes(n, d, m, r), 256), dtype=torch.uint8, device=dev)
+            ms = timed_call(lambda: ok(L.rmm_linear_int8(x.data_ptr(), n, d, d, Wq.data_ptr(), m, m, sc.data_ptr(),
+                                                         Y.data_ptr(), m, r, None, ws.data_ptr(), ws.numel(), sptr)))
+            k = k_of(r, d)
+            nbytes = k * m + (n * d * 2 if k < d else 0) + n * k * 2 + n * m * 2
+            row[str(r)] = {"k": k, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                           "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
+                           "vs_bf16_same_rho": dec[f"n={n}"][str(r)]["ms"] / ms}
+            del ws
+        for r in row:
+            row[r]["speedup_vs_rho1"] = row["1.0"]["ms"] / row[r]["ms"]
+        dq[f"n={n}"] = row
+    out["decode_70b_mlp_up_int8"] = dq
+    del Wq, sc
+    torch.cuda.empty_cache()
 
     # GQA QK^T: 32 query heads / 8 key heads, seq 4096, head_dim 128, causal fp32 scores
     Q, K = synthetic.qk_inputs()

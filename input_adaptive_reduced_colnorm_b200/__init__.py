@@ -53,6 +53,9 @@ _SIGNATURES = {
     "rmm_pv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_pv": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_dbl, _c_p, _c_p,
                         _c_size, _c_p]),
+    "rmm_linear_int8_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_linear_int8": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_dbl,
+                                 _c_p, _c_p, _c_size, _c_p]),
     "rmm_mlp_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_dbl, _c_dbl]),
     "rmm_mlp": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64,
                          _c_p, _c_i64, _c_dbl, _c_dbl, _c_p, _c_p, _c_p, _c_size, _c_p]),
@@ -269,6 +272,29 @@ def pv(P, V, rho: float, *, causal: bool = True, out=None, return_idx: bool = Fa
     ws = _workspace(L.rmm_pv_workspace_bytes(b, h, hkv, nq, nk, dh, float(rho)), dev, workspace)
     _check(L.rmm_pv(_ptr(P), _ptr(V), _ptr(out), b, h, hkv, nq, nk, dh, int(causal), float(rho), _ptr(idx),
                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def linear_int8(A, Wq, scale, rho: float, *, out=None, return_idx: bool = False, workspace=None):
+    """Y = (A[:, I] Wq[I, :]) * scale with I chosen on A (decode, n <= 8 rows).
+    A [n, d] bf16, Wq [d, m] int8, scale [m] float32, all CUDA."""
+    import torch
+    _require(A, "A", torch.bfloat16, 2)
+    _require(Wq, "Wq", torch.int8, 2)
+    _require(scale, "scale", torch.float32, 1)
+    n, d = A.shape
+    d2, m = Wq.shape
+    if d2 != d or scale.numel() != m:
+        raise ValueError("A / Wq / scale shape mismatch")
+    dev = A.device
+    if out is None:
+        out = torch.empty((n, m), dtype=torch.bfloat16, device=dev)
+    Lb = lib()
+    idx = torch.empty((max(rmm_k(rho, d), 0),), dtype=torch.int32, device=dev) if return_idx else None
+    ws = _workspace(Lb.rmm_linear_int8_workspace_bytes(n, d, m, float(rho)), dev, workspace)
+    _check(Lb.rmm_linear_int8(_ptr(A), n, d, A.stride(0), _ptr(Wq), m, Wq.stride(0), _ptr(scale), _ptr(out),
+                              out.stride(0), float(rho), _ptr(idx), _ptr(ws), 0 if ws is None else ws.numel(),
+                              _stream(dev)))
     return (out, idx) if return_idx else out
 
 

@@ -20,6 +20,7 @@
 #include "gemm_pair.cuh"
 #include "gemv.cuh"
 #include "decode_attn.cuh"
+#include "gemv_i8.cuh"
 
 using namespace rmm;
 
@@ -625,6 +626,114 @@ int64_t rmm_k(double rho, int64_t d) {
   if (k < 1) k = 1;
   if (k > d) k = d;
   return k;
+}
+
+// ---------------------------------------------------------------- int8 weights
+}  // extern "C"
+
+namespace {
+// Row chunks of the int8 GEMV: about four CTAs per SM over all column blocks,
+// at most kI8MaxChunk rows each, and few enough chunks that the fp32 partial
+// sums (chunks x n x m x 4 bytes) stay near 12 % of the kept int8 rows.
+void i8_plan(int64_t n, int64_t k, int64_t m, int* chunk, int* chunks) {
+  const int64_t col_blocks = ceil_div(m, 2048);
+  int64_t c = ceil_div(4LL * num_sms(), col_blocks);
+  const int64_t by_bytes = std::max<int64_t>(1, (3 * k) / (100 * n));
+  c = std::max<int64_t>(1, std::min(c, by_bytes));
+  int64_t len = round_up(ceil_div(k, c), 16);
+  if (len > kI8MaxChunk) len = kI8MaxChunk;
+  *chunk = static_cast<int>(len);
+  *chunks = static_cast<int>(ceil_div(k, len));
+}
+
+template <int NR>
+cudaError_t launch_gemv_i8_t(const GemvI8Params& p, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(ceil_div(p.m, 2048)), static_cast<unsigned>(p.chunks));
+  return launch_chained(gemv_i8_kernel<NR>, grid, dim3(256), 0, s, p);
+}
+}  // namespace
+
+extern "C" {
+
+size_t rmm_linear_int8_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
+  const int64_t k = rmm_k(rho, d);
+  if (k < 0 || n < 1 || m < 1) return 0;
+  int chunk = 0, chunks = 0;
+  i8_plan(n, k, m, &chunk, &chunks);
+  Carver c(nullptr);
+  if (k < d) {
+    c.take<double>(d);
+    c.take<int32_t>(k);
+    c.take<uint16_t>(n * round_up(k, 8));
+  }
+  c.take<float>(static_cast<int64_t>(chunks) * n * m);
+  return c.bytes();
+}
+
+rmm_status rmm_linear_int8(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int8_t* Wq, int64_t m,
+                           int64_t ldw, const float* scale, rmm_bf16* Y, int64_t ldy, double rho, int32_t* idx_out,
+                           void* ws, size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (A == nullptr || Wq == nullptr || scale == nullptr || Y == nullptr)
+    return fail(RMM_ERR_INVALID_ARG, "A, Wq, scale and Y are required");
+  if (n < 1 || d < 1 || m < 1) return fail(RMM_ERR_INVALID_ARG, "n, d and m must be >= 1");
+  if (lda < d || ldw < m || ldy < m) return fail(RMM_ERR_INVALID_ARG, "leading dimension too small");
+  if (n > kI8MaxRows) return fail(RMM_ERR_UNSUPPORTED, "the int8 path takes at most 8 activation rows");
+  if (!aligned16(A) || !aligned16(Wq) || !aligned16(Y) || (ws != nullptr && !aligned16(ws)) || (lda % 8) ||
+      (ldw % 8) || (ldy % 8) || (m % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers 16-byte aligned; lda, ldw, ldy and m multiples of 8");
+  if (d > kMaxSelectD || m > kIntMax || static_cast<int64_t>(d) * ldw > (1LL << 40))
+    return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  const size_t need = rmm_linear_int8_workspace_bytes(n, d, m, rho);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t k = rmm_k(rho, d);
+  int chunk = 0, chunks = 0;
+  i8_plan(n, k, m, &chunk, &chunks);
+  if (chunks > 65535) return fail(RMM_ERR_UNSUPPORTED, "too many row chunks");
+  Carver c(ws);
+  GemvI8Params p{};
+  p.W = Wq;
+  p.ldw = ldw;
+  p.x = A;
+  p.ldx = lda;
+  p.k = static_cast<int>(k);
+  p.m = static_cast<int>(m);
+  p.n = static_cast<int>(n);
+  p.chunk = chunk;
+  p.chunks = chunks;
+  if (k < d) {
+    double* colsq = c.take<double>(d);
+    int32_t* idx_ws = c.take<int32_t>(k);
+    const int64_t k_pad = round_up(k, 8);
+    uint16_t* xpack = c.take<uint16_t>(n * k_pad);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
+    if (rmm_status st = pack_columns(A, n, d, lda, idx, k, xpack, k_pad, s)) return st;
+    p.x = xpack;
+    p.ldx = k_pad;
+    p.idx = idx;
+  } else if (idx_out != nullptr) {
+    const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024))),
+                                         dim3(256), 0, s, idx_out, 1, d);
+    if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+  }
+  float* partial = c.take<float>(static_cast<int64_t>(chunks) * n * m);
+  p.partial = partial;
+  cudaError_t e = cudaSuccess;
+  if (n == 1) e = launch_gemv_i8_t<1>(p, s);
+  else if (n == 2) e = launch_gemv_i8_t<2>(p, s);
+  else if (n <= 4) e = launch_gemv_i8_t<4>(p, s);
+  else e = launch_gemv_i8_t<8>(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "int8 GEMV launch");
+  e = launch_chained(gemv_i8_fixup_kernel, dim3(static_cast<unsigned>(ceil_div(m, 256)), static_cast<unsigned>(n)), dim3(256),
+                     0, s, static_cast<const float*>(partial), scale, chunks, static_cast<int>(n), static_cast<int>(m),
+                     reinterpret_cast<uint16_t*>(Y), ldy);
+  if (e != cudaSuccess) return cuda_fail(e, "int8 GEMV fix-up launch");
+  return RMM_OK;
 }
 
 // ---------------------------------------------------------------- MLP block

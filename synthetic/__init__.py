@@ -314,3 +314,13 @@ def mlp_block(seed: int | None = None, n: int = 4096, d: int = 4096, f: int = 14
     Wu = gaussian_weight(g, d, f)
     Wd = gaussian_weight(g, f, m)
     return to_bf16(X), to_bf16(Wg), to_bf16(Wu), to_bf16(Wd)
+
+
+def int8_weight(g: np.random.Generator, d: int, m: int):
+    """A N(0, 1/d) weight quantized to int8 with one scale per output column:
+    scale_c = max_j |W[j, c]| / 127, Wq = round(W / scale) clipped to [-127, 127].
+    Returns (Wq int8 CPU tensor [d, m], scale float32 CPU tensor [m])."""
+    w = gaussian_weight(g, d, m)
+    scale = np.maximum(np.abs(w).max(axis=0), np.float32(1e-30)) / np.float32(127.0)
+    q = np.clip(np.rint(w / scale[None, :]), -127, 127).astype(np.int8)
+    return torch.from_numpy(q), torch.from_numpy(scale.astype(np.float32))

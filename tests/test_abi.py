@@ -174,3 +174,15 @@ def test_mlp_argument_errors(L):
     a = L.rmm_mlp_workspace_bytes(300, 512, 1024, 512, 0.5, 0.5)
     assert a >= L.rmm_linear_workspace_bytes(300, 1024, 512, 0.5) + 300 * 256 * 2 + 2 * 256 * 1024 * 2
     assert L.rmm_mlp_workspace_bytes(300, 512, 1024, 512, 1.0, 1.0) == 0
+
+
+def test_int8_argument_errors(L):
+    def li8(A=P16, n=4, d=512, lda=512, W=P16, m=1024, ldw=1024, s=P16, Y=P16, ldy=1024, rho=0.5, ws=None, wsb=0):
+        return L.rmm_linear_int8(A, n, d, lda, W, m, ldw, s, Y, ldy, rho, None, ws, wsb, None)
+    assert li8(s=None) == INVALID
+    assert li8(rho=0.0) == INVALID
+    assert li8(n=9) == UNSUPPORTED
+    assert li8(m=1020, ldw=1024, ldy=1024) == UNSUPPORTED  # m not a multiple of 8
+    assert li8(ldw=1028) == UNSUPPORTED                    # ldw not a multiple of 8
+    assert li8() == WORKSPACE
+    assert L.rmm_linear_int8_workspace_bytes(1, 8192, 28672, 1.0) > 0  # fp32 partial sums
