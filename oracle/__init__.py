@@ -45,7 +45,7 @@ __all__ = [
     "retained_energy", "select", "reduced_product", "error_bound", "rmm_linear",
     "rmm_linear_rows", "kv_head", "rmm_qk", "rmm_qk_rows", "rmm_pv", "rmm_pv_rows",
     "near_tie_band", "rmm_decode_qk", "rmm_decode_pv", "silu", "rmm_mlp_gate_up", "rmm_mlp",
-    "rmm_linear_int8",
+    "rmm_linear_int8", "rmm_attention",
 ]
 
 
@@ -378,3 +378,35 @@ def rmm_linear_int8(A: np.ndarray, Wq: np.ndarray, scale: np.ndarray, rho: float
     scale = np.asarray(scale, dtype=np.float64)
     I, _, _ = select(A, rho)
     return {"Y": (A[:, I] @ Wq[I, :]) * scale[None, :], "I": I}
+
+
+def rmm_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rho: float, causal: bool = True,
+                  scale: float = 1.0):
+    """Attention whose score product is reduced: per query head h,
+        S_h = scale * Q_h[:, I_h] K_g(h)[:, I_h]^T   (I_h = TopK of Q_h's column norms,
+                                                    -inf above the causal diagonal)
+        O_h = softmax_rows(S_h) V_g(h)               (the value product is not reduced)
+
+    [DD] "Component mapping" (QK^T selects head dims on Q) and "Attention vs MLP"
+    (Table 16: attention-internal reduction of QK^T); [KB] "计算 attention score 时".
+    Softmax and the value product are the ordinary ones: a selection of P's
+    columns would need P whole before the product, so only the score product is
+    reduced here.  Q [B, Hq, nq, dh], K / V [B, Hkv, nk, dh] -> O [B, Hq, nq, dh], I.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    Bsz, hq, nq, dh = Q.shape
+    hkv = K.shape[1]
+    k = retention_count(rho, dh)
+    O = np.empty((Bsz, hq, nq, V.shape[3]))
+    I = np.empty((Bsz, hq, k), dtype=np.int64)
+    for b in range(Bsz):
+        for h in range(hq):
+            g = kv_head(h, hq, hkv)
+            S, I[b, h] = _qk_head(Q[b, h], K[b, g], rho, causal, scale)
+            S = S - S.max(axis=1, keepdims=True)
+            P = np.exp(S)
+            P /= P.sum(axis=1, keepdims=True)
+            O[b, h] = P @ V[b, g]
+    return {"O": O, "I": I}

@@ -436,3 +436,48 @@ def test_int8_keeps_the_bf16_selection():
     keep = np.zeros(20, bool)
     keep[r["I"]] = True
     assert np.allclose(r["Y"], A[:, keep] @ Wq[keep], rtol=1e-12, atol=1e-9)
+
+
+# ----------------------------------------------------------------- fused reduced attention
+def test_attention_hand_fixture():
+    fx = load("attention_hand.json")
+    Q, K, V = (np.array(fx[n], dtype=np.float64) for n in ("Q", "K", "V"))
+    r = oracle.rmm_attention(Q, K, V, fx["rho"], causal=True, scale=fx["scale"])
+    assert list(r["I"][0, 0]) == fx["I"]
+    assert np.allclose(r["O"][0, 0], np.array(fx["O_causal"]), rtol=0, atol=1e-12)
+    nc = oracle.rmm_attention(Q, K, V, fx["rho"], causal=False)
+    assert np.allclose(nc["O"][0, 0, 0], fx["O_noncausal_row0"], rtol=0, atol=1e-12)
+    dense = oracle.rmm_attention(Q, K, V, 1.0, causal=False)
+    assert np.allclose(dense["O"][0, 0, 0], fx["O_dense_noncausal_row0"], rtol=0, atol=1e-12)
+
+
+def test_attention_rho_one_bruteforce_gqa_causal():
+    g = np.random.default_rng(15)
+    B, hq, hkv, n, dh = 1, 4, 2, 5, 3
+    Q, K, V = g.standard_normal((B, hq, n, dh)), g.standard_normal((B, hkv, n, dh)), g.standard_normal((B, hkv, n, dh))
+    O = oracle.rmm_attention(Q, K, V, 1.0, causal=True, scale=0.7)["O"]
+    for h in range(hq):
+        gk = h // 2
+        for i in range(n):
+            sc = [0.7 * sum(Q[0, h, i, t] * K[0, gk, j, t] for t in range(dh)) for j in range(i + 1)]
+            mx = max(sc)
+            w = [math.exp(x - mx) for x in sc]
+            for c in range(dh):
+                ref = sum(w[j] * V[0, gk, j, c] for j in range(i + 1)) / sum(w)
+                assert abs(O[0, h, i, c] - ref) < 1e-12
+
+
+def test_attention_rows_are_convex_combinations_and_first_row_is_v0():
+    """Softmax weights are positive and sum to one, so each output row lies within
+    the per-column range of the visible V rows; under a causal mask with nq = nk the
+    first query sees only key 0."""
+    g = np.random.default_rng(16)
+    Q, K, V = g.standard_normal((1, 2, 9, 8)), g.standard_normal((1, 1, 9, 8)), g.standard_normal((1, 1, 9, 8))
+    O = oracle.rmm_attention(Q, K, V, 0.5, causal=True)["O"]
+    for h in range(2):
+        assert np.allclose(O[0, h, 0], V[0, 0, 0], rtol=0, atol=1e-12)
+        for i in range(9):
+            lo, hi = V[0, 0, :i + 1].min(axis=0), V[0, 0, :i + 1].max(axis=0)
+            assert np.all(O[0, h, i] >= lo - 1e-12) and np.all(O[0, h, i] <= hi + 1e-12)
+    # the same index sets as the score product alone
+    assert np.array_equal(oracle.rmm_attention(Q, K, V, 0.5)["I"], oracle.rmm_qk(Q, K, 0.5)["I"])
