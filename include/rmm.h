@@ -197,6 +197,25 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
                   int64_t nq, int64_t nk, int64_t dh, int causal, double rho, int32_t* idx_out, void* ws,
                   size_t ws_bytes, rmm_stream stream);
 
+/* ---------------------------------------------------------------- fused reduced attention
+ * O_h = softmax_rows(scale * Q_h[:, I_h] K_g(h)[:, I_h]^T, causal) V_g(h) in one
+ * kernel, S and P kept on chip ("Algorithm Deep-Dive: RMM", Component mapping:
+ * QK^T selects head dims by the Q column norm, K gathers them under GQA; Attention
+ * vs MLP, Table 16: attention-internal reduction).  I_h is chosen exactly as in
+ * rmm_qk; the softmax and the value product are the ordinary ones.  When
+ * k = rmm_k(rho, dh) <= 64 the score product contracts over 64 packed dims,
+ * otherwise over 128 with the dropped dims zeroed.
+ *   Q  device bf16 [batch][hq][nq][dh], K / V [batch][hkv][nk][dh], contiguous.
+ *   O  device bf16 [batch][hq][nq][dh].
+ *   causal = 1: bottom-right aligned (key j visible to query i iff j <= i + nk - nq),
+ *   requires nq <= nk.  idx_out device int32 [batch][hq][k] or NULL.
+ * Requires dh == 128.  Workspace: rmm_attention_workspace_bytes (0 at rho = 1). */
+size_t rmm_attention_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh,
+                                     double rho);
+rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V, rmm_bf16* O, int64_t batch,
+                         int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, int causal, float scale,
+                         double rho, int32_t* idx_out, void* ws, size_t ws_bytes, rmm_stream stream);
+
 /* ---------------------------------------------------------------- int8 weights
  * Reduced projection with int8 weights for decode (n <= 8 rows):
  *   Y = (A[:, I] . Wq[I, :]) * scale[None, :]

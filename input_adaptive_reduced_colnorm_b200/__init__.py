@@ -53,6 +53,9 @@ _SIGNATURES = {
     "rmm_pv_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_pv": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_dbl, _c_p, _c_p,
                         _c_size, _c_p]),
+    "rmm_attention_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
+    "rmm_attention": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int,
+                               ctypes.c_float, _c_dbl, _c_p, _c_p, _c_size, _c_p]),
     "rmm_linear_int8_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_linear_int8": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_dbl,
                                  _c_p, _c_p, _c_size, _c_p]),
@@ -272,6 +275,32 @@ def pv(P, V, rho: float, *, causal: bool = True, out=None, return_idx: bool = Fa
     ws = _workspace(L.rmm_pv_workspace_bytes(b, h, hkv, nq, nk, dh, float(rho)), dev, workspace)
     _check(L.rmm_pv(_ptr(P), _ptr(V), _ptr(out), b, h, hkv, nq, nk, dh, int(causal), float(rho), _ptr(idx),
                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
+    return (out, idx) if return_idx else out
+
+
+def attention(Q, K, V, rho: float, *, causal: bool = True, scale: float = 1.0, out=None, return_idx: bool = False,
+              workspace=None):
+    """Fused attention with a reduced score product: O = softmax(scale Q_I K_I^T) V per
+    query head.  Q [B, Hq, nq, 128], K / V [B, Hkv, nk, 128] bf16 contiguous -> O
+    [B, Hq, nq, 128] bf16."""
+    import torch
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V")):
+        _require(t, nm, torch.bfloat16, 4)
+        if not t.is_contiguous():
+            raise ValueError(f"{nm} must be contiguous")
+    b, hq, nq, dh = Q.shape
+    b2, hkv, nk, dh2 = K.shape
+    if b2 != b or dh2 != dh or V.shape != K.shape:
+        raise ValueError("Q / K / V shape mismatch")
+    dev = Q.device
+    if out is None:
+        out = torch.empty((b, hq, nq, dh), dtype=torch.bfloat16, device=dev)
+    k = rmm_k(rho, dh)
+    idx = torch.empty((b, hq, max(k, 0)), dtype=torch.int32, device=dev) if return_idx else None
+    Lb = lib()
+    ws = _workspace(Lb.rmm_attention_workspace_bytes(b, hq, hkv, nq, nk, dh, float(rho)), dev, workspace)
+    _check(Lb.rmm_attention(_ptr(Q), _ptr(K), _ptr(V), _ptr(out), b, hq, hkv, nq, nk, dh, int(causal), float(scale),
+                            float(rho), _ptr(idx), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev)))
     return (out, idx) if return_idx else out
 
 

@@ -21,6 +21,7 @@
 #include "gemv.cuh"
 #include "decode_attn.cuh"
 #include "gemv_i8.cuh"
+#include "attention.cuh"
 
 using namespace rmm;
 
@@ -626,6 +627,152 @@ int64_t rmm_k(double rho, int64_t d) {
   if (k < 1) k = 1;
   if (k > d) k = d;
   return k;
+}
+
+// ---------------------------------------------------------------- fused reduced attention
+}  // extern "C"
+
+namespace {
+// Workspace of rmm_attention (rho < 1): scores, index sets and either the packed
+// Q[:, I] / K[:, I] per query head (k <= 64: the score product contracts over 64
+// dims) or keep bytes and Q with the dropped dims zeroed (k > 64: 128 dims, K as is).
+size_t attention_bytes(int64_t items, int64_t nq, int64_t nk, int64_t dh, int64_t k) {
+  if (k == dh) return 0;
+  Carver c(nullptr);
+  c.take<double>(items * dh);
+  c.take<int32_t>(items * k);
+  if (k <= 64) {
+    c.take<uint16_t>(items * nq * 64);
+    c.take<uint16_t>(items * nk * 64);
+  } else {
+    c.take<uint8_t>(items * dh);
+    c.take<uint16_t>(items * nq * dh);
+  }
+  return c.bytes();
+}
+}  // namespace
+
+extern "C" {
+
+size_t rmm_attention_workspace_bytes(int64_t batch, int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh,
+                                     double rho) {
+  (void)hkv;
+  const int64_t k = rmm_k(rho, dh);
+  if (k < 0 || batch < 1 || hq < 1 || nq < 1 || nk < 1) return 0;
+  return attention_bytes(batch * hq, nq, nk, dh, k);
+}
+
+rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V, rmm_bf16* O, int64_t batch,
+                         int64_t hq, int64_t hkv, int64_t nq, int64_t nk, int64_t dh, int causal, float scale,
+                         double rho, int32_t* idx_out, void* ws, size_t ws_bytes, rmm_stream stream) {
+  t_last_error.clear();
+  if (rmm_status st = check_rho(rho)) return st;
+  if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr)
+    return fail(RMM_ERR_INVALID_ARG, "Q, K, V and O are required");
+  if (batch < 1 || hq < 1 || hkv < 1 || nq < 1 || nk < 1 || dh < 1) return fail(RMM_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (hq % hkv) return fail(RMM_ERR_INVALID_ARG, "hq must be a multiple of hkv");
+  if (causal != 0 && causal != 1) return fail(RMM_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (!std::isfinite(scale)) return fail(RMM_ERR_INVALID_ARG, "scale must be finite");
+  if (dh != 128) return fail(RMM_ERR_UNSUPPORTED, "the fused attention kernel takes head dim 128");
+  if (causal && nq > nk) return fail(RMM_ERR_UNSUPPORTED, "causal attention needs nq <= nk (every query sees a key)");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (ws != nullptr && !aligned16(ws)))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+  const int64_t items = batch * hq;
+  const int64_t m_tiles = ceil_div(nq, 128);
+  if (items * nq > kIntMax - 256 || items * nk > kIntMax - 256 || batch * hkv * nk > kIntMax - 256 ||
+      items * m_tiles > kIntMax)
+    return fail(RMM_ERR_UNSUPPORTED, "problem too large");
+  const int64_t k = rmm_k(rho, dh);
+  const size_t need = attention_bytes(items, nq, nk, dh, k);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  AttnParams ap{};
+  ap.nq = static_cast<int>(nq);
+  ap.nk = static_cast<int>(nk);
+  ap.hq = static_cast<int>(hq);
+  ap.hkv = static_cast<int>(hkv);
+  ap.items = static_cast<int>(items);
+  ap.m_tiles = static_cast<int>(m_tiles);
+  ap.causal = causal;
+  ap.causal_off = nk - nq;
+  ap.scale_log2 = scale * 1.4426950408889634f;
+  ap.O = O;
+  const uint16_t* qsrc = Q;
+  const uint16_t* ksrc = K;
+  ap.kp = 128;
+  ap.k_per_item = 0;
+  if (k < dh) {
+    Carver c(ws);
+    double* colsq = c.take<double>(items * dh);
+    int32_t* idx_ws = c.take<int32_t>(items * k);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (rmm_status st = launch_colsq(Q, items, nq * dh, nq, dh, dh, false, 0, colsq, s)) return st;
+    if (k <= 64) {
+      uint16_t* qp = c.take<uint16_t>(items * nq * 64);
+      uint16_t* kpk = c.take<uint16_t>(items * nk * 64);
+      if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s)) return st;
+      PackParams pq{};
+      pq.src = Q;
+      pq.src_ld = dh;
+      pq.rows = nq;
+      pq.d = dh;
+      pq.g_outer = 1;
+      pq.g_inner = 1;
+      pq.s_outer = nq * dh;
+      pq.idx = idx;
+      pq.k = k;
+      pq.k_pad = 64;
+      pq.dst = qp;
+      pq.batch = items;
+      if (rmm_status st = launch_pack(pq, s)) return st;
+      PackParams pk = pq;  // K of the query head's key/value head, gathered with the query head's I
+      pk.src = K;
+      pk.rows = nk;
+      pk.g_outer = hq;
+      pk.g_inner = hq / hkv;
+      pk.s_outer = hkv * nk * dh;
+      pk.s_inner = nk * dh;
+      pk.dst = kpk;
+      if (rmm_status st = launch_pack(pk, s)) return st;
+      qsrc = qp;
+      ksrc = kpk;
+      ap.kp = 64;
+      ap.k_per_item = 1;
+    } else {
+      uint8_t* keep = c.take<uint8_t>(items * dh);
+      uint16_t* qm = c.take<uint16_t>(items * nq * dh);
+      if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s, keep)) return st;
+      MaskParams mp{};
+      mp.src = Q;
+      mp.dst = qm;
+      mp.rows = nq;
+      mp.cols = dh;
+      mp.keep = keep;
+      mp.by_rows = 0;
+      mp.batch = items;
+      mp.g_outer = 1;
+      mp.g_inner = 1;
+      mp.s_outer = nq * dh;
+      if (rmm_status st = launch_mask(mp, s)) return st;
+      qsrc = qm;
+    }
+  } else if (idx_out != nullptr) {
+    const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(items * dh, 256), 1024))),
+                                         dim3(256), 0, s, idx_out, items, dh);
+    if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+  }
+  CUtensorMap tq, tk, tv;
+  if (rmm_status st = make_tmap(&tq, qsrc, ap.kp, items * nq, ap.kp * 2, 64, 128)) return st;
+  const int64_t krows = ap.k_per_item ? items * nk : batch * hkv * nk;
+  if (rmm_status st = make_tmap(&tk, ksrc, ap.kp, krows, ap.kp * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tv, V, dh, batch * hkv * nk, dh * 2, 64, 64)) return st;
+  cudaError_t e = cudaFuncSetAttribute(attn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  if (e != cudaSuccess) return cuda_fail(e, "attention attribute");
+  e = launch_chained(attn_fused_kernel, dim3(static_cast<unsigned>(items * m_tiles)), dim3(192), kAttnSmem, s, tq, tk, tv,
+                     ap);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return RMM_OK;
 }
 
 // ---------------------------------------------------------------- int8 weights

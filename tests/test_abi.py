@@ -186,3 +186,18 @@ def test_int8_argument_errors(L):
     assert li8(ldw=1028) == UNSUPPORTED                    # ldw not a multiple of 8
     assert li8() == WORKSPACE
     assert L.rmm_linear_int8_workspace_bytes(1, 8192, 28672, 1.0) > 0  # fp32 partial sums
+
+
+def test_attention_argument_errors(L):
+    def att(Q=P16, K=P16, V=P16, O=P16, b=1, hq=4, hkv=2, nq=256, nk=256, dh=128, causal=1, scale=0.1, rho=0.5,
+            ws=None, wsb=0):
+        return L.rmm_attention(Q, K, V, O, b, hq, hkv, nq, nk, dh, causal, scale, rho, None, ws, wsb, None)
+    assert att(hkv=3) == INVALID
+    assert att(V=None) == INVALID
+    assert att(causal=2) == INVALID
+    assert att(dh=64) == UNSUPPORTED
+    assert att(nq=300, nk=256) == UNSUPPORTED   # causal with nq > nk
+    assert att() == WORKSPACE
+    assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 256, 128, 1.0) == 0
+    # k <= 64 packs Q and K per query head to 64 dims
+    assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 512, 128, 0.5) >= 4 * (256 + 512) * 64 * 2

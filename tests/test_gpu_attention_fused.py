@@ -1,0 +1,97 @@
+"""GPU parity of the fused attention with a reduced score product (rmm_attention):
+per query head, the index set of rmm_qk, then softmax(scale Q_I K_I^T) V with S
+and P kept on chip."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from parity import check_close, check_index_set
+
+pytestmark = pytest.mark.gpu
+
+rmm = pytest.importorskip("input_adaptive_reduced_colnorm_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from input_adaptive_reduced_colnorm_b200 import build
+    build.build()
+    yield
+    assert rmm.device_error() == 0
+
+
+def attention_ref(Qh, Kg, Vg, I, causal, scale, rows=None):
+    """Reference output rows of one head on the GPU's index set (float64)."""
+    nq, nk = Qh.shape[0], Kg.shape[0]
+    r = np.arange(nq) if rows is None else np.asarray(rows)
+    S = scale * (Qh[r][:, I] @ Kg[:, I].T)
+    if causal:
+        vis = r + (nk - nq) + 1
+        S[np.arange(nk)[None, :] >= vis[:, None]] = -np.inf
+    S -= S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P /= P.sum(axis=1, keepdims=True)
+    return P @ Vg
+
+
+def fused_parity(Q, K, V, rho, causal, scale, heads=None, rows=None):
+    O, idx = rmm.attention(Q.cuda(), K.cuda(), V.cuda(), rho, causal=causal, scale=scale, return_idx=True)
+    torch.cuda.synchronize()
+    B, hq, nq, dh = Q.shape
+    hkv = K.shape[1]
+    k = oracle.retention_count(rho, dh)
+    heads = range(hq) if heads is None else heads
+    for b in range(B):
+        for h in heads:
+            Qh = synthetic.widen(Q[b, h])
+            g = oracle.kv_head(h, hq, hkv)
+            I = idx[b, h].cpu().numpy().astype(np.int64)
+            check_index_set(I, oracle.column_sq_norms(Qh), k)
+            ref = attention_ref(Qh, synthetic.widen(K[b, g]), synthetic.widen(V[b, g]), I, causal, scale, rows)
+            r = np.arange(nq) if rows is None else np.asarray(rows)
+            check_close(synthetic.widen(O[b, h].cpu())[r], ref, f"fused attention head {h}")
+    return O, idx
+
+
+def qkv(hq, hkv, nq, nk, seed=40):
+    g = synthetic.rng(seed)
+    Q = synthetic.to_bf16(g.standard_normal((1, hq, nq, 128), dtype=np.float32) * np.exp(g.standard_normal(128)).astype(np.float32))
+    K = synthetic.to_bf16(g.standard_normal((1, hkv, nk, 128), dtype=np.float32))
+    V = synthetic.to_bf16(g.standard_normal((1, hkv, nk, 128), dtype=np.float32))
+    return Q, K, V
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.7, 1.0])
+@pytest.mark.parametrize("causal", [True, False])
+def test_fused_attention_small_gqa(rho, causal):
+    """4 query / 2 key-value heads, 300 rows (ragged last query tile and key block)."""
+    Q, K, V = qkv(4, 2, 300, 300)
+    fused_parity(Q, K, V, rho, causal, 0.088)
+
+
+def test_fused_attention_rectangular_causal():
+    """nq < nk: bottom-right alignment, several key blocks per query tile."""
+    Q, K, V = qkv(2, 1, 200, 520, seed=41)
+    fused_parity(Q, K, V, 0.5, True, 0.088)
+
+
+def test_fused_attention_matches_oracle_and_repeats():
+    Q, K, V = qkv(2, 1, 256, 256, seed=42)
+    O1, I1 = rmm.attention(Q.cuda(), K.cuda(), V.cuda(), 0.5, scale=0.1, return_idx=True)
+    O2 = rmm.attention(Q.cuda(), K.cuda(), V.cuda(), 0.5, scale=0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2)
+    ref = oracle.rmm_attention(synthetic.widen(Q), synthetic.widen(K), synthetic.widen(V), 0.5, causal=True, scale=0.1)
+    assert np.array_equal(I1.cpu().numpy(), ref["I"])
+    check_close(synthetic.widen(O1.cpu()), ref["O"], "fused attention entry point")
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.7])
+def test_fused_attention_gqa_seq4096_sampled(rho):
+    """32 query / 8 key-value heads, seq 4096, causal: sampled heads and rows."""
+    Q, K = synthetic.qk_inputs()
+    V = synthetic.to_bf16(synthetic.rng(43).standard_normal((1, 8, 4096, 128), dtype=np.float32))
+    rows = np.concatenate([np.arange(0, 4096, 397), [4095]])
+    fused_parity(Q, K, V, rho, True, 0.088, heads=[0, 5, 31], rows=rows)
