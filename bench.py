@@ -254,6 +254,7 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
     GQA QK^T, long-context PV) at their rho values and at rho = 1, each against its
     roofline: kept FLOPs at the bf16 peak or algorithmic bytes at the HBM peak."""
     import ctypes
+    import numpy as np
     import torch
     import synthetic
 
@@ -386,6 +387,33 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
         pv[r]["speedup_vs_rho1"] = pv["1.0"]["ms"] / pv[r]["ms"]
     out["pv_seq16384"] = pv
     del P, V, O, ws
+    torch.cuda.empty_cache()
+
+    # fused attention with a reduced score product: GQA 32 / 8 heads, seq 4096,
+    # head dim 128, causal; S and P stay on chip.  Kept FLOPs per head: 2 k pairs
+    # (scores) + 2 * 128 pairs (values), pairs = n (n + 1) / 2 visible (query, key).
+    # Algorithmic bytes: Q, K, V read once, O written.
+    Q, K = synthetic.qk_inputs()
+    V = synthetic.to_bf16(synthetic.rng(synthetic.seed_for(4) + 7).standard_normal((1, 8, 4096, 128), dtype=np.float32))
+    Q, K, V = Q.to(dev), K.to(dev), V.to(dev)
+    b_, hq, nq, dh = Q.shape
+    hkv, nk = K.shape[1], K.shape[2]
+    Oa = torch.empty_like(Q)
+    fa = {}
+    pairs = nq * (nq + 1) / 2 * hq * b_
+    for rho in (1.0, 0.7, 0.5):
+        wsa = torch.empty(max(L.rmm_attention_workspace_bytes(b_, hq, hkv, nq, nk, dh, rho), 256), dtype=torch.uint8,
+                          device=dev)
+        ms = timed_call(lambda: ok(L.rmm_attention(Q.data_ptr(), K.data_ptr(), V.data_ptr(), Oa.data_ptr(), b_, hq, hkv,
+                                                   nq, nk, dh, 1, 0.088, rho, None, wsa.data_ptr(), wsa.numel(), sptr)))
+        k = k_of(rho, dh)
+        flops = 2.0 * k * pairs + 2.0 * dh * pairs
+        fa[str(rho)] = {"k": k, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
+        del wsa
+    for r in fa:
+        fa[r]["speedup_vs_rho1"] = fa["1.0"]["ms"] / fa[r]["ms"]
+    out["attention_fused_gqa_seq4096"] = fa
+    del Q, K, V, Oa
     torch.cuda.empty_cache()
 
     # gated MLP block, Llama-3.1-8B at n = 4096 tokens (d = 4096, f = 14336): one

@@ -49,6 +49,13 @@ constexpr uint32_t kAttnVBytes = 128 * 128 * 2;  // one V block: 2 key halves x 
 constexpr uint32_t kAttnPBytes = 128 * 128 * 2;  // P tile, K-major over 128 keys (two atoms)
 constexpr int kAttnSmem = kAttnQBytes + 2 * kAttnKBytes + 2 * kAttnVBytes + kAttnPBytes + 1024 + 256;
 
+// 2^x with the hardware approximation (relative error ~2^-22; exp2(-inf) = 0).
+__device__ __forceinline__ float attn_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Visible key blocks of the query tile starting at row m0.
 __device__ __forceinline__ int attn_key_blocks(const AttnParams& p, int m0) {
   const int all = (p.nk + kAttnTile - 1) / kAttnTile;
@@ -250,40 +257,42 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int64_t key0 = static_cast<int64_t>(j) * kAttnTile;
       const uint32_t s_col = lane_base + static_cast<uint32_t>(s * 128);
-      // pass 1: the block's row maximum (scaled, masked)
-      float mx = -INFINITY;
+      // the whole row of S(j) in registers: scaled, masked, row maximum
+      float x[128];
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         tmem_ld32(s_col + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int64_t key = key0 + c * 32 + e;
-          if (key < p.nk && key <= last_key) mx = fmaxf(mx, __uint_as_float(v[e]) * p.scale_log2);
-        }
+        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_empty[s]);  // S buffer s may be overwritten by S(j + 2)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 128; ++e) {
+        const int64_t key = key0 + e;
+        x[e] = (key < p.nk && key <= last_key) ? x[e] * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[e]);
       }
       const float m_new = fmaxf(m_run, mx);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float corr = exp2f(m_run - m_use);  // 0 for the first block
+      const float corr = attn_exp2(m_run - m_use);  // 0 for the first block
       // the previous PV product must be done before O is rescaled and P overwritten
       if (j > 0 && !warp_wait(pv_done, static_cast<uint32_t>(j - 1) & 1u)) {
         ok = false;
         break;
       }
-      // pass 2: P = exp2(s * scale_log2 - m) as bf16 into the swizzled K-major tile
+      // P = exp2(x - m) as bf16 into the swizzled K-major tile
       float sum = 0.f;
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(s_col + static_cast<uint32_t>(c * 32), v);
-        tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int64_t ka = key0 + c * 32 + 2 * e;
-          const float x0 = (ka < p.nk && ka <= last_key) ? exp2f(__uint_as_float(v[2 * e]) * p.scale_log2 - m_use) : 0.f;
-          const float x1 =
-              (ka + 1 < p.nk && ka + 1 <= last_key) ? exp2f(__uint_as_float(v[2 * e + 1]) * p.scale_log2 - m_use) : 0.f;
-          const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
+          const __nv_bfloat162 t2 =
+              __floats2bfloat162_rn(attn_exp2(x[c * 32 + 2 * e] - m_use), attn_exp2(x[c * 32 + 2 * e + 1] - m_use));
           sum += __low2float(t2) + __high2float(t2);  // the row sum of the rounded weights that multiply V
           pk[e] = *reinterpret_cast<const uint32_t*>(&t2);
         }
@@ -296,12 +305,10 @@ __global__ void __launch_bounds__(192, 1)
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&s_empty[s]);  // S buffer s may be overwritten by S(j + 2)
       l_run = l_run * corr + sum;
       m_run = m_new;
-      if (j > 0) {
-        // O *= corr for this row (every lane of the warp takes part)
+      // O *= corr, only in warps where some row's maximum grew (tcgen05.ld / st are warp-wide)
+      if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
         tc_fence_after();
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];

@@ -5,6 +5,7 @@
     python -m input_adaptive_reduced_colnorm_b200.profile_cases qk --rho 0.5 --heads 8
     python -m input_adaptive_reduced_colnorm_b200.profile_cases pv --rho 0.5 --heads 2 --seq 16384
     python -m input_adaptive_reduced_colnorm_b200.profile_cases decode_attn --rho 0.5 --seq 32768
+    python -m input_adaptive_reduced_colnorm_b200.profile_cases attention --rho 0.5 --heads 32
 
 Each case draws its inputs with the seeded generators in ``synthetic`` (the same
 recipes the tests and the benchmark use), then calls the library ``--iters``
@@ -29,7 +30,7 @@ def main(argv=None) -> int:
     from input_adaptive_reduced_colnorm_b200 import build
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill", "decode", "qk", "pv", "linear", "decode_attn"])
+    ap.add_argument("case", choices=["prefill", "decode", "qk", "pv", "linear", "decode_attn", "attention"])
     ap.add_argument("--rho", type=float, default=0.5)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--n", type=int, default=32, help="decode rows")
@@ -57,6 +58,12 @@ def main(argv=None) -> int:
         Q, K = synthetic.qk_inputs(hq=a.heads, hkv=hkv, n=a.seq or 4096)
         Q, K = Q.to(dev), K.to(dev)
         fn = lambda: rmm.qk(Q, K, a.rho, causal=True)
+    elif a.case == "attention":
+        hkv = max(1, a.heads // 4)
+        Q, K = synthetic.qk_inputs(hq=a.heads, hkv=hkv, n=a.seq or 4096)
+        V = synthetic.to_bf16(synthetic.rng(7).standard_normal(tuple(K.shape), dtype="float32"))
+        Q, K, V = Q.to(dev), K.to(dev), V.to(dev)
+        fn = lambda: rmm.attention(Q, K, V, a.rho, causal=True, scale=0.088)
     elif a.case == "decode_attn":
         Q, Kt, P, V = synthetic.decode_attention_inputs_device(dev, nk=a.seq or 32768)
         fn = lambda: (rmm.decode_qk(Q, Kt, a.rho, scale=0.088), rmm.decode_pv(P, V, a.rho))
