@@ -9,18 +9,17 @@
 // the score product contracts over KP instead of 128.  The value product is the
 // ordinary one (selecting P's columns would need all of P first).
 //
-// One CTA per (query head, 128-row query tile), 192 threads:
-//   warp 0      TMA: the Q tile once, then 128-key blocks of K (K-major, KP
+// One CTA per (query head, pair of 128-row query tiles), see attn_pp_kernel:
+//   warp 0      TMA: both Q tiles once, then 128-key blocks of K (K-major, KP
 //               dims) and V (MN-major, 128 dims) into two-stage rings.
-//   warp 1      tensor memory (512 columns: S double buffer 2 x 128, O 128);
-//               lane 0 issues S(j) = Q K(j)^T (M = 128, N = 128, K = KP) into
-//               S buffer j % 2, and O += P(j) V(j) (M = 128, N = 128, K = 128),
-//               S(j+1) ahead of PV(j) so the score MMA overlaps softmax(j).
-//   warps 2..5  online softmax, one query row per thread: read S(j) from tensor
-//               memory, scale and mask, running max m and sum l (exp2 with the
-//               scale folded in log2 units), rescale the row of O in tensor
-//               memory when m grows, write P(j) as bf16 into the 128-byte-
-//               swizzled K-major layout the PV MMA reads; at the end O / l.
+//   warp 1      tensor memory (512 columns: S_A, S_B, O_A, O_B); lane 0 issues
+//               S_t(j) = Q_t K(j)^T (M = N = 128, K = KP) and O_t += P_t(j) V(j)
+//               (A = P_t from tensor memory, K = 128), alternating the tiles.
+//   warps 2..9  two softmax warpgroups (tile A: warps 2-5, tile B: 6-9), one
+//               query row per thread: running max m and sum l in log2 units,
+//               weights half by ex2.approx, half by a fitted polynomial on the
+//               FMA pipe, P written back as bf16 pairs into tensor memory, rows of
+//               O rescaled there when their maximum grew; at the end O / l.
 // Every wait is bounded (about one second); on a timeout the CTA records an
 // error code, drains its copies, lets the MMA finish and returns.
 #pragma once
@@ -46,14 +45,26 @@ constexpr int kAttnTile = 128;
 constexpr uint32_t kAttnQBytes = 128 * 128 * 2;  // Q tile, up to 128 dims (two 64-dim atoms)
 constexpr uint32_t kAttnKBytes = 128 * 128 * 2;  // one K block, up to 128 dims
 constexpr uint32_t kAttnVBytes = 128 * 128 * 2;  // one V block: 2 key halves x 2 column atoms of 64 x 64
-constexpr uint32_t kAttnPBytes = 128 * 128 * 2;  // P tile, K-major over 128 keys (two atoms)
-constexpr int kAttnSmem = kAttnQBytes + 2 * kAttnKBytes + 2 * kAttnVBytes + kAttnPBytes + 1024 + 256;
 
 // 2^x with the hardware approximation (relative error ~2^-22; exp2(-inf) = 0).
 __device__ __forceinline__ float attn_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for the half of the weights that do not go to the
+// special-function unit: x = n + f with n = floor(x) and f in [0, 1), 2^f from a
+// cubic fitted (relative-error minimax on [0, 1]) to max relative error 7.7e-5,
+// far below the bf16 rounding of P; 2^n is added to the exponent field.
+// Arguments below -126 give 2^-126 (the weight then rounds to 0 or the smallest
+// bf16 normal, far below every weight that matters).
+__device__ __forceinline__ float attn_exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float n = floorf(x);
+  const float f = x - n;
+  const float p = fmaf(fmaf(fmaf(0.0780965686f, f, 0.2259650975f), f, 0.6958683133f), f, 0.9999235868f);
+  return __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
 }
 
 // Visible key blocks of the query tile starting at row m0.
@@ -67,37 +78,55 @@ __device__ __forceinline__ int attn_key_blocks(const AttnParams& p, int m0) {
   return nb < all ? nb : all;
 }
 
-__global__ void __launch_bounds__(192, 1)
-    attn_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  extern __shared__ uint8_t attn_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kAttnQBytes;
-  uint8_t* sV = sK + 2 * kAttnKBytes;
-  uint8_t* sP = sV + 2 * kAttnVBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kAttnPBytes);
-  uint64_t* q_full = bars;           // 1
-  uint64_t* k_full = bars + 1;       // 2
-  uint64_t* k_empty = bars + 3;      // 2
-  uint64_t* v_full = bars + 5;       // 2
-  uint64_t* v_empty = bars + 7;      // 2
-  uint64_t* s_full = bars + 9;       // 2
-  uint64_t* s_empty = bars + 11;     // 2
-  uint64_t* p_full = bars + 13;      // 1
-  uint64_t* pv_done = bars + 14;     // 1
-  uint64_t* drain = bars + 15;       // 1
+}  // namespace rmm
+
+namespace rmm {
+
+// ---------------------------------------------------------------- two query tiles per CTA
+// The same attention with two 128-row query tiles A and B of one head per CTA
+// and two softmax warpgroups, so one tile's softmax runs while the tensor cores
+// work on the other tile (320 threads: TMA warp, MMA warp, softmax warps 2-5 for
+// A and 6-9 for B).  Tensor memory: S_A, S_B, O_A, O_B (128 columns each).  P(j)
+// of a tile is written as packed bf16 pairs over the first 64 columns of its S
+// region and the value MMA reads it from tensor memory (A operand in tensor
+// memory), so shared memory holds only Q_A, Q_B and the K / V rings.  The MMAs of
+// one thread execute in issue order: S_X(j+1) is issued after PV_X(j), so it
+// cannot overwrite P_X(j) early, and the commit that signals S_X(j) also covers
+// PV_X(j-1), which makes O_X safe to rescale.
+constexpr int kAttnPPSmem = 2 * kAttnQBytes + 2 * kAttnKBytes + 2 * kAttnVBytes + 1024 + 256;
+
+__global__ void __launch_bounds__(320, 1)
+    attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  extern __shared__ uint8_t app_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(app_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                    // [2 tiles][kAttnQBytes]
+  uint8_t* sK = sQ + 2 * kAttnQBytes;    // [2 stages]
+  uint8_t* sV = sK + 2 * kAttnKBytes;    // [2 stages]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kAttnVBytes);
+  uint64_t* q_full = bars;        // 1
+  uint64_t* k_full = bars + 1;    // 2 (stages)
+  uint64_t* k_empty = bars + 3;   // 2
+  uint64_t* v_full = bars + 5;    // 2
+  uint64_t* v_empty = bars + 7;   // 2
+  uint64_t* s_full = bars + 9;    // 2 (tiles)
+  uint64_t* p_full = bars + 11;   // 2 (tiles)
+  uint64_t* pv_done = bars + 13;  // 2 (tiles): the last value product
+  uint64_t* drain = bars + 15;    // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // heaviest causal tiles first: the last query tiles of every head lead the grid
+  const int pairs = (p.m_tiles + 1) / 2;
   const int item = static_cast<int>(blockIdx.x % p.items);
-  const int mt = p.m_tiles - 1 - static_cast<int>(blockIdx.x / p.items);
-  const int m0 = mt * kAttnTile;
+  const int pt = pairs - 1 - static_cast<int>(blockIdx.x / p.items);  // heaviest causal pairs first
+  const int m0 = pt * 2 * kAttnTile;
   const int b = item / p.hq, h = item % p.hq;
   const int g = h / (p.hq / p.hkv);
-  const int nkb = attn_key_blocks(p, m0);
+  int nkb_t[2];
+  nkb_t[0] = attn_key_blocks(p, m0);
+  nkb_t[1] = attn_key_blocks(p, m0 + kAttnTile < p.nq ? m0 + kAttnTile : m0);
+  const int nkb = nkb_t[0] > nkb_t[1] ? nkb_t[0] : nkb_t[1];
   const int qrow0 = item * p.nq + m0;
   const int krow0 = p.k_per_item ? item * p.nk : (b * p.hkv + g) * p.nk;
   const int vrow0 = (b * p.hkv + g) * p.nk;
@@ -111,10 +140,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 128);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&pv_done[s], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -137,8 +165,10 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       uint32_t k_issued = 0, v_issued = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, k_bytes);
-      for (int a = 0; a < p.kp / 64; ++a) tma_load_2d(sQ + a * 16384, &tmQ, q_full, a * 64, qrow0);
+      mbar_arrive_expect_tx(q_full, 2 * k_bytes);
+      for (int t = 0; t < 2; ++t)
+        for (int a = 0; a < p.kp / 64; ++a)
+          tma_load_2d(sQ + t * kAttnQBytes + a * 16384, &tmQ, q_full, a * 64, qrow0 + t * kAttnTile);
       for (int j = 0; j < nkb && ok; ++j) {
         const int s = j & 1;
         const uint32_t use = static_cast<uint32_t>(j >> 1);
@@ -184,45 +214,55 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, abort_flag, kDevErrTimeoutMma);
       const uint32_t idesc_s = make_idesc_bf16(128, 128, 0, 0);  // Q and K both K-major
-      const uint32_t idesc_o = make_idesc_bf16(128, 128, 0, 1);  // P K-major, V MN-major
-      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
-      auto issue_s = [&](int j) -> bool {
+      const uint32_t idesc_o = make_idesc_bf16(128, 128, 0, 1);  // P (tensor memory, K-major), V MN-major
+      // S_t(j) = Q_t K(j)^T; the first user of K(j) waits for it, tile B (the last user) releases it
+      auto issue_s = [&](int t, int j) -> bool {
         const int s = j & 1;
         const uint32_t use = static_cast<uint32_t>(j >> 1);
-        if (!mbar_wait(&k_full[s], use & 1u, abort_flag, kDevErrTimeoutMma)) return false;
-        if (!mbar_wait(&s_empty[s], (use & 1u) ^ 1u, abort_flag, kDevErrTimeoutMma)) return false;
+        const bool first = (t == 0) || (j >= nkb_t[0]);
+        if (first && !mbar_wait(&k_full[s], use & 1u, abort_flag, kDevErrTimeoutMma)) return false;
         tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ + t * kAttnQBytes);
         const uint32_t k0 = smem_u32(sK + s * kAttnKBytes);
         for (int kk = 0; kk < p.kp / 16; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
-          umma_bf16(tmem_base + static_cast<uint32_t>(s * 128), make_sw128_desc(q0 + off, 16, 1024),
+          umma_bf16(tmem_base + static_cast<uint32_t>(t * 128), make_sw128_desc(q0 + off, 16, 1024),
                     make_sw128_desc(k0 + off, 16, 1024), idesc_s, kk != 0 ? 1u : 0u);
         }
-        umma_commit(&k_empty[s]);
-        umma_commit(&s_full[s]);
+        if (t == 1) umma_commit(&k_empty[s]);
+        umma_commit(&s_full[t]);
         return true;
       };
-      auto issue_pv = [&](int j) -> bool {
+      // O_t += P_t(j) V(j), P_t(j) in the first 64 columns of S_t
+      auto issue_pv = [&](int t, int j) -> bool {
         const int s = j & 1;
         const uint32_t use = static_cast<uint32_t>(j >> 1);
-        if (!mbar_wait(p_full, static_cast<uint32_t>(j) & 1u, abort_flag, kDevErrTimeoutMma)) return false;
-        if (!mbar_wait(&v_full[s], use & 1u, abort_flag, kDevErrTimeoutMma)) return false;
+        if (!mbar_wait(&p_full[t], static_cast<uint32_t>(j) & 1u, abort_flag, kDevErrTimeoutMma)) return false;
+        const bool first = (t == 0) || (j >= nkb_t[0]);
+        if (first && !mbar_wait(&v_full[s], use & 1u, abort_flag, kDevErrTimeoutMma)) return false;
         tc_fence_after();
         const uint32_t v0 = smem_u32(sV + s * kAttnVBytes);
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 32);
           const uint32_t boff = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 2048);
-          umma_bf16(tmem_base + 256, make_sw128_desc(p0 + aoff, 16, 1024), make_sw128_desc(v0 + boff, 8192, 1024),
-                    idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem_base + 256u + static_cast<uint32_t>(t * 128),
+                       tmem_base + static_cast<uint32_t>(t * 128 + kk * 8), make_sw128_desc(v0 + boff, 8192, 1024),
+                       idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&v_empty[s]);
-        umma_commit(pv_done);
+        if (t == 1) umma_commit(&v_empty[s]);
+        if (j == nkb_t[t] - 1) umma_commit(&pv_done[t]);
         return true;
       };
-      if (ok && nkb > 0) ok = issue_s(0);
+      if (ok && nkb_t[0] > 0) ok = issue_s(0, 0);
+      if (ok && nkb_t[1] > 0) ok = issue_s(1, 0);
       for (int j = 0; j < nkb && ok; ++j) {
-        if (j + 1 < nkb) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+        if (j < nkb_t[0]) {
+          ok = issue_pv(0, j);
+          if (ok && j + 1 < nkb_t[0]) ok = issue_s(0, j + 1);
+        }
+        if (ok && j < nkb_t[1]) {
+          ok = issue_pv(1, j);
+          if (ok && j + 1 < nkb_t[1]) ok = issue_s(1, j + 1);
+        }
       }
       // every MMA issued by this thread is complete once `drain` flips
       umma_commit(drain);
@@ -233,105 +273,121 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
-    // tcgen05.ld / st are warp-collective: lane 0 waits and the warp follows
+    // ------------------------------------------------------------ softmax (tile X) + epilogue
     auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
       int got = 1;
       if (lane == 0) got = mbar_wait(bar, parity, abort_flag, kDevErrTimeoutEpilogue, 32) ? 1 : 0;
       return __shfl_sync(0xffffffffu, got, 0) != 0;
     };
+    const int X = (warp - 2) >> 2;  // 0: tile A (warps 2-5), 1: tile B (warps 6-9)
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // row of the tile (tensor-memory lane)
-    const int64_t qi = static_cast<int64_t>(m0) + r;
+    const int r = quarter * 32 + lane;
+    const int64_t qi = static_cast<int64_t>(m0) + X * kAttnTile + r;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t s_col = lane_base + static_cast<uint32_t>(X * 128);
+    const uint32_t o_col = lane_base + 256u + static_cast<uint32_t>(X * 128);
     const int64_t last_key = p.causal ? qi + p.causal_off : static_cast<int64_t>(p.nk) - 1;
+    const int my_nkb = nkb_t[X];
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkb && ok; ++j) {
-      const int s = j & 1;
-      const uint32_t use = static_cast<uint32_t>(j >> 1);
-      if (!warp_wait(&s_full[s], use & 1u)) {
+    for (int j = 0; j < my_nkb && ok; ++j) {
+      if (!warp_wait(&s_full[X], static_cast<uint32_t>(j) & 1u)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int64_t key0 = static_cast<int64_t>(j) * kAttnTile;
-      const uint32_t s_col = lane_base + static_cast<uint32_t>(s * 128);
-      // the whole row of S(j) in registers: scaled, masked, row maximum
-      float x[128];
-#pragma unroll
+      // every key of the block visible to this row: no masking work
+      const bool full = (key0 + kAttnTile - 1 <= last_key) && (key0 + kAttnTile <= p.nk);
+      // pass 1: the row maximum of the block (scaled, masked)
+      // tcgen05.ld is warp-collective (.sync.aligned): every lane executes the same
+      // loads, outside any branch on row-dependent values; only the arithmetic on
+      // the loaded values depends on whether this row sees the whole block
+      float mx = -INFINITY;
+      const bool fast = full && p.scale_log2 > 0.f;
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         tmem_ld32(s_col + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
+        if (fast) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(&s_empty[s]);  // S buffer s may be overwritten by S(j + 2)
-      float mx = -INFINITY;
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+        } else {
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        const int64_t key = key0 + e;
-        x[e] = (key < p.nk && key <= last_key) ? x[e] * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[e]);
+          for (int e = 0; e < 32; ++e) {
+            const int64_t key = key0 + c * 32 + e;
+            if (key < p.nk && key <= last_key) mx = fmaxf(mx, __uint_as_float(v[e]) * p.scale_log2);
+          }
+        }
       }
+      if (fast) mx *= p.scale_log2;
       const float m_new = fmaxf(m_run, mx);
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float corr = attn_exp2(m_run - m_use);  // 0 for the first block
-      // the previous PV product must be done before O is rescaled and P overwritten
-      if (j > 0 && !warp_wait(pv_done, static_cast<uint32_t>(j - 1) & 1u)) {
-        ok = false;
-        break;
-      }
-      // P = exp2(x - m) as bf16 into the swizzled K-major tile
+      // pass 2: P = exp2(s * scale_log2 - m) packed as bf16 pairs into the first 64
+      // columns of S; chunks 2h, 2h+1 (keys 64h .. 64h+63) become columns 32h .. 32h+31,
+      // which lie in S columns already read
       float sum = 0.f;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * hh + cc;
+          uint32_t v[32];
+          tmem_ld32(s_col + static_cast<uint32_t>(c * 32), v);
+          tmem_ld_wait();
+          // even keys on the FMA pipe, odd keys on the special-function unit
+          if (full) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const __nv_bfloat162 t2 =
-              __floats2bfloat162_rn(attn_exp2(x[c * 32 + 2 * e] - m_use), attn_exp2(x[c * 32 + 2 * e + 1] - m_use));
-          sum += __low2float(t2) + __high2float(t2);  // the row sum of the rounded weights that multiply V
-          pk[e] = *reinterpret_cast<const uint32_t*>(&t2);
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use));
+              const float x1 = attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use));
+              sum += x0 + x1;
+              const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
+              pk[cc * 16 + e] = *reinterpret_cast<const uint32_t*>(&t2);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int64_t ka = key0 + c * 32 + 2 * e;
+              const float x0 =
+                  (ka < p.nk && ka <= last_key) ? attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use)) : 0.f;
+              const float x1 =
+                  (ka + 1 < p.nk && ka + 1 <= last_key) ? attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use))
+                                                        : 0.f;
+              sum += x0 + x1;
+              const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
+              pk[cc * 16 + e] = *reinterpret_cast<const uint32_t*>(&t2);
+            }
+          }
         }
-        // keys c*32 .. c*32+31 = 16-byte chunks 4c .. 4c+3 of the row (atom = chunk / 8)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = c * 4 + q;
-          const int atom = chunk >> 3, cw = chunk & 7;
-          *reinterpret_cast<uint4*>(sP + atom * 16384 + r * 128 + ((cw ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        tmem_st32(s_col + static_cast<uint32_t>(hh * 32), pk);
       }
       l_run = l_run * corr + sum;
       m_run = m_new;
-      // O *= corr, only in warps where some row's maximum grew (tcgen05.ld / st are warp-wide)
+      // O *= corr where some row's maximum grew; PV(j-1) is complete (it was issued before S(j))
       if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
-        tc_fence_after();
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
-          tmem_ld32(lane_base + 256u + static_cast<uint32_t>(c * 32), v);
+          tmem_ld32(o_col + static_cast<uint32_t>(c * 32), v);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
-          tmem_st32(lane_base + 256u + static_cast<uint32_t>(c * 32), v);
+          tmem_st32(o_col + static_cast<uint32_t>(c * 32), v);
         }
-        tmem_st_wait();
       }
-      fence_proxy_async_smem();  // P (generic-proxy stores) is read by the MMA (async proxy)
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[X]);
     }
     // epilogue: O / l as bf16
-    if (ok && nkb > 0 && warp_wait(pv_done, static_cast<uint32_t>(nkb - 1) & 1u)) {
+    if (ok && my_nkb > 0 && warp_wait(&pv_done[X], 0u)) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       uint16_t* orow = p.O + (static_cast<int64_t>(item) * p.nq + qi) * 128;
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
-        tmem_ld32(lane_base + 256u + static_cast<uint32_t>(c * 32), v);
+        tmem_ld32(o_col + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();
         uint32_t o[16];
 #pragma unroll

@@ -230,6 +230,64 @@ __global__ void __launch_bounds__(256) pack_rows_cta_kernel(const PackParams p, 
   }
 }
 
+// Short rows (d <= 512): one warp per row, no shared-memory staging.  Lane l
+// produces the column pairs l, l + 32, ... of the packed row from two 2-byte
+// loads of the source row (its few 128-byte lines stay in L1 while the warp
+// gathers them) and the warp writes 128 contiguous bytes per pair group.  Four
+// rows are in flight per warp; the kept-index pairs of the current batch item
+// stay in registers (lanes x pair groups <= 32 x 4, so k_pad <= 256).
+__global__ void __launch_bounds__(256) pack_short_rows_kernel(const PackParams p) {
+  wait_prior_kernels();
+  constexpr int R = 4;   // rows in flight per warp
+  constexpr int PG = 4;  // pair groups per lane: k_pad <= 2 * 32 * PG
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t total = p.batch * p.rows;
+  const int pairs = static_cast<int>(p.k_pad / 2);
+  int64_t cur_b = -1;
+  int j0[PG], j1[PG];
+  for (int64_t r0 = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * R; r0 < total;
+       r0 += warps * R) {
+    uint32_t out[R][PG];
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+      const int64_t row = r0 + u;
+#pragma unroll
+      for (int q = 0; q < PG; ++q) out[u][q] = 0u;
+      if (row >= total) continue;
+      int64_t b, i;
+      const uint16_t* src = pack_src_row(p, row, b, i);
+      if (b != cur_b) {  // this batch item's kept columns (0xFFFF past k: padding)
+#pragma unroll
+        for (int q = 0; q < PG; ++q) {
+          const int t = 2 * (q * 32 + lane);
+          j0[q] = (t < p.k) ? __ldg(p.idx + b * p.k + t) : 0xFFFF;
+          j1[q] = (t + 1 < p.k) ? __ldg(p.idx + b * p.k + t + 1) : 0xFFFF;
+        }
+        cur_b = b;
+      }
+      const int64_t lim = pack_visible(p, i);
+#pragma unroll
+      for (int q = 0; q < PG; ++q) {
+        const uint32_t v0 = (j0[q] < lim) ? __ldg(src + j0[q]) : 0u;
+        const uint32_t v1 = (j1[q] < lim) ? __ldg(src + j1[q]) : 0u;
+        out[u][q] = v0 | (v1 << 16);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+      const int64_t row = r0 + u;
+      if (row >= total) continue;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(p.dst + row * p.k_pad);
+#pragma unroll
+      for (int q = 0; q < PG; ++q) {
+        const int t2 = q * 32 + lane;
+        if (t2 < pairs) dst[t2] = out[u][q];
+      }
+    }
+  }
+}
+
 // Same pack, with each source row staged by one 1-D bulk copy (TMA) instead
 // of 16-byte cp.async by every thread.  Thread 0 keeps NBUF - 1 rows in
 // flight; the CTA gathers one staged row per step with a single barrier.

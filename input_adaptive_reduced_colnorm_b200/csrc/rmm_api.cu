@@ -348,7 +348,11 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
   const int64_t rows = p.batch * p.rows;
   const int64_t d_round = round_up(p.d, 8);
   cudaError_t e;
-  if (p.d <= 1024) {
+  if (p.d <= 512 && p.k_pad <= 256 && p.k_pad % 2 == 0) {
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(rows, 8 * 4), 8LL * num_sms()));
+    e = launch_chained(pack_short_rows_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p);
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  } else if (p.d <= 1024) {
     const size_t smem = static_cast<size_t>(8 * d_round * 2);
     const int64_t grid = std::min<int64_t>(ceil_div(rows, 8), 8LL * num_sms());
     e = launch_chained(pack_rows_warp_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), smem, s, p, d_round);
@@ -767,10 +771,10 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
   const int64_t krows = ap.k_per_item ? items * nk : batch * hkv * nk;
   if (rmm_status st = make_tmap(&tk, ksrc, ap.kp, krows, ap.kp * 2, 64, 128)) return st;
   if (rmm_status st = make_tmap(&tv, V, dh, batch * hkv * nk, dh * 2, 64, 64)) return st;
-  cudaError_t e = cudaFuncSetAttribute(attn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  cudaError_t e = cudaFuncSetAttribute(attn_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnPPSmem);
   if (e != cudaSuccess) return cuda_fail(e, "attention attribute");
-  e = launch_chained(attn_fused_kernel, dim3(static_cast<unsigned>(items * m_tiles)), dim3(192), kAttnSmem, s, tq, tk, tv,
-                     ap);
+  e = launch_chained(attn_pp_kernel, dim3(static_cast<unsigned>(items * ceil_div(m_tiles, 2))), dim3(320), kAttnPPSmem, s,
+                     tq, tk, tv, ap);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return RMM_OK;
 }
