@@ -4,16 +4,16 @@
 // GQA; Attention vs MLP, Table 16: attention-internal reduction):
 //   S_h = scale * Q_h[:, I_h] K_g(h)[:, I_h]^T   (-inf above the causal diagonal)
 //   O_h = softmax_rows(S_h) V_g(h)
-// The index sets come from the column-norm and selection kernels; Q[:, I_h] and
-// K_g(h)[:, I_h] are packed per query head, zero-padded to KP = 64 or 128 dims, so
-// the score product contracts over KP instead of 128.  The value product is the
+// The index sets come from the column-norm and selection kernels; the score
+// product reads Q with the dropped dims of its head zeroed and K as it is, so it
+// is exactly sum_{t in I_h} Q_h[:, t] K_g(h)[:, t]^T.  The value product is the
 // ordinary one (selecting P's columns would need all of P first).
 //
 // One CTA per (query head, pair of 128-row query tiles), see attn_pp_kernel:
-//   warp 0      TMA: both Q tiles once, then 128-key blocks of K (K-major, KP
+//   warp 0      TMA: both Q tiles once, then 128-key blocks of K (K-major, 128
 //               dims) and V (MN-major, 128 dims) into two-stage rings.
 //   warp 1      tensor memory (512 columns: S_A, S_B, O_A, O_B); lane 0 issues
-//               S_t(j) = Q_t K(j)^T (M = N = 128, K = KP) and O_t += P_t(j) V(j)
+//               S_t(j) = Q_t K(j)^T (M = N = 128, K = 128) and O_t += P_t(j) V(j)
 //               (A = P_t from tensor memory, K = 128), alternating the tiles.
 //   warps 2..9  two softmax warpgroups (tile A: warps 2-5, tile B: 6-9), one
 //               query row per thread: running max m and sum l in log2 units,
@@ -30,11 +30,10 @@ namespace rmm {
 
 struct AttnParams {
   int nq, nk;          // query / key rows of one head
-  int kp;              // packed score dims: 64 or 128
+  int kp;              // score dims staged per tile (the head dim, 128)
   int hq, hkv;         // heads (GQA: query head h reads key/value head h / (hq / hkv))
   int items;           // batch * hq
   int m_tiles;         // ceil(nq / 128)
-  int k_per_item;      // 1: K rows are packed per query head (item * nk); 0: K as given ((b * hkv + g) * nk)
   int causal;
   int64_t causal_off;  // key j is visible to query i iff j <= i + causal_off
   float scale_log2;    // scale * log2(e)
@@ -128,7 +127,7 @@ __global__ void __launch_bounds__(320, 1)
   nkb_t[1] = attn_key_blocks(p, m0 + kAttnTile < p.nq ? m0 + kAttnTile : m0);
   const int nkb = nkb_t[0] > nkb_t[1] ? nkb_t[0] : nkb_t[1];
   const int qrow0 = item * p.nq + m0;
-  const int krow0 = p.k_per_item ? item * p.nk : (b * p.hkv + g) * p.nk;
+  const int krow0 = (b * p.hkv + g) * p.nk;
   const int vrow0 = (b * p.hkv + g) * p.nk;
   const uint32_t k_bytes = static_cast<uint32_t>(p.kp) * kAttnTile * 2;
 

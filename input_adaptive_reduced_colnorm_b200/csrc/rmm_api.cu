@@ -637,21 +637,18 @@ int64_t rmm_k(double rho, int64_t d) {
 }  // extern "C"
 
 namespace {
-// Workspace of rmm_attention (rho < 1): scores, index sets and either the packed
-// Q[:, I] / K[:, I] per query head (k <= 64: the score product contracts over 64
-// dims) or keep bytes and Q with the dropped dims zeroed (k > 64: 128 dims, K as is).
+// Workspace of rmm_attention (rho < 1): scores, index sets, keep bytes and Q with
+// the dropped dims zeroed.  (Packing Q[:, I] and K[:, I] per query head to 64 dims
+// halves the score MMA, but while the fused kernel is bound by its softmax the
+// two packs cost more than they save, so K is read as is.)
 size_t attention_bytes(int64_t items, int64_t nq, int64_t nk, int64_t dh, int64_t k) {
+  (void)nk;
   if (k == dh) return 0;
   Carver c(nullptr);
   c.take<double>(items * dh);
   c.take<int32_t>(items * k);
-  if (k <= 64) {
-    c.take<uint16_t>(items * nq * 64);
-    c.take<uint16_t>(items * nk * 64);
-  } else {
-    c.take<uint8_t>(items * dh);
-    c.take<uint16_t>(items * nq * dh);
-  }
+  c.take<uint8_t>(items * dh);
+  c.take<uint16_t>(items * nq * dh);
   return c.bytes();
 }
 }  // namespace
@@ -705,62 +702,28 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
   const uint16_t* qsrc = Q;
   const uint16_t* ksrc = K;
   ap.kp = 128;
-  ap.k_per_item = 0;
   if (k < dh) {
     Carver c(ws);
     double* colsq = c.take<double>(items * dh);
     int32_t* idx_ws = c.take<int32_t>(items * k);
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if (rmm_status st = launch_colsq(Q, items, nq * dh, nq, dh, dh, false, 0, colsq, s)) return st;
-    if (k <= 64) {
-      uint16_t* qp = c.take<uint16_t>(items * nq * 64);
-      uint16_t* kpk = c.take<uint16_t>(items * nk * 64);
-      if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s)) return st;
-      PackParams pq{};
-      pq.src = Q;
-      pq.src_ld = dh;
-      pq.rows = nq;
-      pq.d = dh;
-      pq.g_outer = 1;
-      pq.g_inner = 1;
-      pq.s_outer = nq * dh;
-      pq.idx = idx;
-      pq.k = k;
-      pq.k_pad = 64;
-      pq.dst = qp;
-      pq.batch = items;
-      if (rmm_status st = launch_pack(pq, s)) return st;
-      PackParams pk = pq;  // K of the query head's key/value head, gathered with the query head's I
-      pk.src = K;
-      pk.rows = nk;
-      pk.g_outer = hq;
-      pk.g_inner = hq / hkv;
-      pk.s_outer = hkv * nk * dh;
-      pk.s_inner = nk * dh;
-      pk.dst = kpk;
-      if (rmm_status st = launch_pack(pk, s)) return st;
-      qsrc = qp;
-      ksrc = kpk;
-      ap.kp = 64;
-      ap.k_per_item = 1;
-    } else {
-      uint8_t* keep = c.take<uint8_t>(items * dh);
-      uint16_t* qm = c.take<uint16_t>(items * nq * dh);
-      if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s, keep)) return st;
-      MaskParams mp{};
-      mp.src = Q;
-      mp.dst = qm;
-      mp.rows = nq;
-      mp.cols = dh;
-      mp.keep = keep;
-      mp.by_rows = 0;
-      mp.batch = items;
-      mp.g_outer = 1;
-      mp.g_inner = 1;
-      mp.s_outer = nq * dh;
-      if (rmm_status st = launch_mask(mp, s)) return st;
-      qsrc = qm;
-    }
+    uint8_t* keep = c.take<uint8_t>(items * dh);
+    uint16_t* qm = c.take<uint16_t>(items * nq * dh);
+    if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s, keep)) return st;
+    MaskParams mp{};
+    mp.src = Q;
+    mp.dst = qm;
+    mp.rows = nq;
+    mp.cols = dh;
+    mp.keep = keep;
+    mp.by_rows = 0;
+    mp.batch = items;
+    mp.g_outer = 1;
+    mp.g_inner = 1;
+    mp.s_outer = nq * dh;
+    if (rmm_status st = launch_mask(mp, s)) return st;
+    qsrc = qm;
   } else if (idx_out != nullptr) {
     const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(items * dh, 256), 1024))),
                                          dim3(256), 0, s, idx_out, items, dh);
@@ -768,8 +731,7 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
   }
   CUtensorMap tq, tk, tv;
   if (rmm_status st = make_tmap(&tq, qsrc, ap.kp, items * nq, ap.kp * 2, 64, 128)) return st;
-  const int64_t krows = ap.k_per_item ? items * nk : batch * hkv * nk;
-  if (rmm_status st = make_tmap(&tk, ksrc, ap.kp, krows, ap.kp * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tk, ksrc, ap.kp, batch * hkv * nk, ap.kp * 2, 64, 128)) return st;
   if (rmm_status st = make_tmap(&tv, V, dh, batch * hkv * nk, dh * 2, 64, 64)) return st;
   cudaError_t e = cudaFuncSetAttribute(attn_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnPPSmem);
   if (e != cudaSuccess) return cuda_fail(e, "attention attribute");

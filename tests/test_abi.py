@@ -199,5 +199,5 @@ def test_attention_argument_errors(L):
     assert att(nq=300, nk=256) == UNSUPPORTED   # causal with nq > nk
     assert att() == WORKSPACE
     assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 256, 128, 1.0) == 0
-    # k <= 64 packs Q and K per query head to 64 dims
-    assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 512, 128, 0.5) >= 4 * (256 + 512) * 64 * 2
+    # Q with the dropped dims zeroed, per query head
+    assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 512, 128, 0.5) >= 4 * 256 * 128 * 2

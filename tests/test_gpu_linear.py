@@ -200,6 +200,19 @@ def test_gemm_packed_narrow_last_wave(n, k, m):
     assert np.abs(tail - ref[-128:, -512:]).max() <= 3e-2 * np.abs(ref).max()
 
 
+@pytest.mark.parametrize("d,k,ld", [(296, 150, 152), (504, 250, 256), (16, 5, 8)])
+def test_gather_columns_short_rows(d, k, ld):
+    """Rows of at most 512 columns take the warp-per-row gather without staging;
+    k_pad up to 256, kept columns in any order."""
+    g = synthetic.rng(44)
+    A = synthetic.to_bf16(g.standard_normal((1001, d), dtype=np.float32)).cuda()
+    idx = torch.as_tensor(g.permutation(d)[:k], dtype=torch.int32).cuda()
+    ap = rmm.gather_columns(A, idx, ld_pack=ld)
+    torch.cuda.synchronize()
+    assert torch.equal(ap[:, :k], A[:, idx.long()])
+    assert not ap[:, k:].any()
+
+
 _DECODE_W = {}
 
 
