@@ -325,15 +325,31 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int
   const int64_t U = p.units, G = grid;
   const int64_t u_lo = static_cast<int64_t>(sup) * p.kb_total;
   const int64_t u_hi = u_lo + p.kb_total - 1;
-  const int c_lo = static_cast<int>(((u_lo + 1) * G - 1) / U);  // owner of unit u_lo
-  const int c_hi = static_cast<int>(((u_hi + 1) * G - 1) / U);  // owner of unit u_hi
   float acc = 0.f;
-  int64_t start_c = (static_cast<int64_t>(c_lo) * U) / G;
-  for (int c = c_lo; c <= c_hi; ++c) {
-    const int64_t start_next = (static_cast<int64_t>(c + 1) * U) / G;
-    if (start_next > start_c)  // CTA c had at least one unit
-      acc += p.partial[((static_cast<int64_t>(sup) + c) * kGemvTiles + tl) * p.n * 128 + r * 128 + i];
-    start_c = start_next;
+  const float* src = p.partial + static_cast<int64_t>(tl) * p.n * 128 + r * 128 + i;
+  const int64_t slot = static_cast<int64_t>(kGemvTiles) * p.n * 128;  // floats per partial super tile
+  if ((U + 1) * G < (1LL << 32)) {
+    // the unit split in 32-bit unsigned arithmetic (the usual case; much cheaper
+    // than 64-bit division)
+    const uint32_t u32 = static_cast<uint32_t>(U), g32 = static_cast<uint32_t>(G);
+    const uint32_t c_lo = (static_cast<uint32_t>(u_lo + 1) * g32 - 1u) / u32;  // owner of unit u_lo
+    const uint32_t c_hi = (static_cast<uint32_t>(u_hi + 1) * g32 - 1u) / u32;  // owner of unit u_hi
+    uint32_t start_c = (c_lo * u32) / g32;
+    for (uint32_t c = c_lo; c <= c_hi; ++c) {
+      const uint32_t start_next = ((c + 1u) * u32) / g32;
+      if (start_next > start_c)  // CTA c had at least one unit
+        acc += src[(static_cast<int64_t>(sup) + c) * slot];
+      start_c = start_next;
+    }
+  } else {
+    const int c_lo = static_cast<int>(((u_lo + 1) * G - 1) / U);
+    const int c_hi = static_cast<int>(((u_hi + 1) * G - 1) / U);
+    int64_t start_c = (static_cast<int64_t>(c_lo) * U) / G;
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const int64_t start_next = (static_cast<int64_t>(c + 1) * U) / G;
+      if (start_next > start_c) acc += src[(static_cast<int64_t>(sup) + c) * slot];
+      start_c = start_next;
+    }
   }
   const __nv_bfloat16 h = __float2bfloat16_rn(acc);
   Y[static_cast<int64_t>(r) * ldy + col] = *reinterpret_cast<const uint16_t*>(&h);

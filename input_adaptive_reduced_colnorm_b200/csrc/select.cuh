@@ -170,7 +170,54 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectParams p) {
   // bit cursor: position (in the 64-bit key) just above the next digit
   int cursor = 32 + ((msk_hi == 0xffffffffu) ? 0 : (32 - __popc(msk_hi)));
 
+  bool lo_checked = false;
   while (!take_bucket && cursor > 0) {
+    if (cursor <= 32 && !lo_checked) {
+      // the high words are resolved: one AND / OR of the low words still in the
+      // bucket skips their shared leading bits, and identical keys (exact ties,
+      // e.g. the squares of a single bf16 row) end the passes at once
+      lo_checked = true;
+      uint32_t la = 0xffffffffu, lr = 0u;
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        if (((valid >> e) & 1u) && (my_keys[e] & msk_hi) == pre_hi) {
+          const uint32_t lo = static_cast<uint32_t>(__double_as_longlong(q[j0 + e]));
+          if ((lo & msk_lo) == pre_lo) {
+            la &= lo;
+            lr |= lo;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        la &= __shfl_xor_sync(0xffffffffu, la, o);
+        lr |= __shfl_xor_sync(0xffffffffu, lr, o);
+      }
+      __syncthreads();  // every thread has read s_and / s_or of the earlier reduction
+      if (lane == 0) {
+        s_and[warp] = la;
+        s_or[warp] = lr;
+      }
+      __syncthreads();
+      la = 0xffffffffu;
+      lr = 0u;
+      for (int w = 0; w < NW; ++w) {
+        la &= s_and[w];
+        lr |= s_or[w];
+      }
+      const uint32_t open = (cursor == 32) ? 0xffffffffu : ((1u << cursor) - 1u);  // unresolved low bits
+      const uint32_t dl = (la ^ lr) & open;
+      if (dl == 0u) {  // every key left has the same value: the lower indices win
+        pre_lo = (pre_lo & ~open) | (la & open);
+        msk_lo = 0xffffffffu;
+        break;
+      }
+      const int top = 31 - __clz(dl);
+      const uint32_t shared = open & ((top == 31) ? 0u : (0xffffffffu << (top + 1)));
+      pre_lo |= la & shared;
+      msk_lo |= shared;
+      cursor = top + 1;
+    }
     const int width = cursor >= kSelBits ? kSelBits : cursor;
     const int shift = cursor - width;  // bit position of the digit in the 64-bit key
     const uint32_t dmask = (1u << width) - 1u;

@@ -91,3 +91,12 @@ def test_mlp_llama8b_sampled(rho_gu, rho_down):
     rows = np.concatenate([np.arange(0, 4096, 331), [4095]])
     mlp_parity(X, Wg, Wu, Wd, rho_gu, rho_down, rows=rows)
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("n", [1, 8, 32])
+def test_mlp_decode_rows(n):
+    """Decode-sized blocks (n <= 32): short-matrix column scores, the down
+    projection on the decode product; H and Y checked as for any n."""
+    X, Wg, Wu, Wd = synthetic.mlp_block(n=n, d=1040, f=776, m=264)
+    mlp_parity(X, Wg, Wu, Wd, 0.5, 0.5)
+    mlp_parity(X, Wg, Wu, Wd, 0.7, 1.0)
