@@ -230,8 +230,9 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
  *   scale  device fp32 [m].
  *   Y      device bf16 [n][ldy].
  *   idx_out device int32 [rmm_k(rho, d)] or NULL.
- * Requires m % 8 == 0, d <= 32768.  Workspace: scores, index set, A[:, I] and
- * fp32 partial sums of the row chunks (added in a fixed order). */
+ * Requires m % 8 == 0, d <= 32768.  Workspace: scores, index set and fp32
+ * partial sums of the row chunks (added in a fixed order); the kernel reads
+ * A[:, I] through the index set, so no packed copy of A is made. */
 size_t rmm_linear_int8_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho);
 rmm_status rmm_linear_int8(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int8_t* Wq, int64_t m,
                            int64_t ldw, const float* scale, rmm_bf16* Y, int64_t ldy, double rho, int32_t* idx_out,

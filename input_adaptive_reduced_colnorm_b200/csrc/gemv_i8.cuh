@@ -26,7 +26,7 @@ constexpr int kI8MaxRows = 8;     // activation rows
 struct GemvI8Params {
   const int8_t* W;     // [d][ldw] int8
   int64_t ldw;
-  const uint16_t* x;   // bf16 [n][ldx]; column t holds kept row t (packed x_I, or x itself for I = [0, k))
+  const uint16_t* x;   // bf16 [n][ldx], all d columns: the kept ones are read through idx
   int64_t ldx;
   const int32_t* idx;  // [k] kept rows, or null for rows [0, k)
   int k, m, n;
@@ -81,10 +81,11 @@ __global__ void __launch_bounds__(256, (NR == 1) ? 4 : ((NR == 2) ? 3 : 2)) gemv
   const int cnt16 = (cnt + 15) & ~15;  // <= chunk <= kI8MaxChunk: the tail reads zeros
   for (int i = threadIdx.x; i < cnt16; i += blockDim.x) {
     const bool in = i < cnt;
-    rows[i] = in ? (p.idx ? __ldg(p.idx + t0 + i) : t0 + i) : 0;
+    const int row = in ? (p.idx ? __ldg(p.idx + t0 + i) : t0 + i) : 0;
+    rows[i] = row;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-      const float xv = (in && r < p.n) ? bf16lo(static_cast<uint32_t>(__ldg(p.x + r * p.ldx + t0 + i))) : 0.f;
+      const float xv = (in && r < p.n) ? bf16lo(static_cast<uint32_t>(__ldg(p.x + r * p.ldx + row))) : 0.f;
       xs[r][i] = f2_pack(xv, xv);
     }
   }

@@ -777,7 +777,6 @@ size_t rmm_linear_int8_workspace_bytes(int64_t n, int64_t d, int64_t m, double r
   if (k < d) {
     c.take<double>(d);
     c.take<int32_t>(k);
-    c.take<uint16_t>(n * round_up(k, 8));
   }
   c.take<float>(static_cast<int64_t>(chunks) * n * m);
   return c.bytes();
@@ -820,14 +819,9 @@ rmm_status rmm_linear_int8(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda,
   if (k < d) {
     double* colsq = c.take<double>(d);
     int32_t* idx_ws = c.take<int32_t>(k);
-    const int64_t k_pad = round_up(k, 8);
-    uint16_t* xpack = c.take<uint16_t>(n * k_pad);
     int32_t* idx = idx_out ? idx_out : idx_ws;
     if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
     if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
-    if (rmm_status st = pack_columns(A, n, d, lda, idx, k, xpack, k_pad, s)) return st;
-    p.x = xpack;
-    p.ldx = k_pad;
     p.idx = idx;
   } else if (idx_out != nullptr) {
     const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024))),
