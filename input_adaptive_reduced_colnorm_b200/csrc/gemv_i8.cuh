@@ -13,7 +13,9 @@
 // permute, then one subtraction.  Conversion and products run on packed fp32
 // pairs (two columns per instruction); accumulation is fp32.  CTAs split
 // the kept rows into chunks and write fp32 partial sums, which
-// gemv_i8_fixup_kernel adds in chunk order and scales (deterministic).
+// gemv_i8_fixup_kernel adds in chunk order and scales (deterministic).  The
+// kept activations x[:, I] are read through the index set while a CTA stages
+// its row chunk, so the call needs no separate pack of x.
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
