@@ -481,3 +481,62 @@ def test_attention_rows_are_convex_combinations_and_first_row_is_v0():
             assert np.all(O[0, h, i] >= lo - 1e-12) and np.all(O[0, h, i] <= hi + 1e-12)
     # the same index sets as the score product alone
     assert np.array_equal(oracle.rmm_attention(Q, K, V, 0.5)["I"], oracle.rmm_qk(Q, K, 0.5)["I"])
+
+
+# ---------------------------------------------------------------- the helpers, each on its own
+def test_column_norms_pythagorean_columns_and_causal_mask():
+    """Columns (3, 4), (5, 12) and (8, 15) have norms 5, 13 and 17; under a causal
+    mask with nq = nk = 2, entry (0, 1) is not visible, so column 1's norm is 12."""
+    A = np.array([[3.0, 5.0, 8.0], [4.0, 12.0, 15.0]])
+    assert oracle.column_norms(A).tolist() == [5.0, 13.0, 17.0]
+    Ac = np.array([[3.0, 99.0], [4.0, 12.0]])  # 99 sits above the diagonal
+    assert oracle.column_norms(Ac, causal=True).tolist() == [5.0, 12.0]
+
+
+def test_topk_ascending_order_ties_and_bounds():
+    s = np.array([2.0, 7.0, 7.0, 1.0, 7.0, 0.0])
+    assert oracle.topk_ascending(s, 1).tolist() == [1]        # three-way tie: the lowest index
+    assert oracle.topk_ascending(s, 2).tolist() == [1, 2]
+    assert oracle.topk_ascending(s, 4).tolist() == [0, 1, 2, 4]
+    assert oracle.topk_ascending(s, 6).tolist() == [0, 1, 2, 3, 4, 5]
+    with pytest.raises(ValueError):
+        oracle.topk_ascending(s, 0)
+    with pytest.raises(ValueError):
+        oracle.topk_ascending(s, 7)
+
+
+def test_retained_energy_closed_form():
+    q = np.array([1.0, 4.0, 9.0, 16.0])  # squared norms of columns with norms 1..4
+    assert oracle.retained_energy(q, np.array([2, 3])) == 25.0 / 30.0
+    assert oracle.retained_energy(q, np.arange(4)) == 1.0
+    assert oracle.retained_energy(np.zeros(3), np.array([0])) == 1.0  # nothing to lose
+
+
+def test_linear_rows_hand_example():
+    """A = [[1, 2], [3, 4]], B = identity, I = {1}: row 1 of A[:, I] B[I, :] is
+    [0, 4] (column 0 of B is not used)."""
+    A = np.array([[1.0, 2.0], [3.0, 4.0]])
+    out = oracle.rmm_linear_rows(A, np.eye(2), np.array([1]), [1])
+    assert out.tolist() == [[0.0, 4.0]]
+
+
+def test_qk_and_pv_rows_match_the_full_products():
+    """The row-sampled QK and PV restatements give exactly the rows of the full
+    per-head products, with the same index sets (the full products are pinned by the
+    hand fixtures and brute force above)."""
+    g = np.random.default_rng(21)
+    Q, K = g.standard_normal((1, 4, 7, 8)), g.standard_normal((1, 2, 7, 8))
+    full = oracle.rmm_qk(Q, K, 0.5, causal=True, scale=0.3)
+    rows = [0, 3, 6]
+    for h in range(4):
+        S, I = oracle.rmm_qk_rows(Q[0, h], K[0, oracle.kv_head(h, 4, 2)], 0.5, rows, causal=True, scale=0.3)
+        assert np.array_equal(I, full["I"][0, h])
+        assert np.array_equal(S, full["S"][0, h][rows])
+    P = np.abs(g.standard_normal((1, 2, 6, 6)))
+    V = g.standard_normal((1, 1, 6, 4))
+    fullp = oracle.rmm_pv(P, V, 0.5, causal=True)
+    for h in range(2):
+        O, I, q = oracle.rmm_pv_rows(P[0, h], V[0, 0], 0.5, [1, 5], causal=True)
+        assert np.array_equal(I, fullp["I"][0, h])
+        assert np.array_equal(O, fullp["O"][0, h][[1, 5]])
+        assert np.array_equal(q, oracle.column_sq_norms(P[0, h], causal=True))
