@@ -33,6 +33,7 @@ PROJ = ["q_proj", "gate_proj", "up_proj", "down_proj"]
 N_TOKENS = 4096
 RHO_MAIN = 0.5
 RHO_SWEEP = (0.9, 0.7)
+WORKLOAD = "llama3.1-8b prefill projections q/gate/up/down, n=4096 tokens, rho=0.5"
 GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm_pair.cuh", "input_adaptive_reduced_colnorm_b200/csrc/gemm.cuh",
                 "input_adaptive_reduced_colnorm_b200/csrc/ptx.cuh"]
 TRAFFIC_PROFILE = "profiles/gemm_packed_llama8b_gate.md"
@@ -239,8 +240,8 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": "llama3.1-8b prefill projections (oracle sample)", "n": N_TOKENS,
-                       "rho": RHO_MAIN, "projections": PROJ},
+            "config": {"workload": WORKLOAD, "n": N_TOKENS, "rho": RHO_MAIN, "projections": PROJ,
+                       "sampled": "16 rows per projection for the product (see cpu_baseline.sample)"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -669,7 +670,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "llama3.1-8b prefill projections q/gate/up/down, n=4096 tokens, rho=0.5",
+        "config": {"workload": WORKLOAD,
                    "n": N_TOKENS, "rho": RHO_MAIN, "projections": PROJ, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (about 0.7 GB touched per step)"},
         "gbs": world * nbytes / (ms_step * 1e-3) / 1e9,
