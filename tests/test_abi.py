@@ -6,7 +6,6 @@ status before touching the device (on a machine without a GPU any device call
 would surface as RMM_ERR_CUDA instead, so the exact codes below also show that
 nothing was enqueued).
 """
-import ctypes
 import json
 import os
 import re
