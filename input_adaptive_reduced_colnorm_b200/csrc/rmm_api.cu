@@ -748,12 +748,15 @@ namespace {
 // Row chunks of the int8 GEMV: about four CTAs per SM over all column blocks,
 // at most kI8MaxChunk rows each, and few enough chunks that the fp32 partial
 // sums (chunks x n x m x 4 bytes) stay near 12 % of the kept int8 rows.
+// Row chunks of the int8 GEMV: as many as one wave of co-resident CTAs holds
+// (the kernel's launch bounds give 4, 3 or 2 CTAs per SM for 1, 2 or more rows),
+// so that every CTA starts at once and no partial second wave follows.  A chunk
+// is a multiple of 16 kept rows and at most kI8MaxChunk.
 void i8_plan(int64_t n, int64_t k, int64_t m, int* chunk, int* chunks) {
   const int64_t col_blocks = ceil_div(m, 2048);
-  int64_t c = ceil_div(4LL * num_sms(), col_blocks);
-  const int64_t by_bytes = std::max<int64_t>(1, (3 * k) / (100 * n));
-  c = std::max<int64_t>(1, std::min(c, by_bytes));
-  int64_t len = round_up(ceil_div(k, c), 16);
+  const int64_t per_sm = (n == 1) ? 4 : ((n == 2) ? 3 : 2);
+  const int64_t max_chunks = std::max<int64_t>(1, (per_sm * num_sms()) / col_blocks);
+  int64_t len = round_up(ceil_div(k, max_chunks), 16);
   if (len > kI8MaxChunk) len = kI8MaxChunk;
   *chunk = static_cast<int>(len);
   *chunks = static_cast<int>(ceil_div(k, len));
