@@ -200,3 +200,27 @@ def test_attention_argument_errors(L):
     assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 256, 128, 1.0) == 0
     # Q with the dropped dims zeroed, per query head
     assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 512, 128, 0.5) >= 4 * 256 * 128 * 2
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 8])
+@pytest.mark.parametrize("rho", [1.0, 0.9, 0.5, 0.01])
+def test_int8_plan_fills_at_most_one_wave(L, n, rho):
+    """The int8 GEMV's row chunks, read back from the workspace size (scores, index
+    set and chunks x n x m fp32 partial sums): the grid of 2048-column blocks x
+    chunks fits in one wave of co-resident CTAs (4, 3 or 2 per SM by the row count;
+    148 SMs when no device is visible) while every chunk holds at most 512 kept rows
+    and a multiple of 16."""
+    d, m = 8192, 28672
+    k = L.rmm_k(rho, d)
+    ws = L.rmm_linear_int8_workspace_bytes(n, d, m, rho)
+    head = 0 if k == d else (d * 8 + 256 - 1) // 256 * 256 + (k * 4 + 256 - 1) // 256 * 256
+    partial = ws - head
+    assert partial > 0 and partial % (n * m * 4) == 0, (ws, head)
+    chunks = partial // (n * m * 4)
+    slots = {1: 4, 2: 3}.get(n, 2) * 148
+    assert chunks * ((m + 2047) // 2048) <= slots
+    chunk = -(-k // chunks)
+    assert chunk <= 512
+    # the chunk length the plan picks is a multiple of 16 covering k in `chunks` pieces
+    lens = [ln for ln in range(16, 513, 16) if -(-k // ln) == chunks]
+    assert lens, (k, chunks)
