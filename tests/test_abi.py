@@ -127,11 +127,31 @@ def test_workspace_queries(L):
 
 
 def test_binding_refuses_cpu_tensors():
+    """Every public call refuses host tensors before anything reaches the library:
+    there is no CPU path."""
     import torch
-    A = torch.zeros((4, 16), dtype=torch.bfloat16)
-    B = torch.zeros((16, 8), dtype=torch.bfloat16)
-    with pytest.raises(TypeError):
-        rmm.linear(A, B, 0.5)
+    bf = torch.bfloat16
+    A = torch.zeros((4, 16), dtype=bf)
+    B = torch.zeros((16, 8), dtype=bf)
+    idx = torch.zeros(8, dtype=torch.int32)
+    Q4 = torch.zeros((1, 2, 8, 64), dtype=bf)
+    calls = [
+        lambda: rmm.linear(A, B, 0.5),
+        lambda: rmm.select(A, 0.5),
+        lambda: rmm.gather_columns(A, idx),
+        lambda: rmm.gather_rows(B, idx),
+        lambda: rmm.gemm_packed(A, 16, B, 8),
+        lambda: rmm.qk(Q4, Q4, 0.5),
+        lambda: rmm.pv(torch.zeros((1, 2, 8, 8), dtype=bf), Q4, 0.5),
+        lambda: rmm.attention(Q4, Q4, Q4, 0.5),
+        lambda: rmm.linear_int8(A, torch.zeros((16, 8), dtype=torch.int8), torch.ones(8), 0.5),
+        lambda: rmm.mlp(A, B, B, torch.zeros((8, 16), dtype=bf), 0.5, 0.5),
+        lambda: rmm.decode_qk(torch.zeros((1, 2, 64), dtype=bf), torch.zeros((1, 1, 64, 8), dtype=bf), 0.5),
+        lambda: rmm.decode_pv(torch.zeros((1, 2, 8), dtype=bf), torch.zeros((1, 1, 8, 64), dtype=bf), 0.5),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(TypeError, match="CUDA tensor"):
+            call()
 
 
 def test_decode_attention_argument_errors(L):
