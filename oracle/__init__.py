@@ -45,7 +45,8 @@ __all__ = [
     "retained_energy", "select", "reduced_product", "error_bound", "rmm_linear",
     "rmm_linear_rows", "kv_head", "rmm_qk", "rmm_qk_rows", "rmm_pv", "rmm_pv_rows",
     "near_tie_band", "rmm_decode_qk", "rmm_decode_pv", "silu", "rmm_mlp_gate_up", "rmm_mlp",
-    "rmm_linear_int8", "rmm_attention",
+    "rmm_linear_int8", "rmm_attention", "qk_scores_rows", "pv_output_rows", "attention_rows",
+    "int8_product_rows", "mlp_gate_up_rows", "rmm_attention_rows",
 ]
 
 
@@ -186,18 +187,43 @@ def kv_head(h: int, hq: int, hkv: int) -> int:
     return h // (hq // hkv)
 
 
-def _qk_head(Qh, Kg, rho, causal, scale, rows=None):
+def _check_index_set(I, d, what):
+    I = np.asarray(I, dtype=np.int64).reshape(-1)
+    if I.size < 1 or I.size > d or np.any(I < 0) or np.any(I >= d) or np.any(np.diff(I) <= 0):
+        raise ValueError(f"{what}: the index set must be strictly ascending within [0, {d})")
+    return I
+
+
+def qk_scores_rows(Qh: np.ndarray, Kg: np.ndarray, I, rows=None, causal: bool = True, scale: float = 1.0):
+    """Rows ``rows`` of one head's reduced scores on a GIVEN index set I:
+        S[i, j] = scale * sum_{t in I} Qh[i, t] * Kg[j, t],
+    -inf where key j is not visible to query i (bottom-right causal alignment).
+
+    [DD] "Component mapping": QK^T contracts over the kept head-feature dims only;
+    under GQA the key head gathers the query head's dims.  Qh [nq, dh], Kg [nk, dh].
+    The product on the index set the library chose is what a parity check compares
+    when two sets differ only inside the near-tie band."""
+    Qh = np.asarray(Qh, dtype=np.float64)
+    Kg = np.asarray(Kg, dtype=np.float64)
     nq, dh = Qh.shape
     nk = Kg.shape[0]
-    k = retention_count(rho, dh)
-    q = column_sq_norms(Qh)
-    I = topk_ascending(np.sqrt(q), k)
+    I = _check_index_set(I, dh, "qk_scores_rows")
     r = np.arange(nq) if rows is None else np.asarray(rows)
     S = scale * (Qh[r][:, I] @ Kg[:, I].T)
     if causal:
         vis = np.array([_visible_cols(i, nq, nk) for i in r])
         S[np.arange(nk)[None, :] >= vis[:, None]] = -np.inf
-    return S, I
+    return S
+
+
+def _qk_head(Qh, Kg, rho, causal, scale, rows=None, I=None):
+    nq, dh = Qh.shape
+    if I is None:
+        k = retention_count(rho, dh)
+        q = column_sq_norms(Qh)
+        I = topk_ascending(np.sqrt(q), k)
+    I = _check_index_set(I, dh, "qk")
+    return qk_scores_rows(Qh, Kg, I, rows, causal, scale), I
 
 
 def rmm_qk(Q: np.ndarray, K: np.ndarray, rho: float, causal: bool = True, scale: float = 1.0):
@@ -222,24 +248,41 @@ def rmm_qk(Q: np.ndarray, K: np.ndarray, rho: float, causal: bool = True, scale:
     return {"S": S, "I": I}
 
 
-def rmm_qk_rows(Qh: np.ndarray, Kg: np.ndarray, rho: float, rows, causal=True, scale=1.0):
+def rmm_qk_rows(Qh: np.ndarray, Kg: np.ndarray, rho: float, rows, causal=True, scale=1.0, I=None):
     """Rows ``rows`` of one head's reduced scores: Qh [nq, dh] (the query head),
-    Kg [nk, dh] (its GQA key head).  Returns (S_rows, I)."""
+    Kg [nk, dh] (its GQA key head).  I = the oracle's own TopK of Qh's column norms,
+    or the given index set.  Returns (S_rows, I)."""
     return _qk_head(np.asarray(Qh, dtype=np.float64), np.asarray(Kg, dtype=np.float64),
-                    rho, causal, scale, rows)
+                    rho, causal, scale, rows, I)
 
 
-def _pv_head(Ph, Vg, rho, causal, rows=None):
+def pv_output_rows(Ph: np.ndarray, Vg: np.ndarray, I, rows=None, causal: bool = True):
+    """Rows ``rows`` of one head's reduced attention output on a GIVEN index set I:
+        O[i, :] = sum_{j in I, j visible to i} Ph[i, j] * Vg[j, :]
+    (entries of P above the bottom-right aligned diagonal count as zero).
+
+    [DD] "Component mapping": PV contracts over the kept token positions only, the
+    V rows of those positions gathered.  Ph [nq, nk], Vg [nk, dh]."""
+    Ph = np.asarray(Ph, dtype=np.float64)
+    Vg = np.asarray(Vg, dtype=np.float64)
     nq, nk = Ph.shape
-    k = retention_count(rho, nk)
-    q = column_sq_norms(Ph, causal)
-    I = topk_ascending(np.sqrt(q), k)
+    I = _check_index_set(I, nk, "pv_output_rows")
     r = np.arange(nq) if rows is None else np.asarray(rows)
     Pr = Ph[r][:, I].copy()
     if causal:
         vis = np.array([_visible_cols(i, nq, nk) for i in r])
         Pr[I[None, :] >= vis[:, None]] = 0.0
-    return Pr @ Vg[I, :], I, q
+    return Pr @ Vg[I, :]
+
+
+def _pv_head(Ph, Vg, rho, causal, rows=None, I=None):
+    nq, nk = Ph.shape
+    q = column_sq_norms(Ph, causal)
+    if I is None:
+        k = retention_count(rho, nk)
+        I = topk_ascending(np.sqrt(q), k)
+    I = _check_index_set(I, nk, "pv")
+    return pv_output_rows(Ph, Vg, I, rows, causal), I, q
 
 
 def rmm_pv(P: np.ndarray, V: np.ndarray, rho: float, causal: bool = True):
@@ -264,9 +307,10 @@ def rmm_pv(P: np.ndarray, V: np.ndarray, rho: float, causal: bool = True):
     return {"O": O, "I": I}
 
 
-def rmm_pv_rows(Ph: np.ndarray, Vg: np.ndarray, rho: float, rows, causal=True):
-    """Rows ``rows`` of one head's reduced PV output.  Returns (O_rows, I, q)."""
-    return _pv_head(np.asarray(Ph, dtype=np.float64), np.asarray(Vg, dtype=np.float64), rho, causal, rows)
+def rmm_pv_rows(Ph: np.ndarray, Vg: np.ndarray, rho: float, rows, causal=True, I=None):
+    """Rows ``rows`` of one head's reduced PV output, on the oracle's own TopK of the
+    column norms of Ph or on the given index set.  Returns (O_rows, I, q)."""
+    return _pv_head(np.asarray(Ph, dtype=np.float64), np.asarray(Vg, dtype=np.float64), rho, causal, rows, I)
 
 
 def _group(hq: int, hkv: int) -> int:
@@ -349,9 +393,22 @@ def rmm_mlp_gate_up(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, rho: float):
     Down component analysis.  Returns dict(H, I, G, U).
     """
     I, _, _ = select(X, rho)
-    G = reduced_product(X, Wg, I)
-    U = reduced_product(X, Wu, I)
-    return {"H": silu(G) * U, "I": I, "G": G, "U": U}
+    H, G, U = mlp_gate_up_rows(X, Wg, Wu, I, rows=None, parts=True)
+    return {"H": H, "I": I, "G": G, "U": U}
+
+
+def mlp_gate_up_rows(X: np.ndarray, Wg: np.ndarray, Wu: np.ndarray, I, rows=None, parts: bool = False):
+    """Rows ``rows`` of H = SiLU(X[:, I] Wg[I, :]) * (X[:, I] Wu[I, :]) on a GIVEN index
+    set I (the one set shared by gate and up, see ``rmm_mlp_gate_up``).  With ``parts``
+    returns (H, G, U)."""
+    X = np.asarray(X, dtype=np.float64)
+    I = _check_index_set(I, X.shape[1], "mlp_gate_up_rows")
+    r = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
+    Xr = X[r]
+    G = reduced_product(Xr, Wg, I)
+    U = reduced_product(Xr, Wu, I)
+    H = silu(G) * U
+    return (H, G, U) if parts else H
 
 
 def rmm_mlp(X, Wg, Wu, Wd, rho_gu: float, rho_down: float):
@@ -374,10 +431,19 @@ def rmm_linear_int8(A: np.ndarray, Wq: np.ndarray, scale: np.ndarray, rho: float
     stored weights are int8.  Returns dict(Y, I).
     """
     A = np.asarray(A, dtype=np.float64)
+    I, _, _ = select(A, rho)
+    return {"Y": int8_product_rows(A, Wq, scale, I), "I": I}
+
+
+def int8_product_rows(A: np.ndarray, Wq: np.ndarray, scale: np.ndarray, I, rows=None) -> np.ndarray:
+    """Rows ``rows`` of (A[:, I] . Wq[I, :]) * scale[None, :] on a GIVEN index set I
+    (int8 codes widened exactly, one scale per output column; see ``rmm_linear_int8``)."""
+    A = np.asarray(A, dtype=np.float64)
     Wq = np.asarray(Wq, dtype=np.float64)
     scale = np.asarray(scale, dtype=np.float64)
-    I, _, _ = select(A, rho)
-    return {"Y": (A[:, I] @ Wq[I, :]) * scale[None, :], "I": I}
+    I = _check_index_set(I, A.shape[1], "int8_product_rows")
+    r = np.arange(A.shape[0]) if rows is None else np.asarray(rows)
+    return (A[r][:, I] @ Wq[I, :]) * scale[None, :]
 
 
 def rmm_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rho: float, causal: bool = True,
@@ -404,9 +470,27 @@ def rmm_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, rho: float, causa
     for b in range(Bsz):
         for h in range(hq):
             g = kv_head(h, hq, hkv)
-            S, I[b, h] = _qk_head(Q[b, h], K[b, g], rho, causal, scale)
-            S = S - S.max(axis=1, keepdims=True)
-            P = np.exp(S)
-            P /= P.sum(axis=1, keepdims=True)
-            O[b, h] = P @ V[b, g]
+            O[b, h], I[b, h] = rmm_attention_rows(Q[b, h], K[b, g], V[b, g], rho, None, causal, scale)
     return {"O": O, "I": I}
+
+
+def attention_rows(Qh: np.ndarray, Kg: np.ndarray, Vg: np.ndarray, I, rows=None, causal: bool = True,
+                   scale: float = 1.0) -> np.ndarray:
+    """Rows ``rows`` of one head's attention output with the reduced score product on
+    a GIVEN index set I: softmax_rows(qk_scores_rows(...)) . Vg (see ``rmm_attention``).
+    The row maximum is subtracted before exponentiating (it cancels in the ratio)."""
+    S = qk_scores_rows(Qh, Kg, I, rows, causal, scale)
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P /= P.sum(axis=1, keepdims=True)
+    return P @ np.asarray(Vg, dtype=np.float64)
+
+
+def rmm_attention_rows(Qh, Kg, Vg, rho: float, rows=None, causal: bool = True, scale: float = 1.0, I=None):
+    """Rows ``rows`` of one head of ``rmm_attention``: I = the oracle's TopK of Qh's
+    column norms (or the given set), then ``attention_rows``.  Returns (O_rows, I)."""
+    Qh = np.asarray(Qh, dtype=np.float64)
+    if I is None:
+        I = topk_ascending(column_norms(Qh), retention_count(rho, Qh.shape[1]))
+    I = _check_index_set(I, Qh.shape[1], "attention")
+    return attention_rows(Qh, Kg, Vg, I, rows, causal, scale), I

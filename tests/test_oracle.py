@@ -540,3 +540,89 @@ def test_qk_and_pv_rows_match_the_full_products():
         assert np.array_equal(I, fullp["I"][0, h])
         assert np.array_equal(O, fullp["O"][0, h][[1, 5]])
         assert np.array_equal(q, oracle.column_sq_norms(P[0, h], causal=True))
+
+
+def test_products_on_a_given_index_set_bruteforce_loops():
+    """The index-set-given restatements (the references of the GPU parity checks when
+    the library's set is used) against explicit Python loops, on a set that is NOT
+    the TopK one, so that a function silently re-selecting would fail."""
+    g = np.random.default_rng(22)
+    nq, nk, dh = 5, 7, 6
+    Qh, Kg, Vg = g.standard_normal((nq, dh)), g.standard_normal((nk, dh)), g.standard_normal((nk, 3))
+    I = np.array([0, 2, 5])
+    Qh[:, 1] *= 10.0  # column 1 dominates the norms, so TopK would keep it; I does not
+    assert 1 in oracle.topk_ascending(oracle.column_norms(Qh), 3) and 1 not in I
+    rows = [0, 2, 4]
+    S = oracle.qk_scores_rows(Qh, Kg, I, rows, causal=True, scale=0.5)
+    for a, i in enumerate(rows):
+        for j in range(nk):
+            if j > i + (nk - nq):
+                assert S[a, j] == -np.inf
+            else:
+                ref = 0.5 * sum(Qh[i, t] * Kg[j, t] for t in I)
+                assert abs(S[a, j] - ref) < 1e-12
+    # attention on the given set: softmax over the visible keys, then V
+    O = oracle.attention_rows(Qh, Kg, Vg, I, rows, causal=True, scale=0.5)
+    for a, i in enumerate(rows):
+        vis = range(i + (nk - nq) + 1)
+        sc = [0.5 * sum(Qh[i, t] * Kg[j, t] for t in I) for j in vis]
+        mx = max(sc)
+        w = [math.exp(x - mx) for x in sc]
+        for c in range(3):
+            ref = sum(w[j] * Vg[j, c] for j in vis) / sum(w)
+            assert abs(O[a, c] - ref) < 1e-12
+    # PV on a given set of key positions: entries above the diagonal count as zero
+    Ph = np.abs(g.standard_normal((nq, nk)))
+    J = np.array([1, 3, 6])
+    Opv = oracle.pv_output_rows(Ph, Vg, J, rows, causal=True)
+    for a, i in enumerate(rows):
+        for c in range(3):
+            ref = sum(Ph[i, j] * Vg[j, c] for j in J if j <= i + (nk - nq))
+            assert abs(Opv[a, c] - ref) < 1e-12
+    # int8 codes with per-column scales, and the MLP gate/up on one shared set
+    A = g.standard_normal((4, 6))
+    Wq = g.integers(-127, 128, size=(6, 5)).astype(np.float64)
+    sc8 = g.uniform(0.01, 0.1, 5)
+    Y8 = oracle.int8_product_rows(A, Wq, sc8, I, [1, 3])
+    Wg, Wu = g.standard_normal((6, 5)), g.standard_normal((6, 5))
+    H = oracle.mlp_gate_up_rows(A, Wg, Wu, I, [1, 3])
+    for a, i in enumerate([1, 3]):
+        for c in range(5):
+            assert abs(Y8[a, c] - sc8[c] * sum(A[i, t] * Wq[t, c] for t in I)) < 1e-12
+            gte = sum(A[i, t] * Wg[t, c] for t in I)
+            up = sum(A[i, t] * Wu[t, c] for t in I)
+            assert abs(H[a, c] - gte / (1.0 + math.exp(-gte)) * up) < 1e-12
+
+
+def test_row_functions_match_the_full_functions():
+    """With no index set given, every row function reproduces exactly the rows of the
+    full function it samples, with the same index set (the full functions are pinned
+    by the hand fixtures and brute force above)."""
+    g = np.random.default_rng(23)
+    Q, K, V = g.standard_normal((1, 4, 9, 8)), g.standard_normal((1, 2, 9, 8)), g.standard_normal((1, 2, 9, 8))
+    full = oracle.rmm_attention(Q, K, V, 0.5, causal=True, scale=0.4)
+    for h in range(4):
+        gk = oracle.kv_head(h, 4, 2)
+        O, I = oracle.rmm_attention_rows(Q[0, h], K[0, gk], V[0, gk], 0.5, [0, 4, 8], causal=True, scale=0.4)
+        assert np.array_equal(I, full["I"][0, h])
+        assert np.array_equal(O, full["O"][0, h][[0, 4, 8]])
+        O2, _ = oracle.rmm_attention_rows(Q[0, h], K[0, gk], V[0, gk], 0.5, [0, 4, 8], causal=True, scale=0.4, I=I)
+        assert np.array_equal(O2, O)
+    X = g.standard_normal((6, 10))
+    Wg, Wu, Wq = g.standard_normal((10, 4)), g.standard_normal((10, 4)), g.integers(-127, 128, (10, 4))
+    sc = g.uniform(0.01, 0.1, 4)
+    gu = oracle.rmm_mlp_gate_up(X, Wg, Wu, 0.6)
+    assert np.array_equal(oracle.mlp_gate_up_rows(X, Wg, Wu, gu["I"], [1, 5]), gu["H"][[1, 5]])
+    i8 = oracle.rmm_linear_int8(X, Wq, sc, 0.6)
+    assert np.array_equal(oracle.int8_product_rows(X, Wq, sc, i8["I"], [0, 2]), i8["Y"][[0, 2]])
+    P = np.abs(g.standard_normal((1, 1, 8, 8)))
+    fullp = oracle.rmm_pv(P, V[:, :1, :8], 0.5, causal=True)
+    Oi, Ii, _ = oracle.rmm_pv_rows(P[0, 0], V[0, 0, :8], 0.5, [2, 7], causal=True, I=fullp["I"][0, 0])
+    assert np.array_equal(Oi, fullp["O"][0, 0][[2, 7]]) and np.array_equal(Ii, fullp["I"][0, 0])
+
+
+@pytest.mark.parametrize("bad", [[2, 1], [1, 1], [-1, 2], [0, 8], []])
+def test_given_index_sets_must_be_ascending_and_in_range(bad):
+    Qh, Kg = np.ones((3, 8)), np.ones((3, 8))
+    with pytest.raises(ValueError):
+        oracle.qk_scores_rows(Qh, Kg, np.array(bad, dtype=np.int64), None)
