@@ -25,3 +25,22 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Log of the index-set comparisons: how many sets were compared and how many
+    differed from the oracle's inside the near-tie band (norms within 1e-5
+    relative of the k-th largest)."""
+    try:
+        from parity import NEAR_TIE_LOG
+    except Exception:  # pragma: no cover
+        return
+    if not NEAR_TIE_LOG:
+        return
+    sets = len(NEAR_TIE_LOG)
+    differing = [(w, k, t) for w, k, t in NEAR_TIE_LOG if t]
+    total = sum(t for _, _, t in differing)
+    terminalreporter.write_line(f"index sets compared with the oracle: {sets}; sets with near-tie differences: "
+                                f"{len(differing)}; indices swapped inside the band: {total}")
+    for w, k, t in differing[:20]:
+        terminalreporter.write_line(f"  {w}: {t} of k={k}")

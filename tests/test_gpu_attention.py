@@ -1,13 +1,17 @@
 """GPU parity of the attention-side reductions: rmm_qk (head-dim selection on Q,
 K gathered under GQA, causal -inf scores) and rmm_pv (token-position selection
-on P, V rows gathered)."""
+on P, V rows gathered).
+
+Every reference below is an oracle function: the index sets against the oracle's
+TopK of its own fp64 scores (near-tie band logged), the products against
+oracle.qk_scores_rows / oracle.pv_output_rows on the library's own index set."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synthetic
-from parity import check_close, check_index_set
+from parity import check_close, check_colsq, check_index_set
 
 pytestmark = pytest.mark.gpu
 
@@ -22,29 +26,27 @@ def built():
     assert rmm.device_error() == 0
 
 
-def qk_parity(Q, K, rho, causal, scale=1.0, heads=None, rows=None):
-    S, idx = rmm.qk(Q.cuda(), K.cuda(), rho, causal=causal, scale=scale, return_idx=True)
-    torch.cuda.synchronize()
+def check_qk_heads(S, idx, Q, K, rho, causal, scale, rows=None):
+    """Every head: index set vs the oracle's, sampled (or all) rows of S vs
+    oracle.qk_scores_rows on the library's set."""
     Qw, Kw = synthetic.widen(Q), synthetic.widen(K)
     b_, hq, nq, dh = Q.shape
     hkv = K.shape[1]
     k = oracle.retention_count(rho, dh)
-    heads = range(hq) if heads is None else heads
+    r = np.arange(nq) if rows is None else np.asarray(rows)
+    rsel = torch.as_tensor(r, device=S.device)
     for b in range(b_):
-        for h in heads:
-            q = oracle.column_sq_norms(Qw[b, h])
+        for h in range(hq):
             I = idx[b, h].cpu().numpy().astype(np.int64)
-            check_index_set(I, q, k)
-            r = np.arange(nq) if rows is None else np.asarray(rows)
-            Qh = Qw[b, h][r][:, I]
-            Kg = Kw[b, oracle.kv_head(h, hq, hkv)][:, I]
-            ref = scale * (Qh @ Kg.T)
-            if causal:
-                nk = K.shape[2]
-                vis = np.minimum(nk, r + (nk - nq) + 1)
-                ref[np.arange(nk)[None, :] >= vis[:, None]] = -np.inf
-            got = S[b, h][torch.as_tensor(r, device=S.device)].cpu().numpy()
-            check_close(got, ref, f"qk head {h}")
+            check_index_set(I, oracle.column_sq_norms(Qw[b, h]), k, f"qk rho={rho} head {b}/{h}")
+            ref = oracle.qk_scores_rows(Qw[b, h], Kw[b, oracle.kv_head(h, hq, hkv)], I, r, causal, scale)
+            check_close(S[b, h][rsel].cpu().numpy(), ref, f"qk head {h}")
+
+
+def qk_parity(Q, K, rho, causal, scale=1.0, rows=None):
+    S, idx = rmm.qk(Q.cuda(), K.cuda(), rho, causal=causal, scale=scale, return_idx=True)
+    torch.cuda.synchronize()
+    check_qk_heads(S, idx, Q, K, rho, causal, scale, rows)
     return S, idx
 
 
@@ -71,37 +73,48 @@ def test_qk_rectangular_causal_alignment():
     qk_parity(Q, K, 0.5, True)
 
 
-@pytest.mark.parametrize("rho", [0.5, 0.7])
-def test_qk_gqa_seq4096_sampled(rho):
-    """32 query heads / 8 key-value heads, head_dim 128, seq 4096, causal fp32 scores."""
+def test_qk_gqa_seq4096_all_heads():
+    """32 query heads / 8 key-value heads, head_dim 128, seq 4096, causal fp32 scores
+    at rho = 0.7 and 0.5: the GPU's fp64 column scores of all 32 heads against the
+    oracle's, every head's index set, and a row sample of every head's scores."""
     Q, K = synthetic.qk_inputs()
-    rows = np.concatenate([np.arange(0, 4096, 257), [4095]])
-    qk_parity(Q, K, rho, True, heads=[0, 3, 4, 17, 31], rows=rows)
-
-
-def pv_parity(P, V, rho, causal, heads=None, rows=None):
-    O, idx = rmm.pv(P.cuda() if not P.is_cuda else P, V.cuda() if not V.is_cuda else V, rho, causal=causal,
-                    return_idx=True)
+    Qd, Kd = Q.cuda(), K.cuda()
+    _, cs, _ = rmm.select(Qd[0], 0.5)  # the selection kernels rmm_qk runs, batched over heads
     torch.cuda.synchronize()
+    Qw = synthetic.widen(Q)
+    for h in range(Q.shape[1]):
+        check_colsq(cs[h].cpu().numpy(), oracle.column_sq_norms(Qw[0, h]))
+    rows = np.concatenate([np.arange(0, 4096, 257), [4095]])
+    for rho in (0.7, 0.5):
+        S, idx = rmm.qk(Qd, Kd, rho, causal=True, return_idx=True)
+        torch.cuda.synchronize()
+        check_qk_heads(S, idx, Q, K, rho, True, 1.0, rows)
+        del S
+    torch.cuda.empty_cache()
+
+
+def check_pv_heads(O, idx, P, V, rho, causal, rows=None):
     b_, h_, nq, nk = P.shape
     hkv = V.shape[1]
     k = oracle.retention_count(rho, nk)
-    heads = range(h_) if heads is None else heads
+    r = np.arange(nq) if rows is None else np.asarray(rows)
+    rsel = torch.as_tensor(r, device=O.device)
     for b in range(b_):
-        for h in heads:
+        for h in range(h_):
             Ph = synthetic.widen(P[b, h])
             Vg = synthetic.widen(V[b, oracle.kv_head(h, h_, hkv)])
             q = oracle.column_sq_norms(Ph, causal=causal)
             I = idx[b, h].cpu().numpy().astype(np.int64)
-            check_index_set(I, q, k)
-            r = np.arange(nq) if rows is None else np.asarray(rows)
-            Pr = Ph[r][:, I].copy()
-            if causal:
-                vis = np.minimum(nk, r + (nk - nq) + 1)
-                Pr[I[None, :] >= vis[:, None]] = 0.0
-            ref = Pr @ Vg[I, :]
-            got = synthetic.widen(O[b, h][torch.as_tensor(r, device=O.device)].cpu())
-            check_close(got, ref, f"pv head {h}")
+            check_index_set(I, q, k, f"pv rho={rho} head {b}/{h}")
+            ref = oracle.pv_output_rows(Ph, Vg, I, r, causal)
+            check_close(synthetic.widen(O[b, h][rsel].cpu()), ref, f"pv head {h}")
+
+
+def pv_parity(P, V, rho, causal, rows=None):
+    O, idx = rmm.pv(P.cuda() if not P.is_cuda else P, V.cuda() if not V.is_cuda else V, rho, causal=causal,
+                    return_idx=True)
+    torch.cuda.synchronize()
+    check_pv_heads(O, idx, P, V, rho, causal, rows)
     return O, idx
 
 
@@ -118,17 +131,18 @@ def test_pv_head_dim_64_and_gqa():
 
 
 def test_pv_entry_point_with_junk_above_diagonal():
+    """Garbage above the diagonal: index sets against the oracle's causal scores, the
+    output against oracle.pv_output_rows on the library's own sets (always), and the
+    oracle's entry point as a whole (its own sets equal the library's here)."""
     P, V = synthetic.pv_inputs(heads=2, n=200)
     junk = torch.triu(torch.full((200, 200), 3.0), 1).to(torch.bfloat16)
     Pj = P + junk
     O, idx = rmm.pv(Pj.cuda(), V.cuda(), 0.5, causal=True, return_idx=True)
     torch.cuda.synchronize()
+    check_pv_heads(O, idx, Pj, V, 0.5, True)
     ref = oracle.rmm_pv(synthetic.widen(Pj), synthetic.widen(V), 0.5, causal=True)
-    for h in range(2):
-        q = oracle.column_sq_norms(synthetic.widen(Pj[0, h]), causal=True)
-        check_index_set(idx[0, h].cpu().numpy(), q, 100)
-    if np.array_equal(idx.cpu().numpy(), ref["I"]):
-        check_close(synthetic.widen(O.cpu()), ref["O"], "pv entry point")
+    assert np.array_equal(idx.cpu().numpy(), ref["I"])
+    check_close(synthetic.widen(O.cpu()), ref["O"], "pv entry point")
 
 
 @pytest.mark.parametrize("rho", [1.0, 0.8])
@@ -136,25 +150,36 @@ def test_pv_dense_and_reduced_ignore_entries_above_the_diagonal(rho):
     """Causal PV treats P[i, j] with j > i + (nk - nq) as zero on every path."""
     P, V = synthetic.pv_inputs(heads=2, n=328)
     junk = torch.triu(torch.full((328, 328), 5.0), 1).to(torch.bfloat16)
-    Pj = P + junk
-    O, idx = rmm.pv(Pj.cuda(), V.cuda(), rho, causal=True, return_idx=True)
-    torch.cuda.synchronize()
-    for h in range(2):
-        q = oracle.column_sq_norms(synthetic.widen(Pj[0, h]), causal=True)
-        I = idx[0, h].cpu().numpy().astype(np.int64)
-        check_index_set(I, q, oracle.retention_count(rho, 328))
-        Ph = synthetic.widen(Pj[0, h])
-        Pr = Ph[:, I].copy()
-        Pr[I[None, :] > np.arange(328)[:, None]] = 0.0
-        check_close(synthetic.widen(O[0, h].cpu()), Pr @ synthetic.widen(V[0, h])[I, :], f"pv junk head {h}")
+    pv_parity(P + junk, V, rho, True)
 
 
-@pytest.mark.parametrize("rho", [0.5, 0.8])
-def test_pv_seq16384_sampled(rho):
+def test_pv_seq16384_all_heads():
     """Long-context PV: 32 heads x 16384 x 16384 causal softmax probabilities drawn on
-    the device; two heads and a row sample are checked against the oracle."""
+    the device, rho = 0.8 and 0.5.  All 32 heads: the GPU's fp64 causal column scores
+    against the oracle's, the index sets, and a row sample of each head's output
+    against oracle.pv_output_rows on the library's set.  Each head is widened once for
+    both rho values."""
     P, V = synthetic.pv_inputs_device("cuda", heads=32, n=16384)
+    b_, h_, nq, nk = P.shape
     rows = np.concatenate([np.arange(0, 16384, 1031), [16383]])
-    pv_parity(P, V, rho, True, heads=[0, 29], rows=rows)
+    rsel = torch.as_tensor(rows, device="cuda")
+    runs = {}
+    for rho in (0.8, 0.5):
+        O, idx = rmm.pv(P, V, rho, causal=True, return_idx=True)
+        torch.cuda.synchronize()
+        runs[rho] = (synthetic.widen(O[0][:, rsel].cpu()), idx[0].cpu().numpy().astype(np.int64))
+        del O
+    _, cs, _ = rmm.select(P[0], 0.5, causal=True)
+    torch.cuda.synchronize()
+    cs = cs.cpu().numpy()
+    for h in range(h_):
+        Ph = synthetic.widen(P[0, h].cpu())
+        Vg = synthetic.widen(V[0, h].cpu())
+        q = oracle.column_sq_norms(Ph, causal=True)
+        check_colsq(cs[h], q)
+        for rho, (Orows, I) in runs.items():
+            check_index_set(I[h], q, oracle.retention_count(rho, nk), f"pv seq16384 rho={rho} head {h}")
+            check_close(Orows[h], oracle.pv_output_rows(Ph, Vg, I[h], rows, True), f"pv seq16384 head {h}")
+        del Ph
     del P, V
     torch.cuda.empty_cache()

@@ -1,13 +1,14 @@
 """GPU parity of the fused attention with a reduced score product (rmm_attention):
 per query head, the index set of rmm_qk, then softmax(scale Q_I K_I^T) V with S
-and P kept on chip."""
+and P kept on chip.  References: the oracle's TopK for the index sets (near-tie
+band logged) and oracle.attention_rows on the library's own set for the output."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synthetic
-from parity import check_close, check_index_set
+from parity import check_close, check_colsq, check_index_set
 
 pytestmark = pytest.mark.gpu
 
@@ -22,36 +23,26 @@ def built():
     assert rmm.device_error() == 0
 
 
-def attention_ref(Qh, Kg, Vg, I, causal, scale, rows=None):
-    """Reference output rows of one head on the GPU's index set (float64)."""
-    nq, nk = Qh.shape[0], Kg.shape[0]
-    r = np.arange(nq) if rows is None else np.asarray(rows)
-    S = scale * (Qh[r][:, I] @ Kg[:, I].T)
-    if causal:
-        vis = r + (nk - nq) + 1
-        S[np.arange(nk)[None, :] >= vis[:, None]] = -np.inf
-    S -= S.max(axis=1, keepdims=True)
-    P = np.exp(S)
-    P /= P.sum(axis=1, keepdims=True)
-    return P @ Vg
-
-
-def fused_parity(Q, K, V, rho, causal, scale, heads=None, rows=None):
-    O, idx = rmm.attention(Q.cuda(), K.cuda(), V.cuda(), rho, causal=causal, scale=scale, return_idx=True)
-    torch.cuda.synchronize()
+def check_heads(O, idx, Q, K, V, rho, causal, scale, rows=None):
     B, hq, nq, dh = Q.shape
     hkv = K.shape[1]
     k = oracle.retention_count(rho, dh)
-    heads = range(hq) if heads is None else heads
+    r = np.arange(nq) if rows is None else np.asarray(rows)
+    rsel = torch.as_tensor(r, device=O.device)
     for b in range(B):
-        for h in heads:
+        for h in range(hq):
             Qh = synthetic.widen(Q[b, h])
             g = oracle.kv_head(h, hq, hkv)
             I = idx[b, h].cpu().numpy().astype(np.int64)
-            check_index_set(I, oracle.column_sq_norms(Qh), k)
-            ref = attention_ref(Qh, synthetic.widen(K[b, g]), synthetic.widen(V[b, g]), I, causal, scale, rows)
-            r = np.arange(nq) if rows is None else np.asarray(rows)
-            check_close(synthetic.widen(O[b, h].cpu())[r], ref, f"fused attention head {h}")
+            check_index_set(I, oracle.column_sq_norms(Qh), k, f"fused attention rho={rho} head {b}/{h}")
+            ref = oracle.attention_rows(Qh, synthetic.widen(K[b, g]), synthetic.widen(V[b, g]), I, r, causal, scale)
+            check_close(synthetic.widen(O[b, h][rsel].cpu()), ref, f"fused attention head {h}")
+
+
+def fused_parity(Q, K, V, rho, causal, scale, rows=None):
+    O, idx = rmm.attention(Q.cuda(), K.cuda(), V.cuda(), rho, causal=causal, scale=scale, return_idx=True)
+    torch.cuda.synchronize()
+    check_heads(O, idx, Q, K, V, rho, causal, scale, rows)
     return O, idx
 
 
@@ -88,10 +79,16 @@ def test_fused_attention_matches_oracle_and_repeats():
     check_close(synthetic.widen(O1.cpu()), ref["O"], "fused attention entry point")
 
 
-@pytest.mark.parametrize("rho", [0.5, 0.7])
-def test_fused_attention_gqa_seq4096_sampled(rho):
-    """32 query / 8 key-value heads, seq 4096, causal: sampled heads and rows."""
+def test_fused_attention_gqa_seq4096_all_heads():
+    """32 query / 8 key-value heads, seq 4096, causal, rho = 0.7 and 0.5: the GPU's
+    fp64 column scores and index sets of all 32 heads, and a row sample of every
+    head's output."""
     Q, K = synthetic.qk_inputs()
     V = synthetic.to_bf16(synthetic.rng(43).standard_normal((1, 8, 4096, 128), dtype=np.float32))
+    _, cs, _ = rmm.select(Q[0].cuda(), 0.5)
+    torch.cuda.synchronize()
+    for h in range(32):
+        check_colsq(cs[h].cpu().numpy(), oracle.column_sq_norms(synthetic.widen(Q[0, h])))
     rows = np.concatenate([np.arange(0, 4096, 397), [4095]])
-    fused_parity(Q, K, V, rho, True, 0.088, heads=[0, 5, 31], rows=rows)
+    for rho in (0.7, 0.5):
+        fused_parity(Q, K, V, rho, True, 0.088, rows=rows)

@@ -37,7 +37,7 @@ def decode_qk_parity(Q, Kt, rho, nk, scale=1.0, groups=None):
                 continue
             A = Qw[b, g * G:(g + 1) * G]
             I = idx[b, g].cpu().numpy().astype(np.int64)
-            check_index_set(I, oracle.column_sq_norms(A), k)
+            check_index_set(I, oracle.column_sq_norms(A), k, f"decode qk rho={rho} group {b}/{g}")
             ref = scale * oracle.reduced_product(A, synthetic.widen(Kt[b, g, :, :nk]), I)
             check_close(Sc[b, g * G:(g + 1) * G, :nk], ref, f"decode qk group {b}/{g}")
     return S, idx
@@ -58,7 +58,7 @@ def decode_pv_parity(P, V, rho, nk, groups=None):
                 continue
             A = synthetic.widen(P[b, g * G:(g + 1) * G, :nk].cpu())
             I = idx[b, g].cpu().numpy().astype(np.int64)
-            check_index_set(I, oracle.column_sq_norms(A), k)
+            check_index_set(I, oracle.column_sq_norms(A), k, f"decode pv rho={rho} group {b}/{g}")
             ref = oracle.reduced_product(A, synthetic.widen(V[b, g, :nk].cpu()), I)
             check_close(Oc[b, g * G:(g + 1) * G], ref, f"decode pv group {b}/{g}")
     return O, idx
@@ -90,8 +90,15 @@ def test_decode_matches_oracle_entry_points_and_repeats():
     rp = oracle.rmm_decode_pv(synthetic.widen(P), synthetic.widen(V), 0.5, nk=333)
     assert np.array_equal(I1.cpu().numpy(), rq["I"])
     check_close(S1.cpu().numpy(), rq["S"], "decode qk entry point")
-    if np.array_equal(J1.cpu().numpy(), rp["I"]):
-        check_close(synthetic.widen(O1.cpu()), rp["O"], "decode pv entry point")
+    # the output on the library's own index set, whatever the near-tie band holds ...
+    A = synthetic.widen(P[0, :, :333])
+    J = J1[0, 0].cpu().numpy().astype(np.int64)
+    check_index_set(J, oracle.column_sq_norms(A), oracle.retention_count(0.5, 333), "decode pv entry point")
+    check_close(synthetic.widen(O1.cpu())[0], oracle.reduced_product(A, synthetic.widen(V[0, 0, :333]), J),
+                "decode pv on the library's set")
+    # ... and the oracle's entry point as a whole (its set equals the library's here)
+    assert np.array_equal(J1.cpu().numpy(), rp["I"])
+    check_close(synthetic.widen(O1.cpu()), rp["O"], "decode pv entry point")
 
 
 def test_decode_cache_past_nk_is_not_read():

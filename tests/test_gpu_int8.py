@@ -1,6 +1,7 @@
 """GPU parity of the reduced projection with int8 weights (rmm_linear_int8):
 the selection on the bf16 activations, then (A[:, I] Wq[I, :]) * scale from the
-kept int8 rows only."""
+kept int8 rows only.  References: the oracle's TopK for the index set and
+oracle.int8_product_rows on the library's own set for the product."""
 import numpy as np
 import pytest
 import torch
@@ -27,8 +28,9 @@ def int8_parity(A, Wq, s, rho):
     torch.cuda.synchronize()
     Aw = synthetic.widen(A)
     I = idx.cpu().numpy().astype(np.int64)
-    check_index_set(I, oracle.column_sq_norms(Aw), oracle.retention_count(rho, A.shape[1]))
-    ref = (Aw[:, I] @ Wq.numpy().astype(np.float64)[I, :]) * s.numpy().astype(np.float64)[None, :]
+    check_index_set(I, oracle.column_sq_norms(Aw), oracle.retention_count(rho, A.shape[1]),
+                    f"int8 n={A.shape[0]} d={A.shape[1]} rho={rho}")
+    ref = oracle.int8_product_rows(Aw, Wq.numpy(), s.numpy(), I)
     check_close(synthetic.widen(Y.cpu()), ref, "int8 product")
     return Y, idx
 

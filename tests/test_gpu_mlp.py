@@ -3,9 +3,9 @@ the fused tensor-core product writing H = SiLU(gate) * up, and the down projecti
 as RMM on H with its own rho.
 
 Stage by stage: the gate / up index set is compared with the oracle's on X; H
-with the oracle's SiLU(gate) * up on the GPU's index set; the down projection
-with the oracle's RMM on the GPU's own H (H is bf16, so its column norms, and
-with them the down selection, are those of the rounded H)."""
+with oracle.mlp_gate_up_rows on the GPU's index set; the down projection with
+the oracle's RMM on the GPU's own H (H is bf16, so its column norms, and with
+them the down selection, are those of the rounded H)."""
 import numpy as np
 import pytest
 import torch
@@ -35,15 +35,15 @@ def mlp_parity(X, Wg, Wu, Wd, rho_gu, rho_down, rows=None):
     f = Wg.shape[1]
     Xw = synthetic.widen(X)
     I = i_gu.cpu().numpy().astype(np.int64)
-    check_index_set(I, oracle.column_sq_norms(Xw), oracle.retention_count(rho_gu, d))
+    check_index_set(I, oracle.column_sq_norms(Xw), oracle.retention_count(rho_gu, d),
+                    f"mlp gate/up n={n} d={d} rho={rho_gu}")
     r = np.arange(n) if rows is None else np.asarray(rows)
-    Gm = Xw[r][:, I] @ synthetic.widen(Wg)[I, :]
-    Um = Xw[r][:, I] @ synthetic.widen(Wu)[I, :]
     Hw = synthetic.widen(H.cpu())
-    check_close(Hw[r], oracle.silu(Gm) * Um, "mlp H")
+    check_close(Hw[r], oracle.mlp_gate_up_rows(Xw, synthetic.widen(Wg), synthetic.widen(Wu), I, r), "mlp H")
     J = i_dn.cpu().numpy().astype(np.int64)
-    check_index_set(J, oracle.column_sq_norms(Hw), oracle.retention_count(rho_down, f))
-    check_close(synthetic.widen(Y.cpu())[r], oracle.reduced_product(Hw[r], synthetic.widen(Wd), J), "mlp Y")
+    check_index_set(J, oracle.column_sq_norms(Hw), oracle.retention_count(rho_down, f),
+                    f"mlp down n={n} f={f} rho={rho_down}")
+    check_close(synthetic.widen(Y.cpu())[r], oracle.rmm_linear_rows(Hw, synthetic.widen(Wd), J, r), "mlp Y")
     return Y, H
 
 
