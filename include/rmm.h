@@ -101,7 +101,10 @@ rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, in
  *     return RMM_ERR_UNSUPPORTED with a message naming the limit.
  *   - The first call on a device looks up the scratch array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make that
- *     first call before any stream capture on the device.
+ *     first call before any stream capture on the device.  The cache is keyed
+ *     on the current context's unique id, so a call after cudaDeviceReset (a
+ *     new context) looks the address up again: make that call before any
+ *     stream capture too.
  *   - Every call on a device shares the one array.  Calls whose kernels can
  *     overlap on the GPU (different streams without ordering between them)
  *     race on it and give undefined results; order them on one stream or with
@@ -311,6 +314,29 @@ const char* rmm_last_error(void);
 rmm_status rmm_device_error(int32_t* code_out);
 /* Library version, e.g. "rmm-b200 0.1". */
 const char* rmm_version(void);
+
+/* ---------------------------------------------------------------- test hooks
+ * Two entry points that exist only so that tests can reach device code no
+ * product call exposes on its own; neither is part of the method.
+ *
+ * rmm_debug_exp2_poly: y_poly[i] = the fused attention's FMA-pipe 2^x (a cubic
+ * fitted to 2^f on [0, 1): relative error <= 7.7e-5 for x in [-125, 0], <= 1.6e-4
+ * on [-126, -125) where the result can fall into the subnormal range, about
+ * 2^-126 below -126) and y_exp2f[i] = CUDA's exp2f(x[i]), i < n.  All three are
+ * device fp32 buffers.
+ *
+ * rmm_debug_gemm_expire_producer: rmm_gemm_packed's one-CTA tensor-core product
+ * (n <= 128 only) in which the producer, once its ring of shared-memory stages
+ * is full (k > 256), waits on a barrier that nothing arrives on, through the
+ * same bounded wait as every other wait but with a 1 ms limit instead of about
+ * one second.  That wait runs out and the kernel takes its timeout path: it
+ * records code 1 (producer timeout) in the device error word (rmm_device_error),
+ * the other roles see the abort and stop, copies in flight are drained, tensor
+ * memory is freed and the kernel returns.  Y is left partly written. */
+rmm_status rmm_debug_exp2_poly(const float* x, float* y_poly, float* y_exp2f, int64_t n, rmm_stream stream);
+rmm_status rmm_debug_gemm_expire_producer(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t lda,
+                                          const rmm_bf16* B_pack, int64_t m, int64_t ldb, rmm_bf16* Y, int64_t ldy,
+                                          rmm_stream stream);
 
 #ifdef __cplusplus
 }

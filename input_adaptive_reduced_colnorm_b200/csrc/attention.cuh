@@ -54,16 +54,32 @@ __device__ __forceinline__ float attn_exp2(float x) {
 
 // 2^x on the FMA pipe, for the half of the weights that do not go to the
 // special-function unit: x = n + f with n = floor(x) and f in [0, 1), 2^f from a
-// cubic fitted (relative-error minimax on [0, 1]) to max relative error 7.7e-5,
-// far below the bf16 rounding of P; 2^n is added to the exponent field.
-// Arguments below -126 give 2^-126 (the weight then rounds to 0 or the smallest
-// bf16 normal, far below every weight that matters).
+// cubic fitted (relative-error minimax on [0, 1]) to max relative error 7.7e-5
+// (7.64e-5, at f = 0), far below the bf16 rounding of P; 2^n is added to the
+// exponent field.  That bound holds for x in [-125, 0].  On [-126, -125) the
+// result is a normal float with the same bound except where n = -126 and the
+// cubic is below 1 (f < 1.1e-4): the sum then lands in the subnormal range and
+// the relative error reaches 1.5e-4.  Arguments below -126 give about 2^-126.
+// (Weights that small are 2^-125 of the row's largest weight, 1, and vanish
+// next to it in every sum.)
 __device__ __forceinline__ float attn_exp2_poly(float x) {
   x = fmaxf(x, -126.f);
   const float n = floorf(x);
   const float f = x - n;
   const float p = fmaf(fmaf(fmaf(0.0780965686f, f, 0.2259650975f), f, 0.6958683133f), f, 0.9999235868f);
   return __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
+}
+
+// Elementwise attn_exp2_poly and CUDA's exp2f, for the unit test of the fit
+// (rmm_debug_exp2_poly).
+__global__ void attn_exp2_probe_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                       float* __restrict__ y_ref, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    y_poly[i] = attn_exp2_poly(v);
+    y_ref[i] = exp2f(v);
+  }
 }
 
 // Visible key blocks of the query tile starting at row m0.

@@ -65,7 +65,15 @@ struct GemmParams {
   // narrow last wave (MN-major B only): the last tail_tiles tiles are cut into
   // tail_split pieces of BN / tail_split (>= 64) columns; 0 / 1 = no cut
   int tail_tiles, tail_split;
+  // test hook (0 in every product call): 1 makes the producer, once the stage
+  // ring is full, wait on a barrier that nothing arrives on, with a 1 ms limit,
+  // so that its bounded wait runs out and the kernel takes its timeout path
+  int expire_producer_waits;
 };
+
+// wait limit of the test hook's producer wait: far below the ~1 s of every other
+// wait, far above the polling granularity
+constexpr uint64_t kGemmHookWaitNs = 1000ull * 1000ull;
 
 template <int BN>
 struct GemmCfg {
@@ -76,7 +84,7 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
   static constexpr int EPI_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 chunks of 32 rows x 128 bytes
   static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + EPI_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(8 * (3 * STAGES + 5) + 8 <= 256, "barrier area");
+  static_assert(8 * (3 * STAGES + 6) + 8 <= 256, "barrier area");
 };
 
 __device__ __forceinline__ int64_t gemm_b_row_base(const GemmParams& p, int b) {
@@ -205,7 +213,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* ready = drain + 1;  // [STAGES]: diagonal A tiles masked (causal PV)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + STAGES);
+  uint64_t* never = ready + STAGES;  // test hook only: no thread ever arrives on it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,6 +229,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(drain, 1);
     for (int st = 0; st < STAGES; ++st) mbar_init(&ready[st], 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tmA);
@@ -254,7 +264,12 @@ __global__ void __launch_bounds__(192, 1)
       const int64_t brow0 = gemm_b_row_base(p, b);
       for (int kb = 0; kb < nkb; ++kb) {
         int w = 1;
-        if (lane == 0) w = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+        if (lane == 0) {
+          if (p.expire_producer_waits && issued == static_cast<uint32_t>(STAGES))
+            w = mbar_wait(never, 0u, abort_flag, kDevErrTimeoutProducer, 0, false, kGemmHookWaitNs) ? 1 : 0;
+          else
+            w = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+        }
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) {
           ok = false;

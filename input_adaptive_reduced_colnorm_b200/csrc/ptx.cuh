@@ -92,13 +92,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // Wait for the phase of ``bar`` with parity ``parity`` to complete.  Gives up
-// after kWaitTimeoutNs without progress, or as soon as *abort is set by another
-// role of the same CTA; on a timeout it sets *abort and records ``code``.
+// after ``limit_ns`` (kWaitTimeoutNs unless a test hook asks for less) without
+// progress, or as soon as *abort is set by another role of the same CTA; on a
+// timeout it sets *abort and records ``code``.
 // ``sleep_ns`` > 0 backs off between polls: threads that wait long (epilogue
 // warps waiting for a finished accumulator) then leave the issue slots to the
 // warps that are moving data.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t code,
-                                          uint32_t sleep_ns = 0, bool cluster_scope = false) {
+                                          uint32_t sleep_ns = 0, bool cluster_scope = false,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   const uint32_t a = smem_u32(bar);
   auto poll = [&]() { return cluster_scope ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity); };
   if (poll()) return true;
@@ -108,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (poll()) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         record_device_error(code);
         return false;

@@ -1159,6 +1159,44 @@ rmm_status rmm_device_error(int32_t* code_out) {
   return RMM_OK;
 }
 
+// ---------------------------------------------------------------- test hooks
+rmm_status rmm_debug_exp2_poly(const float* x, float* y_poly, float* y_exp2f, int64_t n, rmm_stream stream) {
+  t_last_error.clear();
+  if (x == nullptr || y_poly == nullptr || y_exp2f == nullptr || n < 1) return fail(RMM_ERR_INVALID_ARG, "bad arguments");
+  const int64_t grid = std::min<int64_t>(ceil_div(n, 256), 4LL * num_sms());
+  attn_exp2_probe_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_exp2f, n);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 probe launch");
+  return RMM_OK;
+}
+
+rmm_status rmm_debug_gemm_expire_producer(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t lda,
+                                          const rmm_bf16* B_pack, int64_t m, int64_t ldb, rmm_bf16* Y, int64_t ldy,
+                                          rmm_stream stream) {
+  t_last_error.clear();
+  if (A_pack == nullptr || B_pack == nullptr || Y == nullptr) return fail(RMM_ERR_INVALID_ARG, "null pointer");
+  if (n < 1 || k < 1 || m < 1 || lda < k || ldb < m || ldy < m)
+    return fail(RMM_ERR_INVALID_ARG, "need n, k, m >= 1, lda >= k, ldb and ldy >= m");
+  if (n > 128) return fail(RMM_ERR_UNSUPPORTED, "the hook runs the one-CTA product (n <= 128)");
+  if (!aligned16(A_pack) || !aligned16(B_pack) || !aligned16(Y) || (lda % 8) || (ldb % 8) || (ldy % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "pointers must be 16-byte aligned and leading dims multiples of 8");
+  if (m > kIntMax - 256 || k > kIntMax - 64) return fail(RMM_ERR_UNSUPPORTED, "dimension too large");
+  CUtensorMap ta, tb;
+  if (rmm_status st = make_tmap(&ta, A_pack, k, n, lda * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tb, B_pack, m, k, ldb * 2, 64, 64)) return st;
+  GemmParams g = gemm_defaults();
+  g.M = static_cast<int>(n);
+  g.N = static_cast<int>(m);
+  g.out = Y;
+  g.ldo = ldy;
+  g.m_tiles = 1;
+  g.n_tiles = static_cast<int>(ceil_div(m, 256));
+  g.k = static_cast<int>(k);
+  g.num_kb = static_cast<int>(ceil_div(k, 64));
+  g.expire_producer_waits = 1;
+  return launch_gemm<256, kBTileMN, kEpiBf16, kCausalNone>(ta, tb, g, static_cast<cudaStream_t>(stream));
+}
+
 // ---------------------------------------------------------------- select
 size_t rmm_select_workspace_bytes(int64_t batch, int64_t n, int64_t d) {
   (void)n;
@@ -1205,25 +1243,59 @@ rmm_status rmm_select(const rmm_bf16* A, int64_t batch, int64_t batch_stride, in
 }  // extern "C"
 
 namespace {
-constexpr int64_t kNoAllocScores = 262144;  // equals RMM_SELECT_NOALLOC_MAX_SCORES in rmm.h
+constexpr int64_t kNoAllocScores = RMM_SELECT_NOALLOC_MAX_SCORES;
+static_assert(kNoAllocScores * sizeof(double) == 2u * 1024u * 1024u, "the header documents a 2 MiB scratch array");
 static __device__ __align__(256) double g_noalloc_scores[kNoAllocScores];
 
+// Unique id of the calling thread's current CUDA context (cuCtxGetId, resolved
+// through the runtime's driver entry-point query so the library needs no link
+// against libcuda).  0 if the query is unavailable.
+unsigned long long current_context_id() {
+  using CtxGetCurrent = CUresult (*)(CUcontext*);
+  using CtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrent get_current = nullptr;
+  static CtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // Device address of g_noalloc_scores for the current device.  In host code the
-// array's name only stands for the symbol, so the address is looked up once per
-// device with cudaGetSymbolAddress and cached.
+// array's name only stands for the symbol, so the address is looked up with
+// cudaGetSymbolAddress, with that device current, once per device and context,
+// and cached.  The cache remembers the context's unique id: after a device
+// reset (a new primary context) the next call looks the address up again.
 rmm_status noalloc_scores(double** out) {
   static std::mutex mu;
   static double* cached[64] = {};
+  static unsigned long long cached_ctx[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(RMM_ERR_UNSUPPORTED, "device index %d out of range", dev);
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (cached[dev] == nullptr || ctx == 0 || cached_ctx[dev] != ctx) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scores);
     if (e != cudaSuccess || ptr == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(score scratch)");
     cached[dev] = static_cast<double*>(ptr);
+    cached_ctx[dev] = current_context_id();  // the lookup may have created the primary context
   }
   *out = cached[dev];
   return RMM_OK;
@@ -1243,10 +1315,12 @@ rmm_status rmm_select_noalloc(const rmm_bf16* A, int64_t batch, int64_t batch_st
   if (batch > 1 && batch_stride < (n - 1) * lda + d) return fail(RMM_ERR_INVALID_ARG, "batch_stride too small");
   if (causal != 0 && causal != 1) return fail(RMM_ERR_INVALID_ARG, "causal must be 0 or 1");
   if (d > kMaxSelectD) return fail(RMM_ERR_UNSUPPORTED, "d > %lld", static_cast<long long>(kMaxSelectD));
-  if (batch * d > kNoAllocScores)
+  // batch > kNoAllocScores / d  <=>  batch * d > kNoAllocScores, without forming the product
+  if (batch > kNoAllocScores / d)
     return fail(RMM_ERR_UNSUPPORTED,
-                "rmm_select_noalloc holds at most %lld scores (batch * d); got %lld -- use rmm_select with a workspace",
-                static_cast<long long>(kNoAllocScores), static_cast<long long>(batch * d));
+                "rmm_select_noalloc holds at most %lld scores (batch * d); got batch %lld x d %lld -- use rmm_select "
+                "with a workspace",
+                static_cast<long long>(kNoAllocScores), static_cast<long long>(batch), static_cast<long long>(d));
   if (n > kIntMax || batch > 65535) return fail(RMM_ERR_UNSUPPORTED, "n or batch too large");
   if (!aligned16(A) || (lda % 8) != 0 || (batch > 1 && (batch_stride % 8) != 0))
     return fail(RMM_ERR_UNSUPPORTED, "A must be 16-byte aligned with lda and batch_stride multiples of 8");

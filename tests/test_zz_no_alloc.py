@@ -86,3 +86,31 @@ def test_select_noalloc_rejects_sizes_beyond_its_scratch():
             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == UNSUPPORTED
     assert str(MAX_SCORES).encode() in L.rmm_last_error()
+
+
+def test_select_noalloc_back_to_back_calls_with_different_inputs():
+    """Two calls on one stream with no synchronisation between them, on inputs whose
+    top-k columns differ (the second input's column scales are reversed).  Both
+    calls share the scratch array, so the second call's column-score kernel must
+    not overwrite scores the first call's selection is still reading: each call's
+    index set must equal rmm_select's on its own input."""
+    L, fn = noalloc_fn()
+    g = synthetic.rng(4242)
+    n, d, rho = 512, 4096, 0.5
+    base = synthetic.outlier_activations(g, n, d, 1.5)
+    A1 = synthetic.to_bf16(base).cuda()
+    A2 = synthetic.to_bf16(base[:, ::-1].copy()).cuda()  # column j of A2 is column d-1-j of A1
+    ref1, _, _ = rmm.select(A1, rho)
+    ref2, _, _ = rmm.select(A2, rho)
+    torch.cuda.synchronize()
+    assert not torch.equal(ref1, ref2)
+    k = ref1.numel()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    out = [torch.full((k,), -1, dtype=torch.int32, device="cuda") for _ in range(4)]
+    for i, A in enumerate((A1, A2, A1, A2)):
+        st = fn(A.data_ptr(), 1, n * d, n, d, d, 0, rho, out[i].data_ptr(), None, stream)
+        assert st == 0, L.rmm_last_error()
+    torch.cuda.synchronize()
+    for i, ref in enumerate((ref1, ref2, ref1, ref2)):
+        assert torch.equal(out[i], ref), f"call {i} returned another input's index set"
+    assert rmm.device_error() == 0
