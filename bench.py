@@ -11,6 +11,12 @@ path at rho in {0.9, 0.7, 0.5}.
 
 `--impl reference` times the CPU oracle instead (a deliberately slow program:
 fp64 numpy on the host cores, a bounded sample of rows per step).
+
+`--profile CASE` runs one entry point ``--iters`` times on a named workload and
+exits (the command profiler captures run), e.g.
+    python bench.py --profile decode --n 32 --rho 0.5 --iters 3
+    python bench.py --profile prefill --proj gate_proj --rho 0.5
+    python bench.py --profile pv --rho 0.5 --heads 2 --seq 16384
 """
 from __future__ import annotations
 
@@ -18,7 +24,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -36,7 +41,11 @@ RHO_SWEEP = (0.9, 0.7)
 WORKLOAD = "llama3.1-8b prefill projections q/gate/up/down, n=4096 tokens, rho=0.5"
 GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm_pair.cuh", "input_adaptive_reduced_colnorm_b200/csrc/gemm.cuh",
                 "input_adaptive_reduced_colnorm_b200/csrc/ptx.cuh"]
-TRAFFIC_PROFILE = "profiles/gemm_packed_llama8b_gate.md"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one gate_proj product
+# launch at rho = 0.5 from one ncu capture, with the sha1 of the kernel sources it was
+# taken on; reported only while the sources are unchanged (the capture's summary is
+# in profiles/).
+GEMM_TRAFFIC = {"bytes": 158915584, "source_sha1": "b1d08603fb9c5b2752351bccc2067702dd0df5f1"}
 
 
 def parse_args():
@@ -48,6 +57,15 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the per-call timings of the other workloads")
     ap.add_argument("--cpu-rows", type=int, default=4096, help="rows per projection in the CPU-oracle sample")
+    ap.add_argument("--profile", default=None,
+                    choices=["prefill", "decode", "qk", "pv", "linear", "decode_attn", "attention", "int8", "mlp"],
+                    help="run one entry point --iters times on a named workload and exit (for profilers)")
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--rho", type=float, default=0.5)
+    ap.add_argument("--n", type=int, default=32, help="decode rows (--profile decode / int8)")
+    ap.add_argument("--proj", default="gate_proj", help="projection (--profile prefill)")
+    ap.add_argument("--heads", type=int, default=32)
+    ap.add_argument("--seq", type=int, default=None)
     return ap.parse_args()
 
 
@@ -153,17 +171,11 @@ def gemm_source_sha1():
 
 
 def profiled_traffic():
-    """DRAM bytes per packed-GEMM launch from the committed ncu summary, if the
-    kernel source is unchanged since that capture; else None."""
-    path = os.path.join(ROOT, TRAFFIC_PROFILE)
-    if not os.path.exists(path):
+    """DRAM bytes per product launch from the recorded ncu capture, while the kernel
+    sources are unchanged since that capture; else None."""
+    if GEMM_TRAFFIC.get("source_sha1") != gemm_source_sha1():
         return None
-    text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    s = re.search(r"source_sha1:\s*([0-9a-f]{40})", text)
-    if not m or not s or s.group(1) != gemm_source_sha1():
-        return None
-    return float(m.group(1))
+    return float(GEMM_TRAFFIC["bytes"])
 
 
 def measured_peaks():
@@ -172,6 +184,18 @@ def measured_peaks():
             return json.load(f), "measured"
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def cpu_threads():
@@ -213,8 +237,8 @@ def cpu_baseline(nrows):
     t0 = time.perf_counter()
     flops = oracle_step(host, rows, RHO_MAIN)
     dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-            "seconds": dt,
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+            "kind": "oracle", "seconds": dt,
             "sample": f"q/gate/up/down at rho={RHO_MAIN}: fp64 column norms and TopK over all {N_TOKENS} rows, "
                       f"reduced product for {nrows} of {N_TOKENS} rows per projection (kept FLOPs of those rows / "
                       f"wall time of the whole sample)"}
@@ -242,8 +266,8 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD, "n": N_TOKENS, "rho": RHO_MAIN, "projections": PROJ,
                        "sampled": "16 rows per projection for the product (see cpu_baseline.sample)"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "cpu_model": cpu_model(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -614,35 +638,58 @@ def run_ours(args):
         return max_over_ranks(e0.elapsed_time(e1) / steps)
 
     K, W = args.steps, args.warmup
-    # ---- main timed region: rho = 0.5 through the stage entry points, GEMM bracketed by events
+    # ---- main timed region: K steps through the public rmm_linear call at rho = 0.5
     for _ in range(W):
-        step_stages(RHO_MAIN)
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in bufs]
-           for _ in range(K)]
+        step_linear(RHO_MAIN)
     barrier()
     sampler = ClockSampler(local)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with sampler:
         e0.record(stream)
-        for s in range(K):
-            step_stages(RHO_MAIN, evs[s])
+        for _ in range(K):
+            step_linear(RHO_MAIN)
         e1.record(stream)
         barrier()
     ms_step = max_over_ranks(e0.elapsed_time(e1) / K)
-    gemm_ms = [statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(K)) for i in range(len(bufs))]
+
+    # ---- the dominant kernel: the same launches through the stage entry points (the
+    # kernels rmm_linear launches, in the same order, on the same stream), each product
+    # launch bracketed by CUDA events
+    for _ in range(W):
+        step_stages(RHO_MAIN)
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in bufs]
+           for _ in range(K)]
+    barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for s_ in range(K):
+        step_stages(RHO_MAIN, evs[s_])
+    s1.record(stream)
+    barrier()
+    ms_stages = max_over_ranks(s0.elapsed_time(s1) / K)
+    gemm_ms = [statistics.mean(evs[s_][i][0].elapsed_time(evs[s_][i][1]) for s_ in range(K)) for i in range(len(bufs))]
     gemm_ms = [max_over_ranks(x) for x in gemm_ms]
 
-    # ---- rho sweep and the rho = 1 dense path through rmm_linear
-    ms_rho = {RHO_MAIN: ms_step}
-    for rho in RHO_SWEEP:
-        ms_rho[rho] = timed(lambda: step_linear(rho), K, W)
-    ms_linear_main = timed(lambda: step_linear(RHO_MAIN), K, W)
-    ms_dense = timed(lambda: step_linear(1.0), K, W)
-
+    # ---- rho sweep on one path (rmm_linear at rho = 0.9, 0.7, 0.5 and the dense rho = 1
+    # path) and cuBLAS on the same shapes, in interleaved rounds so that every variant
+    # runs under the same clock and power state
     def step_cublas():
         for b in bufs:
             torch.matmul(b["A"], b["W"], out=b["Y"])
-    ms_cublas = timed(step_cublas, K, W)
+    variants = {"1.0": lambda: step_linear(1.0), "0.9": lambda: step_linear(0.9), "0.7": lambda: step_linear(0.7),
+                "0.5": lambda: step_linear(0.5), "cublas": step_cublas}
+    rounds = 5
+    per_round = max(1, K // rounds)
+    for fn in variants.values():
+        for _ in range(W):
+            fn()
+    sweep_ms = {key: 0.0 for key in variants}
+    for _ in range(rounds):
+        for key, fn in variants.items():
+            sweep_ms[key] += timed(fn, per_round, 0) / rounds
+    ms_rho = {float(r): sweep_ms[r] for r in ("0.9", "0.7", "0.5")}
+    ms_dense = sweep_ms["1.0"]
+    ms_cublas = sweep_ms["cublas"]
 
     # ---- end to end: host activations in, host outputs out, through rmm.linear.  Every
     # step copies each projection's activations in from pinned host memory and its
@@ -702,7 +749,9 @@ def run_ours(args):
     nbytes = step_bytes(RHO_MAIN)
     value = weak_scaled_value(world, flops, ms_step)
     peaks, peak_src = measured_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    # the product launches are timed inside a region of well under a second, so the
+    # burst figure (a short cuBLAS loop) is the matching peak, not the seconds-long one
+    peak = float(peaks["bf16_tflops"])
     gate = [i for i, b in enumerate(bufs) if b["name"] == "gate_proj"][0]
     b = bufs[gate]
     gate_flops = kept_flops(b["n"], b["d"], b["m"], RHO_MAIN)
@@ -721,13 +770,16 @@ def run_ours(args):
                                "gbs": world * step_bytes(r) / (ms_rho[r] * 1e-3) / 1e9,
                                "speedup_vs_rho1": ms_dense / ms_rho[r]} for r in (0.9, 0.7, 0.5)},
         "speedup_vs_rho1": {str(r): ms_dense / ms_rho[r] for r in (0.9, 0.7, 0.5)},
+        "rho_sweep_method": (f"rmm_linear at every rho and the dense rho = 1 path, cuBLAS beside them, {rounds} "
+                             f"interleaved rounds of {per_round} steps each"),
         "rho1": {"ms_per_step": ms_dense, "tflops": world * step_flops(1.0) / (ms_dense * 1e-3) / 1e12,
                  "cublas_ms_per_step": ms_cublas, "speedup_vs_cublas": ms_cublas / ms_dense},
-        "rmm_linear_ms_per_step_rho0.5": ms_linear_main,
+        "stage_chain_ms_per_step": ms_stages,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(),
-                     "kernel": "rmm_gemm_pair_kernel (CTA pairs, 256 x 256 tiles) on packed gate_proj operands (4096 x 14336, k=2048)",
-                     "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                     "kernel": "the reduced product of gate_proj (4096 x 14336, k=2048) at rho = 0.5",
+                     "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                     "timed": f"{K} launches, CUDA events around each on the launching stream",
                      "all_gemm_launches_tflops": all_gemm},
         "gemm_ms_per_launch": {x["name"]: gemm_ms[i] for i, x in enumerate(bufs)},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -746,8 +798,67 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ profiler cases
+def run_profile(args):
+    """One entry point, ``--iters`` calls on a named seeded workload, then exit: the
+    command that profiler captures run (head counts and sequence lengths can be
+    reduced so a capture holds a few GB on the device)."""
+    import numpy as np
+    import torch
+
+    from input_adaptive_reduced_colnorm_b200 import build as rmm_build
+    rmm_build.build()
+    import input_adaptive_reduced_colnorm_b200 as rmm
+    import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    case, rho = args.profile, args.rho
+    if case == "linear":
+        A, B = (t.to(dev) for t in synthetic.linear_small())
+        fn = lambda: rmm.linear(A, B, rho)
+    elif case == "prefill":
+        A, B = (t.to(dev) for t in synthetic.prefill_projection(args.proj))
+        fn = lambda: rmm.linear(A, B, rho)
+    elif case == "decode":
+        A, B = (t.to(dev) for t in synthetic.decode_gemv(args.n))
+        fn = lambda: rmm.linear(A, B, rho)
+    elif case == "int8":
+        x, _ = synthetic.decode_gemv(args.n, weight=False)
+        Wq, sc = synthetic.int8_weight(synthetic.rng(synthetic.seed_for(3) + 100), 8192, 28672)
+        x, Wq, sc = x.to(dev), Wq.to(dev), sc.to(dev)
+        fn = lambda: rmm.linear_int8(x, Wq, sc, rho)
+    elif case == "mlp":
+        X, Wg, Wu, Wd = (t.to(dev) for t in synthetic.mlp_block())
+        fn = lambda: rmm.mlp(X, Wg, Wu, Wd, rho, rho)
+    elif case == "qk":
+        hkv = max(1, args.heads // 4)
+        Q, K = (t.to(dev) for t in synthetic.qk_inputs(hq=args.heads, hkv=hkv, n=args.seq or 4096))
+        fn = lambda: rmm.qk(Q, K, rho, causal=True)
+    elif case == "attention":
+        hkv = max(1, args.heads // 4)
+        Q, K = synthetic.qk_inputs(hq=args.heads, hkv=hkv, n=args.seq or 4096)
+        V = synthetic.to_bf16(synthetic.rng(7).standard_normal(tuple(K.shape), dtype=np.float32))
+        Q, K, V = Q.to(dev), K.to(dev), V.to(dev)
+        fn = lambda: rmm.attention(Q, K, V, rho, causal=True, scale=0.088)
+    elif case == "decode_attn":
+        Q, Kt, P, V = synthetic.decode_attention_inputs_device(dev, nk=args.seq or 32768)
+        fn = lambda: (rmm.decode_qk(Q, Kt, rho, scale=0.088), rmm.decode_pv(P, V, rho))
+    else:  # pv
+        P, V = synthetic.pv_inputs_device(dev, heads=args.heads, n=args.seq or 16384)
+        fn = lambda: rmm.pv(P, V, rho, causal=True)
+    for _ in range(args.iters):
+        fn()
+    torch.cuda.synchronize(dev)
+    err = rmm.device_error()
+    print(f"{case}: {args.iters} calls done, device error word {err}")
+    return 0 if err == 0 else 1
+
+
 def main():
     args = parse_args()
+    if args.profile is not None:
+        return run_profile(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
