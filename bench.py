@@ -599,7 +599,7 @@ def run_ours(args):
 
     def step_stages(rho, ev=None):
         """One step through the stage entry points: select, gather_columns,
-        gather_rows, gemm_packed (the same kernels rmm_linear launches)."""
+        gather_rows, gemm_packed (the kernels rmm_linear launches)."""
         for i, b in enumerate(bufs):
             n, d, m = b["n"], b["d"], b["m"]
             k = k_of(rho, d)
@@ -777,7 +777,8 @@ def run_ours(args):
         "stage_chain_ms_per_step": ms_stages,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(),
-                     "kernel": "the reduced product of gate_proj (4096 x 14336, k=2048) at rho = 0.5",
+                     "kernel": "rmm_gemm_pair_kernel<false, false>: the reduced product of gate_proj (4096 x 14336, "
+                               "k=2048) at rho = 0.5 on the packed A[:, I] and B[I, :]",
                      "peak_source": f"bf16_tflops (burst) of {peak_src}",
                      "timed": f"{K} launches, CUDA events around each on the launching stream",
                      "all_gemm_launches_tflops": all_gemm},
@@ -785,7 +786,7 @@ def run_ours(args):
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
                 "streams": "copies in, kernels and copies out on three streams, overlapped across projections"},
-        "gpu_launches": 20 * K,
+        "gpu_launches": 20 * K,  # per projection: column scores, selection, A pack, B row pack, product
         "clocks": sampler.summary(),
     }
     if world == 1 and not args.no_workloads:

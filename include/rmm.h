@@ -127,8 +127,11 @@ rmm_status rmm_select_noalloc(const rmm_bf16* A, int64_t batch, int64_t batch_st
  *   Y   device bf16 [n][ldy], n x m output.
  *   idx_out  device int32 [k] or NULL: the index set used.
  * rho == 1 runs the dense product A.B (no scores, no selection, no pack).
+ * n > 128 reads the kept rows of B straight from B inside the tensor-core
+ * product (CTA pairs); 32 < n <= 128 packs them first (one-CTA tiles).
  * n <= 32 runs the decode path (a gathered GEMV-shaped kernel that streams only
- * the kept rows of B).  Limits: d <= 32768, n, m < 2^31. */
+ * the kept rows of B; the scores, the selection and x[:, I] come from one
+ * cluster launch when d <= 16384).  Limits: d <= 32768, n, m < 2^31. */
 size_t rmm_linear_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho);
 rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const rmm_bf16* B, int64_t m,
                       int64_t ldb, rmm_bf16* Y, int64_t ldy, double rho, int32_t* idx_out, void* ws, size_t ws_bytes,
@@ -137,8 +140,10 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
 /* ---------------------------------------------------------------- linear stages
  * The steps that follow the selection in rmm_linear, exposed so a caller can
  * run (or time) them on their own.  rmm_linear with rho < 1 is rmm_select's
- * kernels followed by exactly rmm_gather_columns, rmm_gather_rows and
- * rmm_gemm_packed; with rho = 1 it is rmm_gemm_packed on A and B themselves.
+ * kernels followed by exactly rmm_gather_columns and rmm_gemm_gathered for
+ * n > 128 rows, rmm_gather_columns, rmm_gather_rows and rmm_gemm_packed for
+ * 32 < n <= 128 (one-CTA tiles); with rho = 1 it is rmm_gemm_packed on A and B
+ * themselves.
  *
  * rmm_gather_columns: A_pack[i, t] = A[i, idx[t]] for t < k and 0 for
  * k <= t < ld_pack -- the gathered A[:, I] of "Core Approach", stored K-major.
@@ -152,13 +157,21 @@ rmm_status rmm_linear(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, cons
  * rmm_gemm_packed: Y = A_pack[:, :k] . B_pack[:k, :] on the tensor cores
  * (tcgen05, fp32 accumulation in tensor memory, bf16 output).
  *   A_pack [n][lda] (lda >= k), B_pack [k][ldb] (ldb >= m), Y [n][ldy].
- * None of the three needs a workspace. */
+ * rmm_gemm_gathered: Y = A_pack[:, :k] . B[idx[0:k], :] -- the reduced product
+ * of "Core Approach" with the kept rows of B read through the index set
+ * straight from B (no packed copy), on pairs of CTAs (tcgen05 cta_group::2).
+ *   A_pack [n][lda] (lda >= k), B [d][ldb] (ldb >= m), idx device int32 [k]
+ *   with entries in [0, d) (not checked on the host), Y [n][ldy].  The result
+ *   equals rmm_gemm_packed on rmm_gather_rows' copy, bit for bit.
+ * None of the four needs a workspace. */
 rmm_status rmm_gather_columns(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int32_t* idx, int64_t k,
                               rmm_bf16* A_pack, int64_t ld_pack, rmm_stream stream);
 rmm_status rmm_gather_rows(const rmm_bf16* B, int64_t d, int64_t m, int64_t ldb, const int32_t* idx, int64_t k,
                            rmm_bf16* B_pack, int64_t ld_pack, rmm_stream stream);
 rmm_status rmm_gemm_packed(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t lda, const rmm_bf16* B_pack,
                            int64_t m, int64_t ldb, rmm_bf16* Y, int64_t ldy, rmm_stream stream);
+rmm_status rmm_gemm_gathered(const rmm_bf16* A_pack, int64_t n, int64_t k, int64_t lda, const rmm_bf16* B, int64_t d,
+                             int64_t m, int64_t ldb, const int32_t* idx, rmm_bf16* Y, int64_t ldy, rmm_stream stream);
 
 /* ---------------------------------------------------------------- attention scores
  * rmm_qk: per query head h, I_h = TopK of the column norms of Q_h over its nq

@@ -13,7 +13,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["lib", "rmm_k", "select", "linear", "gather_columns", "gather_rows", "gemm_packed", "qk", "pv", "RMMError", "device_error", "library_path"]
+__all__ = ["lib", "rmm_k", "select", "linear", "gather_columns", "gather_rows", "gemm_packed", "gemm_gathered", "qk", "pv",
+           "RMMError", "device_error", "library_path"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -47,6 +48,8 @@ _SIGNATURES = {
     "rmm_gather_columns": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_i64, _c_p]),
     "rmm_gather_rows": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_p, _c_i64, _c_p]),
     "rmm_gemm_packed": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_p]),
+    "rmm_gemm_gathered": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64,
+                                   _c_p]),
     "rmm_qk_workspace_bytes": (_c_size, [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_dbl]),
     "rmm_qk": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_float, _c_dbl,
                         _c_p, _c_p, _c_size, _c_p]),
@@ -226,6 +229,21 @@ def gemm_packed(A_pack, k, B_pack, m, out=None):
         out = torch.empty((n, m), dtype=torch.bfloat16, device=A_pack.device)
     _check(lib().rmm_gemm_packed(_ptr(A_pack), n, int(k), A_pack.stride(0), _ptr(B_pack), int(m), B_pack.stride(0),
                                  _ptr(out), out.stride(0), _stream(A_pack.device)))
+    return out
+
+
+def gemm_gathered(A_pack, k, B, idx, out=None):
+    """Y = A_pack[:, :k] . B[idx[:k], :] with the kept rows of B read through the index set."""
+    import torch
+    _require(A_pack, "A_pack", torch.bfloat16, 2)
+    _require(B, "B", torch.bfloat16, 2)
+    _require(idx, "idx", torch.int32, 1)
+    n = A_pack.shape[0]
+    d, m = B.shape
+    if out is None:
+        out = torch.empty((n, m), dtype=torch.bfloat16, device=A_pack.device)
+    _check(lib().rmm_gemm_gathered(_ptr(A_pack), n, int(k), A_pack.stride(0), _ptr(B), d, m, B.stride(0), _ptr(idx),
+                                   _ptr(out), out.stride(0), _stream(A_pack.device)))
     return out
 
 

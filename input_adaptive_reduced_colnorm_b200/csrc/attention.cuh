@@ -82,6 +82,12 @@ __global__ void attn_exp2_probe_kernel(const float* __restrict__ x, float* __res
   }
 }
 
+// The softmax's reference maximum of a row moves only when the row's maximum
+// exceeds it by more than this (log2 units), so the unnormalised weights stay
+// below 2^8 = 256 (exact range for fp32 sums and bf16 P) and O is rescaled only
+// on such jumps.  The result is the same softmax: O and l share the reference.
+constexpr float kAttnRescaleLog2 = 8.f;
+
 // Visible key blocks of the query tile starting at row m0.
 __device__ __forceinline__ int attn_key_blocks(const AttnParams& p, int m0) {
   const int all = (p.nk + kAttnTile - 1) / kAttnTile;
@@ -314,50 +320,64 @@ __global__ void __launch_bounds__(320, 1)
       const int64_t key0 = static_cast<int64_t>(j) * kAttnTile;
       // every key of the block visible to this row: no masking work
       const bool full = (key0 + kAttnTile - 1 <= last_key) && (key0 + kAttnTile <= p.nk);
-      // pass 1: the row maximum of the block (scaled, masked)
-      // tcgen05.ld is warp-collective (.sync.aligned): every lane executes the same
-      // loads, outside any branch on row-dependent values; only the arithmetic on
-      // the loaded values depends on whether this row sees the whole block
-      float mx = -INFINITY;
+      // pass 1: the row maximum of the block (scaled, masked), eight independent
+      // chains.  tcgen05.ld is warp-collective (.sync.aligned): every lane
+      // executes the same loads, outside any branch on row-dependent values; only
+      // the arithmetic on the loaded values depends on whether this row sees the
+      // whole block
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
       const bool fast = full && p.scale_log2 > 0.f;
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(s_col + static_cast<uint32_t>(c * 32), v);
+      for (int hh = 0; hh < 2; ++hh) {  // half a block per read: two loads, one wait
+        uint32_t v[2][32];
+        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64), v[0]);
+        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64 + 32), v[1]);
         tmem_ld_wait();
         if (fast) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+          for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e >> 5][e & 31]));
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int64_t key = key0 + c * 32 + e;
-            if (key < p.nk && key <= last_key) mx = fmaxf(mx, __uint_as_float(v[e]) * p.scale_log2);
+          for (int e = 0; e < 64; ++e) {
+            const int64_t key = key0 + hh * 64 + e;
+            if (key < p.nk && key <= last_key)
+              mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e >> 5][e & 31]) * p.scale_log2);
           }
         }
       }
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       if (fast) mx *= p.scale_log2;
-      const float m_new = fmaxf(m_run, mx);
+      // the reference maximum moves only when the row's maximum grows by more than
+      // kAttnRescaleLog2 (log2 units): the weights exp2(s - m) then stay below 2^8,
+      // and O and l are rescaled rarely instead of at almost every block
+      const bool grow = (m_run == -INFINITY) || (mx > m_run + kAttnRescaleLog2);
+      const float m_new = grow ? fmaxf(m_run, mx) : m_run;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float corr = attn_exp2(m_run - m_use);  // 0 for the first block
+      const float corr = grow ? attn_exp2(m_run - m_use) : 1.f;  // 0 for the first block
       // pass 2: P = exp2(s * scale_log2 - m) packed as bf16 pairs into the first 64
-      // columns of S; chunks 2h, 2h+1 (keys 64h .. 64h+63) become columns 32h .. 32h+31,
-      // which lie in S columns already read
-      float sum = 0.f;
+      // columns of S (keys 64h .. 64h+63 become columns 32h .. 32h+31, already read)
+      float sum8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
+        uint32_t vv[2][32];  // half a block per read: two loads, one wait
+        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64), vv[0]);
+        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64 + 32), vv[1]);
+        tmem_ld_wait();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * hh + cc;
-          uint32_t v[32];
-          tmem_ld32(s_col + static_cast<uint32_t>(c * 32), v);
-          tmem_ld_wait();
+          const uint32_t (&v)[32] = vv[cc];
           // even keys on the FMA pipe, odd keys on the special-function unit
           if (full) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const float x0 = attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use));
               const float x1 = attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use));
-              sum += x0 + x1;
+              sum8[e & 7] += x0 + x1;
               const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
               pk[cc * 16 + e] = *reinterpret_cast<const uint32_t*>(&t2);
             }
@@ -365,12 +385,13 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int64_t ka = key0 + c * 32 + 2 * e;
-              const float x0 =
-                  (ka < p.nk && ka <= last_key) ? attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use)) : 0.f;
-              const float x1 =
-                  (ka + 1 < p.nk && ka + 1 <= last_key) ? attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use))
-                                                        : 0.f;
-              sum += x0 + x1;
+              const float x0 = (ka < p.nk && ka <= last_key)
+                                   ? attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use))
+                                   : 0.f;
+              const float x1 = (ka + 1 < p.nk && ka + 1 <= last_key)
+                                   ? attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use))
+                                   : 0.f;
+              sum8[e & 7] += x0 + x1;
               const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
               pk[cc * 16 + e] = *reinterpret_cast<const uint32_t*>(&t2);
             }
@@ -378,17 +399,19 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_st32(s_col + static_cast<uint32_t>(hh * 32), pk);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * corr + sum;
       m_run = m_new;
-      // O *= corr where some row's maximum grew; PV(j-1) is complete (it was issued before S(j))
+      // O *= corr where some row's reference maximum moved; PV(j-1) is complete (it
+      // was issued before S(j))
       if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
         for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(o_col + static_cast<uint32_t>(c * 32), v);
+          uint32_t o[32];
+          tmem_ld32(o_col + static_cast<uint32_t>(c * 32), o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
-          tmem_st32(o_col + static_cast<uint32_t>(c * 32), v);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+          tmem_st32(o_col + static_cast<uint32_t>(c * 32), o);
         }
       }
       tmem_st_wait();

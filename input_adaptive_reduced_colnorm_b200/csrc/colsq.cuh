@@ -256,8 +256,6 @@ __global__ void __launch_bounds__(kColsqThreads, 2)
       uint4 v[S::RPT];
 #pragma unroll
       for (int u = 0; u < S::RPT; ++u) v[u] = lds_v4(base + stage * kColsqTileBytes + u * S::TY * W * 2);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
       const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
       float a32[8];
 #pragma unroll
@@ -287,6 +285,11 @@ __global__ void __launch_bounds__(kColsqThreads, 2)
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
+      // release the stage only once its values are consumed, with the warp's
+      // reads ordered before the producer's next TMA write into it
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
     }
   }
 
@@ -332,23 +335,23 @@ namespace rmm {
 // order.  Non-causal only.
 constexpr int kColsqShortMaxRows = 32;
 
-__global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {
-  wait_prior_kernels();
-  const int64_t b = blockIdx.y;
-  const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
-  if (col0 >= p.d) return;
-  const uint16_t* A = p.A + b * p.batch_stride + col0;
-  const bool full = col0 + 8 <= p.d;
-  double acc[8];
+// Sums of squares of columns [col0, col0 + 8) of an n-row matrix (n may be
+// anything; used for n <= 32): rows summed 4 at a time in fp32 (exact bf16
+// squares) and folded into fp64, in row order.  Columns at or past d read as 0.
+// The decode selection kernel computes its scores with this same function, so
+// its keys are bit-identical to colsq_short_kernel's.
+__device__ __forceinline__ void colsq_short_cols8(const uint16_t* A, int64_t lda, int64_t n, int64_t col0, int64_t d,
+                                                  double (&acc)[8]) {
+  const bool full = col0 + 8 <= d;
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-  for (int64_t r0 = 0; r0 < p.n; r0 += 8) {
+  for (int64_t r0 = 0; r0 < n; r0 += 8) {
     uint32_t w[8][4];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       w[u][0] = w[u][1] = w[u][2] = w[u][3] = 0u;
-      if (r0 + u < p.n) {
-        const uint16_t* src = A + (r0 + u) * p.lda;
+      if (r0 + u < n) {
+        const uint16_t* src = A + (r0 + u) * lda + col0;
         if (full) {
           const uint4 v = ldg_nc_v4(src);
           w[u][0] = v.x;
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {
           w[u][3] = v.w;
         } else {
           for (int e = 0; e < 8; ++e)
-            if (col0 + e < p.d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
+            if (col0 + e < d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
         }
       }
     }
@@ -378,6 +381,15 @@ __global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {
       for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
     }
   }
+}
+
+__global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {
+  wait_prior_kernels();
+  const int64_t b = blockIdx.y;
+  const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+  if (col0 >= p.d) return;
+  double acc[8];
+  colsq_short_cols8(p.A + b * p.batch_stride, p.lda, p.n, col0, p.d, acc);
   double* out = p.colsq + b * p.d + col0;
 #pragma unroll
   for (int e = 0; e < 8; ++e)

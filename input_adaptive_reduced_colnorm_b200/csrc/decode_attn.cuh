@@ -222,8 +222,6 @@ __global__ void __launch_bounds__(288) decode_qk_staged_kernel(const DecodeQkPar
 #pragma unroll
     for (int q = 0; q < kDqkRowsPerStage; ++q)
       v[q] = (q < nr) ? lds_v4(base + s * kDqkStageBytes + q * kDqkRowBytes) : make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
     for (int q = 0; q < kDqkRowsPerStage; ++q) {
       if (q >= nr) break;
@@ -235,6 +233,11 @@ __global__ void __launch_bounds__(288) decode_qk_staged_kernel(const DecodeQkPar
         for (int h = 0; h < G; ++h) acc[h][e] = fmaf(qs[h][r0 + q], x, acc[h][e]);
       }
     }
+    // release the stage only once its values are consumed, with the warp's reads
+    // ordered before the producer's next bulk copy into it
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
   const int64_t jt = j0 + threadIdx.x * 8;
   if (jt >= p.nk) return;

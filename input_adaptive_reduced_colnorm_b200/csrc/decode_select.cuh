@@ -1,0 +1,331 @@
+// Decode-time selection in one launch: the column scores q_j = sum_i x[i, j]^2
+// of a short activation matrix x (n <= 32 rows), the TopK index set I of the
+// k = ceil(rho d) largest (lower index on ties, ascending), and the packed
+// activations x[:, I] ("Algorithm Deep-Dive: RMM", Core Approach: s_j =
+// ||A[:, j]||_2, keep the TopK-largest; the reduced product then reads x[:, I]).
+//
+// At decode sizes each of the three steps is a latency-bound launch of a few
+// microseconds, and one CTA selecting over d = 8192 keys is issue-bound, so the
+// work is spread over one cluster of C = ceil(d / 2048) CTAs (C <= 8):
+//   * CTA r owns columns [2048 r, 2048 (r + 1)); each of its 256 threads owns 8
+//     consecutive columns and computes their fp64 scores with the arithmetic of
+//     the short-matrix column-score kernel (bit-identical keys);
+//   * the k-th largest key is found by an MSB-first radix select over the
+//     64-bit key patterns (non-negative doubles order like their bits): leading
+//     bits shared by every key are skipped (cluster-wide AND / OR), each pass
+//     resolves 8 bits with per-warp histograms merged per CTA and then across
+//     the cluster through distributed shared memory, one cluster barrier per
+//     pass; when the bucket holding the k-th key has become small, one more
+//     AND / OR of its members skips their shared bits, so exact ties (squares
+//     of a single bf16 row) end the passes at once;
+//   * the compaction takes every key above the threshold and the lowest-index
+//     keys equal to it, in index order: counts are exchanged once across the
+//     cluster (CTA order is column order), then two block scans give each
+//     thread its positions; the thread writes I and, for its kept columns,
+//     x[:, I] (zero-padded to the packed row length).
+// Every count is an integer, so the result does not depend on atomic order.
+#pragma once
+#include "ptx.cuh"
+#include "colsq.cuh"
+#include "select.cuh"
+
+namespace rmm {
+
+struct DecodeSelParams {
+  const uint16_t* x;  // bf16 [n][ldx]
+  int64_t ldx;
+  int n;              // 1..32
+  int d;              // 1..kDecSelMaxD
+  int k;              // 1..d
+  int32_t* idx;       // [k]
+  uint16_t* xpack;    // [n][ld_pack] or nullptr: x[:, I], columns [k, ld_pack) zeroed
+  int64_t ld_pack;
+};
+
+constexpr int kDecSelThreads = 256;
+constexpr int kDecSelCols = kDecSelThreads * 8;  // columns per CTA
+constexpr int kDecSelMaxCtas = 8;                // portable cluster size
+constexpr int kDecSelMaxD = kDecSelCols * kDecSelMaxCtas;
+constexpr int kDecSelMaxRows = 32;
+constexpr int kDecSelSkipBelow = 64;             // bucket size at which shared bits are skipped again
+
+__device__ __forceinline__ uint64_t ld_shared_cluster_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// AND and OR of v over the whole cluster.  Each CTA stages its block result in
+// `slot` (two words), the cluster barrier publishes them, lanes q < C of warp 0
+// read CTA q's pair, and the combined result is broadcast through `res`.  No
+// CTA rewrites `slot` before every CTA has passed the next cluster barrier.
+__device__ __forceinline__ void decsel_cluster_andor(uint64_t& a, uint64_t& o, uint64_t* s_warp_and,
+                                                     uint64_t* s_warp_or, uint64_t* slot, uint64_t* res, int C) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    a &= __shfl_xor_sync(0xffffffffu, a, off);
+    o |= __shfl_xor_sync(0xffffffffu, o, off);
+  }
+  if (lane == 0) {
+    s_warp_and[warp] = a;
+    s_warp_or[warp] = o;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint64_t ba = ~0ull, bo = 0ull;
+    for (int w = 0; w < kDecSelThreads / 32; ++w) {
+      ba &= s_warp_and[w];
+      bo |= s_warp_or[w];
+    }
+    slot[0] = ba;
+    slot[1] = bo;
+  }
+  cluster_sync();
+  if (warp == 0) {
+    uint64_t ra = ~0ull, ro = 0ull;
+    if (lane < C) {
+      const uint32_t base = smem_u32(slot);
+      ra = ld_shared_cluster_u64(map_shared_rank(base, static_cast<uint32_t>(lane)));
+      ro = ld_shared_cluster_u64(map_shared_rank(base + 8, static_cast<uint32_t>(lane)));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ra &= __shfl_xor_sync(0xffffffffu, ra, off);
+      ro |= __shfl_xor_sync(0xffffffffu, ro, off);
+    }
+    if (lane == 0) {
+      res[0] = ra;
+      res[1] = ro;
+    }
+  }
+  __syncthreads();
+  a = res[0];
+  o = res[1];
+}
+
+__global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const DecodeSelParams p) {
+  __shared__ uint32_t whist[kDecSelThreads / 32][256];
+  __shared__ uint32_t hist[2][256];
+  __shared__ uint64_t s_wand[kDecSelThreads / 32], s_wor[kDecSelThreads / 32];
+  __shared__ uint64_t s_andor[2], s_andor_res[2];
+  __shared__ int s_warp[32];
+  __shared__ int s_total;
+  __shared__ int s_digit, s_above, s_cnt;
+  __shared__ int s_counts[2];  // this CTA's keys above the threshold / equal to it (read by the cluster)
+  __shared__ int s_sel_base, s_eq_before;
+
+  wait_prior_kernels();
+  const int C = static_cast<int>(gridDim.x);  // the grid is one cluster
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t col0 = static_cast<int64_t>(rank) * kDecSelCols + tid * 8;
+
+  // ---- scores (fp64, bit-identical to colsq_short_kernel) and their key patterns
+  uint64_t key[8];
+  uint32_t valid = 0;
+  {
+    double acc[8];
+    if (col0 < p.d) {
+      colsq_short_cols8(p.x, p.ldx, p.n, col0, p.d, acc);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      key[e] = static_cast<uint64_t>(__double_as_longlong(acc[e]));
+      if (col0 + e < p.d) valid |= 1u << e;
+    }
+  }
+
+  // ---- radix select of the k-th largest key
+  uint64_t pre = 0, msk = 0;
+  int need = p.k;
+  bool take = (p.k == p.d);
+  int cursor = 0;  // bits [0, cursor) of the key are unresolved
+  {
+    uint64_t a = ~0ull, o = 0ull;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if ((valid >> e) & 1u) {
+        a &= key[e];
+        o |= key[e];
+      }
+    decsel_cluster_andor(a, o, s_wand, s_wor, s_andor, s_andor_res, C);
+    const uint64_t differ = a ^ o;
+    if (!take) {
+      if (differ == 0ull) {  // every key is the same: the lower indices win
+        pre = a;
+        msk = ~0ull;
+      } else {
+        const int top = 63 - __clzll(static_cast<long long>(differ));
+        msk = (top == 63) ? 0ull : (~0ull << (top + 1));
+        pre = a & msk;
+        cursor = top + 1;
+      }
+    }
+  }
+  int pass = 0;
+  while (!take && cursor > 0) {
+    const int width = cursor >= 8 ? 8 : cursor;
+    const int shift = cursor - width;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (((valid >> e) & 1u) && (key[e] & msk) == pre)
+        atomicAdd(&whist[warp][static_cast<uint32_t>(key[e] >> shift) & dmask], 1u);
+    __syncthreads();
+    uint32_t c = 0;
+#pragma unroll
+    for (int w = 0; w < kDecSelThreads / 32; ++w) c += whist[w][tid];
+    uint32_t* hb = hist[pass & 1];
+    hb[tid] = c;
+    cluster_sync();  // every CTA's histogram of this pass is visible (and the one two passes back is no longer read)
+    // thread t takes digit 255 - t, so the exclusive scan in thread order counts the larger digits
+    const int bin = 255 - tid;
+    uint32_t cnt = 0;
+    const uint32_t haddr = smem_u32(hb + bin);
+    for (int q = 0; q < C; ++q) cnt += ld_shared_cluster_u32(map_shared_rank(haddr, static_cast<uint32_t>(q)));
+    const int above = block_exclusive_scan<kDecSelThreads>(static_cast<int>(cnt), s_warp, &s_total);
+    if (bin <= static_cast<int>(dmask) && above < need && need <= above + static_cast<int>(cnt)) {
+      s_digit = bin;
+      s_above = above;
+      s_cnt = static_cast<int>(cnt);
+    }
+    __syncthreads();
+    need -= s_above;
+    pre |= static_cast<uint64_t>(s_digit) << shift;
+    msk |= static_cast<uint64_t>(dmask) << shift;
+    cursor = shift;
+    const int bucket = s_cnt;
+    if (bucket == need) take = true;
+    ++pass;
+    if (!take && cursor > 0 && bucket <= kDecSelSkipBelow) {
+      // a small bucket: skip the bits its members share (all of them for exact ties)
+      uint64_t a = ~0ull, o = 0ull;
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (((valid >> e) & 1u) && (key[e] & msk) == pre) {
+          a &= key[e];
+          o |= key[e];
+        }
+      __syncthreads();  // every thread has read the scan results of this pass
+      decsel_cluster_andor(a, o, s_wand, s_wor, s_andor, s_andor_res, C);
+      const uint64_t open = (cursor >= 64) ? ~0ull : ((1ull << cursor) - 1ull);
+      const uint64_t dl = (a ^ o) & open;
+      if (dl == 0ull) {
+        pre |= a & open;
+        msk = ~0ull;
+        cursor = 0;
+      } else {
+        const int top = 63 - __clzll(static_cast<long long>(dl));
+        const uint64_t shared = open & ~((top == 63) ? ~0ull : ((1ull << (top + 1)) - 1ull));
+        pre |= a & shared;
+        msk |= shared;
+        cursor = top + 1;
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- classify: above the threshold, or equal to it
+  uint32_t gt = 0, eq = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if (!((valid >> e) & 1u)) continue;
+    const uint64_t km = key[e] & msk;
+    if (km > pre) gt |= 1u << e;
+    else if (km == pre) eq |= 1u << e;
+  }
+  // this CTA's counts, exchanged across the cluster (column order = CTA order)
+  const int eq_rank = block_exclusive_scan<kDecSelThreads>(__popc(eq), s_warp, &s_total);
+  const int eq_cta = s_total;
+  const int gt_rank = block_exclusive_scan<kDecSelThreads>(__popc(gt), s_warp, &s_total);
+  (void)gt_rank;
+  const int gt_cta = s_total;
+  if (tid == 0) {
+    s_counts[0] = gt_cta;
+    s_counts[1] = eq_cta;
+  }
+  cluster_sync();
+  if (tid == 0) {
+    int sel_before = 0, eq_before = 0;
+    const uint32_t base = smem_u32(s_counts);
+    for (int q = 0; q < rank; ++q) {
+      const int g = static_cast<int>(ld_shared_cluster_u32(map_shared_rank(base, static_cast<uint32_t>(q))));
+      const int e = static_cast<int>(ld_shared_cluster_u32(map_shared_rank(base + 4, static_cast<uint32_t>(q))));
+      int taken = take ? e : need - eq_before;
+      taken = taken < 0 ? 0 : (taken > e ? e : taken);
+      sel_before += g + taken;
+      eq_before += e;
+    }
+    s_sel_base = sel_before;
+    s_eq_before = eq_before;
+  }
+  cluster_sync();  // no CTA reads another's shared memory past this point
+  uint32_t sel = gt;
+  {
+    int r = s_eq_before + eq_rank;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if ((eq >> e) & 1u) {
+        if (take || r < need) sel |= 1u << e;
+        ++r;
+      }
+  }
+  const int pos0 = s_sel_base + block_exclusive_scan<kDecSelThreads>(__popc(sel), s_warp, &s_total);
+  {
+    int pos = pos0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if ((sel >> e) & 1u) p.idx[pos++] = static_cast<int32_t>(col0 + e);
+  }
+  if (p.xpack != nullptr) {
+    if (sel != 0u) {
+      // eight rows' loads are issued before any of their stores, so each batch
+      // costs one round trip instead of eight
+      const bool full = col0 + 8 <= p.d;
+      for (int r0 = 0; r0 < p.n; r0 += 8) {
+        uint32_t w[8][4];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          w[u][0] = w[u][1] = w[u][2] = w[u][3] = 0u;
+          if (r0 + u < p.n) {
+            const uint16_t* src = p.x + static_cast<int64_t>(r0 + u) * p.ldx + col0;
+            if (full) {
+              const uint4 v = ldg_nc_v4(src);
+              w[u][0] = v.x;
+              w[u][1] = v.y;
+              w[u][2] = v.z;
+              w[u][3] = v.w;
+            } else {
+              for (int e = 0; e < 8; ++e)
+                if (col0 + e < p.d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (r0 + u >= p.n) break;
+          uint16_t* dst = p.xpack + static_cast<int64_t>(r0 + u) * p.ld_pack;
+          int pos = pos0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if ((sel >> e) & 1u) dst[pos++] = static_cast<uint16_t>(w[u][e >> 1] >> (16 * (e & 1)));
+        }
+      }
+    }
+    if (rank == C - 1 && tid < p.n)
+      for (int64_t t = p.k; t < p.ld_pack; ++t) p.xpack[static_cast<int64_t>(tid) * p.ld_pack + t] = 0;
+  }
+}
+
+}  // namespace rmm

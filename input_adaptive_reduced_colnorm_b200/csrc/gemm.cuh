@@ -65,6 +65,12 @@ struct GemmParams {
   // narrow last wave (MN-major B only): the last tail_tiles tiles are cut into
   // tail_split pieces of BN / tail_split (>= 64) columns; 0 / 1 = no cut
   int tail_tiles, tail_split;
+  // gathered B (CTA-pair kernel only): the kept rows B[I[t], :] are read straight
+  // from the weights through the index set instead of from a packed copy
+  const uint16_t* gw0;   // [d][gldw] bf16 (gate weights with SWIGLU)
+  const uint16_t* gw1;   // up weights (SWIGLU), else unused
+  int64_t gldw;
+  const int32_t* gidx;   // [k] ascending kept rows
   // test hook (0 in every product call): 1 makes the producer, once the stage
   // ring is full, wait on a barrier that nothing arrives on, with a 1 ms limit,
   // so that its bounded wait runs out and the kernel takes its timeout path

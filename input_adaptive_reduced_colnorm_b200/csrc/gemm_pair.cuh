@@ -28,6 +28,20 @@
 // gate (columns 0-127) and up (128-255) for its rows; the epilogue writes
 // H = SiLU(gate) * up (128 columns per 256-wide tile, bf16).  A narrow piece of
 // width w holds gate in columns [0, w/2) and up in [w/2, w).
+// GATHER (the reduced product without a packed copy of B[I, :]): each CTA's B
+// half comes straight from the kept rows of the weights, B[I[t], :] for the 64
+// kept indices t of a k-block, read through the index set by four more warps
+// (warps 6-9, 320 threads per CTA).  A kept row contributes one contiguous
+// 256-byte run (128 columns) per CTA and k-block; the warps copy the runs with
+// 16-byte cp.async straight into the 128-byte-swizzled MN-major stage (a TMA
+// copy per row or per four rows stages only ~7-8 B/clk/SM on B200, 16-byte
+// cp.async ~35, and the pair needs ~22 B/clk/SM of B at full tensor rate).
+// Each warp keeps two k-blocks of copies in flight; when a k-block has landed
+// its lanes fence the async proxy and lane 0 arrives, with cluster-scope
+// release, on the even CTA's full barrier, which then counts the A bytes of
+// both CTAs (TMA) and the eight B warps of the pair.  The MMA thread waits on
+// it with cluster-scope acquire.  Kept indices t >= k and columns past N read
+// as zeros.
 // Work split as in the one-CTA kernel, with pairs as the workers: whole tiles
 // round-robin, then the tiles of a partial last wave cut into two 256 x 128
 // pieces.  Every wait is bounded; the CTAs meet at a cluster barrier before
@@ -48,6 +62,18 @@ struct PairCfg {
   static_assert(8 * (2 * STAGES + 5) + 8 <= 256, "barrier area");
 };
 
+constexpr int kPairGatherWarps = 4;  // B producer warps per CTA with GATHER (warps 6-9)
+constexpr int kPairGatherLag = 2;    // k-blocks of copies a B warp keeps in flight before arriving
+
+__device__ __forceinline__ void pair_cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void pair_cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void pair_cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Pair tile order: batch item, then N tile, then 256-row M tile fastest.
 __device__ __forceinline__ void pair_tile_coords(const GemmParams& p, int tile, int& b, int& m0, int& nt) {
   const int per_b = p.m_tiles * p.n_tiles;
@@ -57,8 +83,8 @@ __device__ __forceinline__ void pair_tile_coords(const GemmParams& p, int tile, 
   m0 = (r - nt * p.m_tiles) * 256;
 }
 
-template <bool SWIGLU>
-__global__ void __launch_bounds__(192, 1)
+template <bool SWIGLU, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     rmm_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmO,
                          const GemmParams p) {
@@ -83,7 +109,8 @@ __global__ void __launch_bounds__(192, 1)
   const int npairs = static_cast<int>(gridDim.x >> 1);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // GATHER: the A bytes of both CTAs (one expect_tx arrival) and the B warps of both CTAs
+      mbar_init(&full[s], GATHER ? 1 + 2 * kPairGatherWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -94,8 +121,8 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-    if (SWIGLU) prefetch_tensormap(&tmB2);
+    if (!GATHER) prefetch_tensormap(&tmB);
+    if (SWIGLU && !GATHER) prefetch_tensormap(&tmB2);
     prefetch_tensormap(&tmO);
   }
   if (warp == 1) {
@@ -129,7 +156,7 @@ __global__ void __launch_bounds__(192, 1)
         const int nb = SWIGLU ? nt * 128 + wk.n_off / 2 : nt * 256 + wk.n_off + static_cast<int>(rank) * half;
         const CUtensorMap* tb = (SWIGLU && rank == 1) ? &tmB2 : &tmB;
         const int64_t brow0 = gemm_b_row_base(p, b);
-        const uint32_t pair_bytes = 2u * static_cast<uint32_t>(C::A_BYTES + half * 64 * 2);
+        const uint32_t pair_bytes = 2u * static_cast<uint32_t>(C::A_BYTES + (GATHER ? 0 : half * 64 * 2));
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer)) {
             ok = false;
@@ -138,9 +165,10 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t bar = full_even + 8u * static_cast<uint32_t>(stage);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], pair_bytes);
           tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * 64, a_row);
-          for (int j = 0; j < half / 64; ++j)
-            tma_load_2d_pair(sB + stage * C::B_BYTES + j * 8192, tb, bar, nb + j * 64,
-                             static_cast<int32_t>(brow0 + kb * 64));
+          if (!GATHER)
+            for (int j = 0; j < half / 64; ++j)
+              tma_load_2d_pair(sB + stage * C::B_BYTES + j * 8192, tb, bar, nb + j * 64,
+                               static_cast<int32_t>(brow0 + kb * 64));
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -179,7 +207,8 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t idesc = make_idesc_bf16(256, wk.w, 0, 1);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma)) {
+          // GATHER: the B warps of the odd CTA arrive with cluster-scope release
+          if (!mbar_wait(&full[stage], phase, abort_flag, kDevErrTimeoutMma, 0, GATHER)) {
             ok = false;
             break;
           }
@@ -210,6 +239,97 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
+  } else if (GATHER && warp >= 6) {
+    // ------------------------------------------------------------ gathered B (both CTAs)
+    // warp g copies kept rows 16g .. 16g+15 of each k-block: a row's run is cpr
+    // 16-byte chunks (cpr = 16, or 8 for a 64-column half), rpi = 32 / cpr rows
+    // per warp instruction; each lane holds the row numbers of its rows for the
+    // current and the next k-block (loaded one k-block ahead, no shuffles).
+    const int g = warp - 6;
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0;
+    bool ok = true;
+    int rows_next[8];
+    auto load_rows = [&](int kb, int rpi, int (&dst)[8]) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int t = kb * 64 + g * 16 + j * rpi + lane / (32 / rpi);
+        dst[j] = (j * rpi < 16 && t < p.k) ? __ldg(p.gidx + t) : -1;
+      }
+    };
+    GemmWork wk;
+    int cur_rpi = 0;
+    for (int it = 0; ok && gemm_work<256>(p, total_tiles, it, wk, npairs, pair); ++it) {
+      int b, m0, nt;
+      pair_tile_coords(p, wk.tile, b, m0, nt);
+      const int half = wk.w / 2;
+      const int cpr = half / 8;   // chunks per row: 16 (128 columns) or 8 (64)
+      const int rpi = 32 / cpr;   // rows per warp instruction: 2 or 4
+      const int nb = SWIGLU ? nt * 128 + wk.n_off / 2 : nt * 256 + wk.n_off + static_cast<int>(rank) * half;
+      const uint16_t* W = (SWIGLU && rank == 1) ? p.gw1 : p.gw0;
+      const int c16 = lane % cpr;
+      const int col = nb + c16 * 8;
+      uint32_t col_bytes = 0;
+      if (col < p.N) col_bytes = (col + 8 <= p.N) ? 16u : static_cast<uint32_t>((p.N - col) * 2);
+      const int atom = c16 >> 3, cw = c16 & 7;
+      if (rpi != cur_rpi) {
+        load_rows(0, rpi, rows_next);
+        cur_rpi = rpi;
+      }
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        int rows[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rows[j] = rows_next[j];
+        load_rows(kb + 1 < p.num_kb ? kb + 1 : 0, rpi, rows_next);
+        int go = 1;
+        if (lane == 0) go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst0 = smem_u32(sB + stage * C::B_BYTES) + static_cast<uint32_t>(atom * 8192);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j * rpi < 16) {
+            const int r = g * 16 + j * rpi + lane / cpr;  // kept row within the k-block
+            const uint32_t dst = dst0 + static_cast<uint32_t>(r * 128 + ((cw ^ (r & 7)) << 4));
+            const int64_t src_row = rows[j];
+            const uint16_t* src = W;
+            uint32_t bytes = 0;
+            if (src_row >= 0 && col_bytes != 0) {
+              src = W + src_row * p.gldw + col;
+              bytes = col_bytes;
+            }
+            pair_cp_async16(dst, src, bytes);
+          }
+        }
+        pair_cp_async_commit();
+        ++issued;
+        if (issued > kPairGatherLag) {
+          // the copies of the k-block issued kPairGatherLag groups ago have landed
+          pair_cp_async_wait<kPairGatherLag>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          const uint32_t s_old = (issued - 1 - kPairGatherLag) % STAGES;
+          if (lane == 0) mbar_arrive_cluster(full_even + 8u * s_old);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // the k-blocks still in flight: land them (also on the abort path, so nothing
+    // lands after exit) and, unless aborting, signal them
+    pair_cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (ok && lane == 0) {
+      const uint32_t first = issued > kPairGatherLag ? issued - kPairGatherLag : 0u;
+      for (uint32_t q = first; q < issued; ++q) mbar_arrive_cluster(full_even + 8u * (q % STAGES));
+    }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;

@@ -20,7 +20,10 @@
 // Work split (stream-K): the (super tile, 64-row k-block) units are cut into
 // one contiguous range per CTA; a CTA writes one partial super tile per super
 // tile it touches, into slot (super tile + cta), and gemv_fixup_kernel adds the
-// partials of each column in CTA order, so the result is deterministic.
+// partials of each column in CTA order, so the result is deterministic.  (Adding
+// them in the last CTA of each super tile, behind an arrival counter, was
+// measured slower: 128 epilogue threads cannot keep enough partial loads in
+// flight once n >= 8.)
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -39,6 +42,38 @@ struct GemvParams {
   int64_t units;       // m_super * kb_total
   float* partial;      // [m_super + gridDim.x][4][n][128]
 };
+
+// Owners of the units of super tile `sup`: CTAs c_lo..c_hi (each with at least
+// one unit when the grid does not exceed the unit count).  ``fn(c)`` is called
+// for every CTA that touched the super tile, in increasing c.
+template <typename F>
+__device__ __forceinline__ void gemv_for_each_owner(const GemvParams& p, int64_t G, int sup, F&& fn) {
+  const int64_t U = p.units;
+  const int64_t u_lo = static_cast<int64_t>(sup) * p.kb_total;
+  const int64_t u_hi = u_lo + p.kb_total - 1;
+  if ((U + 1) * G < (1LL << 32)) {
+    // the unit split in 32-bit unsigned arithmetic (the usual case; much cheaper
+    // than 64-bit division)
+    const uint32_t u32 = static_cast<uint32_t>(U), g32 = static_cast<uint32_t>(G);
+    const uint32_t c_lo = (static_cast<uint32_t>(u_lo + 1) * g32 - 1u) / u32;  // owner of unit u_lo
+    const uint32_t c_hi = (static_cast<uint32_t>(u_hi + 1) * g32 - 1u) / u32;  // owner of unit u_hi
+    uint32_t start_c = (c_lo * u32) / g32;
+    for (uint32_t c = c_lo; c <= c_hi; ++c) {
+      const uint32_t start_next = ((c + 1u) * u32) / g32;
+      if (start_next > start_c) fn(static_cast<int64_t>(c));  // CTA c had at least one unit
+      start_c = start_next;
+    }
+  } else {
+    const int64_t c_lo = ((u_lo + 1) * G - 1) / U;
+    const int64_t c_hi = ((u_hi + 1) * G - 1) / U;
+    int64_t start_c = (c_lo * U) / G;
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      const int64_t start_next = ((c + 1) * U) / G;
+      if (start_next > start_c) fn(c);
+      start_c = start_next;
+    }
+  }
+}
 
 constexpr int kGemvTiles = 4;                  // 128-column MMA tiles per super tile
 constexpr int kGemvCols = 128 * kGemvTiles;    // 512 columns = 1 KB of each kept row per stage
@@ -312,47 +347,61 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
 }
 
 // Y[r, col] = bf16( sum over the CTAs c that touched the column's super tile, in
-// increasing c, of their partial sums ).  One thread per (output column, row r =
-// blockIdx.y); the owning CTAs are found from the same unit split as the kernel.
+// increasing c, of their partial sums ).  One CTA per (128-column MMA tile of a
+// super tile, 4 rows): thread 0 lists the owning CTAs in shared memory once (at
+// most grid + 1 of them: dynamic shared memory of (grid + 1) ints), then each
+// thread adds the float4 partials of 4 columns of one row over the list
+// (independent loads, summed in CTA order).
 __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy) {
+  extern __shared__ int s_own[];
+  __shared__ int s_count;
+  const int sup = blockIdx.x / kGemvTiles;
+  const int tl = blockIdx.x % kGemvTiles;
+  // the owner list depends only on the launch shape: built before the wait, while
+  // the product kernel is still running
+  if (threadIdx.x == 0) {
+    int c_count = 0;
+    gemv_for_each_owner(p, grid, sup, [&](int64_t c) { s_own[c_count++] = static_cast<int>(c); });
+    s_count = c_count;
+  }
+  __syncthreads();
   wait_prior_kernels();
-  const int col = blockIdx.x * 128 + threadIdx.x;
-  const int r = blockIdx.y;
-  if (col >= p.m) return;
-  const int sup = col / kGemvCols;
-  const int tl = (col % kGemvCols) / 128;
-  const int i = col % 128;
-  const int64_t U = p.units, G = grid;
-  const int64_t u_lo = static_cast<int64_t>(sup) * p.kb_total;
-  const int64_t u_hi = u_lo + p.kb_total - 1;
-  float acc = 0.f;
-  const float* src = p.partial + static_cast<int64_t>(tl) * p.n * 128 + r * 128 + i;
+  const int count = s_count;
+  const int i4 = (threadIdx.x & 31) * 4;
+  const int r = blockIdx.y * 4 + (threadIdx.x >> 5);
+  if (r >= p.n) return;
   const int64_t slot = static_cast<int64_t>(kGemvTiles) * p.n * 128;  // floats per partial super tile
-  if ((U + 1) * G < (1LL << 32)) {
-    // the unit split in 32-bit unsigned arithmetic (the usual case; much cheaper
-    // than 64-bit division)
-    const uint32_t u32 = static_cast<uint32_t>(U), g32 = static_cast<uint32_t>(G);
-    const uint32_t c_lo = (static_cast<uint32_t>(u_lo + 1) * g32 - 1u) / u32;  // owner of unit u_lo
-    const uint32_t c_hi = (static_cast<uint32_t>(u_hi + 1) * g32 - 1u) / u32;  // owner of unit u_hi
-    uint32_t start_c = (c_lo * u32) / g32;
-    for (uint32_t c = c_lo; c <= c_hi; ++c) {
-      const uint32_t start_next = ((c + 1u) * u32) / g32;
-      if (start_next > start_c)  // CTA c had at least one unit
-        acc += src[(static_cast<int64_t>(sup) + c) * slot];
-      start_c = start_next;
-    }
-  } else {
-    const int c_lo = static_cast<int>(((u_lo + 1) * G - 1) / U);
-    const int c_hi = static_cast<int>(((u_hi + 1) * G - 1) / U);
-    int64_t start_c = (static_cast<int64_t>(c_lo) * U) / G;
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const int64_t start_next = (static_cast<int64_t>(c + 1) * U) / G;
-      if (start_next > start_c) acc += src[(static_cast<int64_t>(sup) + c) * slot];
-      start_c = start_next;
+  const float* src = p.partial + static_cast<int64_t>(sup) * slot + (static_cast<int64_t>(tl) * p.n + r) * 128 + i4;
+  float ax = 0.f, ay = 0.f, az = 0.f, aw = 0.f;
+  int q = 0;
+  for (; q + 4 <= count; q += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float4*>(src + static_cast<int64_t>(s_own[q + u]) * slot);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      ax += v[u].x;
+      ay += v[u].y;
+      az += v[u].z;
+      aw += v[u].w;
     }
   }
-  const __nv_bfloat16 h = __float2bfloat16_rn(acc);
-  Y[static_cast<int64_t>(r) * ldy + col] = *reinterpret_cast<const uint16_t*>(&h);
+  for (; q < count; ++q) {
+    const float4 v = *reinterpret_cast<const float4*>(src + static_cast<int64_t>(s_own[q]) * slot);
+    ax += v.x;
+    ay += v.y;
+    az += v.z;
+    aw += v.w;
+  }
+  const int col = sup * kGemvCols + tl * 128 + i4;
+  const float a[4] = {ax, ay, az, aw};
+  uint16_t* y = Y + static_cast<int64_t>(r) * ldy + col;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (col + e < p.m) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(a[e]);
+      y[e] = *reinterpret_cast<const uint16_t*>(&h);
+    }
 }
 
 }  // namespace rmm

@@ -382,6 +382,7 @@ __global__ void __launch_bounds__(256) pack_rows_bulk_kernel(const PackParams p,
       const uint32_t v1 = (j1 < lim) ? row[j1] : 0u;
       dst[t] = v0 | (v1 << 16);
     }
+    fence_proxy_async_smem();  // this row's reads are ordered before the next bulk copy into its buffer
     gather_at.next(p);
   }
   if (threadIdx.x == 0 && *abort_flag) {

@@ -191,6 +191,7 @@ def test_mlp_argument_errors(L):
     assert mlp(d=40000, ldx=40000) == UNSUPPORTED
     assert mlp() == WORKSPACE
     a = L.rmm_mlp_workspace_bytes(300, 512, 1024, 512, 0.5, 0.5)
+    # the down projection's workspace plus X[:, I], the kept gate and up rows and the selection
     assert a >= L.rmm_linear_workspace_bytes(300, 1024, 512, 0.5) + 300 * 256 * 2 + 2 * 256 * 1024 * 2
     assert L.rmm_mlp_workspace_bytes(300, 512, 1024, 512, 1.0, 1.0) == 0
 

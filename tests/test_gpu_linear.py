@@ -128,11 +128,14 @@ def test_linear_llama8b_prefill_sampled(name, rho):
     parity_linear(A, W, rho, rows=rows)
 
 
-def test_stage_entry_points_compose_to_rmm_linear():
-    """rmm_select -> rmm_gather_columns -> rmm_gather_rows -> rmm_gemm_packed gives
-    the same bits as rmm_linear."""
+@pytest.mark.parametrize("n", [300, 100])
+def test_stage_entry_points_compose_to_rmm_linear(n):
+    """rmm_select -> rmm_gather_columns -> rmm_gemm_gathered (n > 128), or
+    -> rmm_gather_rows -> rmm_gemm_packed (n <= 128), gives the same bits as
+    rmm_linear; and the gathered product equals the packed one bit for bit (the
+    same k-blocks in the same order, only the source of B's rows differs)."""
     g = synthetic.rng(31)
-    A = synthetic.to_bf16(synthetic.outlier_activations(g, 300, 1000, 1.5)).cuda()
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, n, 1000, 1.5)).cuda()
     B = synthetic.to_bf16(synthetic.gaussian_weight(g, 1000, 520)).cuda()
     Y, idx = rmm.linear(A, B, 0.7, return_idx=True)
     idx2, _, _ = rmm.select(A, 0.7)
@@ -140,11 +143,14 @@ def test_stage_entry_points_compose_to_rmm_linear():
     ap = rmm.gather_columns(A, idx2, ld_pack=712)
     bp = rmm.gather_rows(B, idx2, ld_pack=528)
     Y2 = rmm.gemm_packed(ap, k, bp, 520)
+    Y3 = rmm.gemm_gathered(ap, k, B, idx2)
     torch.cuda.synchronize()
     assert torch.equal(idx, idx2)
-    assert torch.equal(Y, Y2)
+    assert torch.equal(Y, Y3 if n > 128 else Y2)
+    if n > 128:
+        assert torch.equal(Y2, Y3)
     I = idx2.cpu().long()
-    expect = torch.zeros((300, 712), dtype=torch.bfloat16)
+    expect = torch.zeros((n, 712), dtype=torch.bfloat16)
     expect[:, :k] = A.cpu()[:, I]
     assert torch.equal(ap.cpu(), expect)
     assert torch.equal(bp.cpu()[:, :520], B.cpu()[I, :])
@@ -259,3 +265,33 @@ def test_linear_decode_deterministic():
     b = rmm.linear(Ad, Wd, 0.7, return_idx=True)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("n,d,m,k", [(4096, 4096, 14336, 2048), (300, 2056, 520, 1000), (257, 1000, 300, 1),
+                                     (512, 14336, 4096, 12903), (1000, 777, 136, 700), (129, 64, 8, 64)])
+def test_gemm_gathered_matches_the_packed_product(n, d, m, k):
+    """The gathered product against the packed one (bit for bit) and against the fp32
+    reference: ragged n, m and k, m not a multiple of 8 (partial 16-byte rows), a
+    single kept row, narrow last-wave pieces, unsorted-free ascending sets."""
+    g = synthetic.rng(n + d + m + k)
+    ldp = (k + 7) // 8 * 8
+    A = torch.zeros((n, ldp), dtype=torch.bfloat16)
+    A[:, :k] = synthetic.to_bf16(g.standard_normal((n, k), dtype=np.float32))
+    ldb = (m + 7) // 8 * 8
+    Bfull = torch.zeros((d, ldb), dtype=torch.bfloat16)
+    Bfull[:, :m] = synthetic.to_bf16(g.standard_normal((d, m), dtype=np.float32) / np.float32(np.sqrt(k)))
+    idx = torch.as_tensor(np.sort(g.choice(d, size=k, replace=False)), dtype=torch.int32)
+    A, Bd, idx = A.cuda(), Bfull.cuda()[:, :m], idx.cuda()
+
+    def out():  # the library's rule: output rows start 16-byte aligned
+        return torch.zeros((n, ldb), dtype=torch.bfloat16, device="cuda")[:, :m]
+    Yg = rmm.gemm_gathered(A, k, Bd, idx, out=out())
+    bp = rmm.gather_rows(Bd, idx)
+    Yp = rmm.gemm_packed(A, k, bp, m, out=out())
+    Yg2 = rmm.gemm_gathered(A, k, Bd, idx, out=out())
+    torch.cuda.synchronize()
+    assert torch.equal(Yg, Yg2), "not deterministic"
+    if n > 128:
+        assert torch.equal(Yg, Yp), "gathered and packed products differ"
+    ref = (A[:, :k].float() @ Bd.float()[idx.long()]).cpu().numpy()
+    check_close(Yg.float().cpu().numpy(), ref, f"gathered product n={n} d={d} m={m} k={k}")
