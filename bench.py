@@ -45,7 +45,7 @@ GEMM_SOURCES = ["input_adaptive_reduced_colnorm_b200/csrc/gemm_pair.cuh", "input
 # launch at rho = 0.5 from one ncu capture, with the sha1 of the kernel sources it was
 # taken on; reported only while the sources are unchanged (the capture's summary is
 # in profiles/).
-GEMM_TRAFFIC = {"bytes": 158915584, "source_sha1": "b1d08603fb9c5b2752351bccc2067702dd0df5f1"}
+GEMM_TRAFFIC = {"bytes": 75694592 + 80094976, "source_sha1": "d5866c3ea16070f468720ef7468763ade97ec69b"}
 
 
 def parse_args():
@@ -654,18 +654,22 @@ def run_ours(args):
 
     # ---- the dominant kernel: the same launches through the stage entry points (the
     # kernels rmm_linear launches, in the same order, on the same stream), each product
-    # launch bracketed by CUDA events
+    # launch bracketed by CUDA events.  A short idle first lets the clocks recover from
+    # the main region (under the 1 kW power cap a long GEMM run lowers them).
+    time.sleep(1.0)
     for _ in range(W):
         step_stages(RHO_MAIN)
     evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in bufs]
            for _ in range(K)]
     barrier()
+    stage_clocks = ClockSampler(local)
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for s_ in range(K):
-        step_stages(RHO_MAIN, evs[s_])
-    s1.record(stream)
-    barrier()
+    with stage_clocks:
+        s0.record(stream)
+        for s_ in range(K):
+            step_stages(RHO_MAIN, evs[s_])
+        s1.record(stream)
+        barrier()
     ms_stages = max_over_ranks(s0.elapsed_time(s1) / K)
     gemm_ms = [statistics.mean(evs[s_][i][0].elapsed_time(evs[s_][i][1]) for s_ in range(K)) for i in range(len(bufs))]
     gemm_ms = [max_over_ranks(x) for x in gemm_ms]
@@ -685,6 +689,7 @@ def run_ours(args):
             fn()
     sweep_ms = {key: 0.0 for key in variants}
     for _ in range(rounds):
+        time.sleep(0.5)  # every round starts from the same idle clock state
         for key, fn in variants.items():
             sweep_ms[key] += timed(fn, per_round, 0) / rounds
     ms_rho = {float(r): sweep_ms[r] for r in ("0.9", "0.7", "0.5")}
@@ -780,7 +785,9 @@ def run_ours(args):
                      "kernel": "rmm_gemm_pair_kernel<false, false>: the reduced product of gate_proj (4096 x 14336, "
                                "k=2048) at rho = 0.5 on the packed A[:, I] and B[I, :]",
                      "peak_source": f"bf16_tflops (burst) of {peak_src}",
-                     "timed": f"{K} launches, CUDA events around each on the launching stream",
+                     "timed": f"{K} launches, CUDA events around each on the launching stream, in a pass through the "
+                              f"stage entry points after a 1 s idle",
+                     "clocks": stage_clocks.summary(),
                      "all_gemm_launches_tflops": all_gemm},
         "gemm_ms_per_launch": {x["name"]: gemm_ms[i] for i, x in enumerate(bufs)},
         "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
