@@ -15,9 +15,9 @@
 //     bits shared by every key are skipped (cluster-wide AND / OR), each pass
 //     resolves 8 bits with per-warp histograms merged per CTA and then across
 //     the cluster through distributed shared memory, one cluster barrier per
-//     pass; when the bucket holding the k-th key has become small, one more
-//     AND / OR of its members skips their shared bits, so exact ties (squares
-//     of a single bf16 row) end the passes at once;
+//     pass; the same barrier carries each pass's AND / OR of the bucket's
+//     members, so bits the bucket shares are skipped and a bucket of identical
+//     keys (squares of a single bf16 row) ends the passes at once;
 //   * the compaction takes every key above the threshold and the lowest-index
 //     keys equal to it, in index order: counts are exchanged once across the
 //     cluster (CTA order is column order), then two block scans give each
@@ -47,7 +47,10 @@ constexpr int kDecSelCols = kDecSelThreads * 8;  // columns per CTA
 constexpr int kDecSelMaxCtas = 8;                // portable cluster size
 constexpr int kDecSelMaxD = kDecSelCols * kDecSelMaxCtas;
 constexpr int kDecSelMaxRows = 32;
-constexpr int kDecSelSkipBelow = 64;             // bucket size at which shared bits are skipped again
+
+// The two halves of a cluster barrier, for work that can overlap its latency.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t ld_shared_cluster_u64(uint32_t addr) {
   uint64_t v;
@@ -114,6 +117,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   __shared__ uint32_t hist[2][256];
   __shared__ uint64_t s_wand[kDecSelThreads / 32], s_wor[kDecSelThreads / 32];
   __shared__ uint64_t s_andor[2], s_andor_res[2];
+  __shared__ uint64_t s_pass_andor[2][2];  // the bucket's AND / OR per pass (read by the cluster), double-buffered
   __shared__ int s_warp[32];
   __shared__ int s_total;
   __shared__ int s_digit, s_above, s_cnt;
@@ -178,17 +182,60 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
     const uint32_t dmask = (1u << width) - 1u;
     for (int i = lane; i < 256; i += 32) whist[warp][i] = 0u;
     __syncwarp();
+    // the bucket's histogram of the next digit, and the AND / OR of its members
+    uint64_t ba = ~0ull, bo = 0ull;
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      if (((valid >> e) & 1u) && (key[e] & msk) == pre)
+      if (((valid >> e) & 1u) && (key[e] & msk) == pre) {
+        ba &= key[e];
+        bo |= key[e];
         atomicAdd(&whist[warp][static_cast<uint32_t>(key[e] >> shift) & dmask], 1u);
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ba &= __shfl_xor_sync(0xffffffffu, ba, off);
+      bo |= __shfl_xor_sync(0xffffffffu, bo, off);
+    }
+    if (lane == 0) {
+      s_wand[warp] = ba;
+      s_wor[warp] = bo;
+    }
     __syncthreads();
     uint32_t c = 0;
 #pragma unroll
     for (int w = 0; w < kDecSelThreads / 32; ++w) c += whist[w][tid];
     uint32_t* hb = hist[pass & 1];
     hb[tid] = c;
-    cluster_sync();  // every CTA's histogram of this pass is visible (and the one two passes back is no longer read)
+    uint64_t* ab = s_pass_andor[pass & 1];
+    if (tid == 0) {
+      uint64_t xa = ~0ull, xo = 0ull;
+      for (int w = 0; w < kDecSelThreads / 32; ++w) {
+        xa &= s_wand[w];
+        xo |= s_wor[w];
+      }
+      ab[0] = xa;
+      ab[1] = xo;
+    }
+    // every CTA's histogram and AND / OR of this pass are visible (and the ones
+    // two passes back are no longer read)
+    cluster_sync();
+    if (warp == 0) {
+      uint64_t ra = ~0ull, ro = 0ull;
+      if (lane < C) {
+        const uint32_t aaddr = smem_u32(ab);
+        ra = ld_shared_cluster_u64(map_shared_rank(aaddr, static_cast<uint32_t>(lane)));
+        ro = ld_shared_cluster_u64(map_shared_rank(aaddr + 8, static_cast<uint32_t>(lane)));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        ra &= __shfl_xor_sync(0xffffffffu, ra, off);
+        ro |= __shfl_xor_sync(0xffffffffu, ro, off);
+      }
+      if (lane == 0) {
+        s_andor_res[0] = ra;
+        s_andor_res[1] = ro;
+      }
+    }
     // thread t takes digit 255 - t, so the exclusive scan in thread order counts the larger digits
     const int bin = 255 - tid;
     uint32_t cnt = 0;
@@ -201,34 +248,36 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
       s_cnt = static_cast<int>(cnt);
     }
     __syncthreads();
+    const uint64_t ga = s_andor_res[0], go = s_andor_res[1];
+    const uint64_t open = (cursor >= 64) ? ~0ull : ((1ull << cursor) - 1ull);  // unresolved bits
+    ++pass;
+    if (((ga ^ go) & open) == 0ull) {
+      // every member of the bucket has the same key: the lower indices win
+      pre |= ga & open;
+      msk = ~0ull;
+      cursor = 0;
+      __syncthreads();
+      break;
+    }
     need -= s_above;
     pre |= static_cast<uint64_t>(s_digit) << shift;
     msk |= static_cast<uint64_t>(dmask) << shift;
     cursor = shift;
-    const int bucket = s_cnt;
-    if (bucket == need) take = true;
-    ++pass;
-    if (!take && cursor > 0 && bucket <= kDecSelSkipBelow) {
-      // a small bucket: skip the bits its members share (all of them for exact ties)
-      uint64_t a = ~0ull, o = 0ull;
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (((valid >> e) & 1u) && (key[e] & msk) == pre) {
-          a &= key[e];
-          o |= key[e];
-        }
-      __syncthreads();  // every thread has read the scan results of this pass
-      decsel_cluster_andor(a, o, s_wand, s_wor, s_andor, s_andor_res, C);
-      const uint64_t open = (cursor >= 64) ? ~0ull : ((1ull << cursor) - 1ull);
-      const uint64_t dl = (a ^ o) & open;
+    if (s_cnt == need) {
+      take = true;
+    } else if (cursor > 0) {
+      // bits below the digit that the whole bucket shares are shared by the
+      // digit's sub-bucket too: skip them (all of them for exact ties)
+      const uint64_t below = (1ull << cursor) - 1ull;
+      const uint64_t dl = (ga ^ go) & below;
       if (dl == 0ull) {
-        pre |= a & open;
+        pre |= ga & below;
         msk = ~0ull;
         cursor = 0;
       } else {
         const int top = 63 - __clzll(static_cast<long long>(dl));
-        const uint64_t shared = open & ~((top == 63) ? ~0ull : ((1ull << (top + 1)) - 1ull));
-        pre |= a & shared;
+        const uint64_t shared = below & ~((1ull << (top + 1)) - 1ull);
+        pre |= ga & shared;
         msk |= shared;
         cursor = top + 1;
       }
@@ -270,7 +319,10 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
     s_sel_base = sel_before;
     s_eq_before = eq_before;
   }
-  cluster_sync();  // no CTA reads another's shared memory past this point
+  __syncthreads();
+  // no CTA reads another's shared memory past this point: arrive now, and wait
+  // (so that no CTA exits while another may still read it) only at the end
+  cluster_arrive();
   uint32_t sel = gt;
   {
     int r = s_eq_before + eq_rank;
@@ -326,6 +378,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
     if (rank == C - 1 && tid < p.n)
       for (int64_t t = p.k; t < p.ld_pack; ++t) p.xpack[static_cast<int64_t>(tid) * p.ld_pack + t] = 0;
   }
+  cluster_wait();
 }
 
 }  // namespace rmm
