@@ -343,7 +343,7 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
     del W
     torch.cuda.empty_cache()
     dq = {}
-    for n in (1, 8):
+    for n in (1, 8, 32):
         x, _ = synthetic.decode_gemv(n, weight=False)
         x = x.to(dev)
         d, m = 8192, 28672
@@ -356,6 +356,7 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
             k = k_of(r, d)
             nbytes = k * m + (n * d * 2 if k < d else 0) + n * k * 2 + n * m * 2
             row[str(r)] = {"k": k, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                           "kernel": "CUDA cores" if n <= 2 else "tensor cores (dequantised in shared memory)",
                            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm,
                            "vs_bf16_same_rho": dec[f"n={n}"][str(r)]["ms"] / ms}
             del ws

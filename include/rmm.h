@@ -233,22 +233,24 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
                          double rho, int32_t* idx_out, void* ws, size_t ws_bytes, rmm_stream stream);
 
 /* ---------------------------------------------------------------- int8 weights
- * Reduced projection with int8 weights for decode (n <= 8 rows):
+ * Reduced projection with int8 weights for decode (n <= 32 rows):
  *   Y = (A[:, I] . Wq[I, :]) * scale[None, :]
  * with I = TopK of A's column norms exactly as in rmm_linear ("Reduced Matrix
  * Multiplication ... Technical Summary", Compatibility: INT8 weight
  * quantization; "Algorithm Deep-Dive: RMM", Compatibility & generalization).
  * The weights are stored int8 with one fp32 scale per output column (W = Wq *
  * scale, a reading: the pages name no scheme); only the kept rows of Wq are
- * read, on the CUDA cores, with fp32 accumulation.
- *   A      device bf16 [n][lda], n x d, n <= 8.
+ * read, with fp32 accumulation: on the CUDA cores for n <= 2, on the tensor
+ * cores for 3 <= n <= 32 (the kept rows dequantised exactly to bf16 in shared
+ * memory, the scales applied to the fp32 sums).
+ *   A      device bf16 [n][lda], n x d, n <= 32.
  *   Wq     device int8 [d][ldw], d x m (contraction index as the row), ldw % 8 == 0.
  *   scale  device fp32 [m].
  *   Y      device bf16 [n][ldy].
  *   idx_out device int32 [rmm_k(rho, d)] or NULL.
  * Requires m % 8 == 0, d <= 32768.  Workspace: scores, index set and fp32
- * partial sums of the row chunks (added in a fixed order); the kernel reads
- * A[:, I] through the index set, so no packed copy of A is made. */
+ * partial sums (added in a fixed order); for n <= 2 the kernel reads A[:, I]
+ * through the index set, for larger n the selection packs it. */
 size_t rmm_linear_int8_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho);
 rmm_status rmm_linear_int8(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda, const int8_t* Wq, int64_t m,
                            int64_t ldw, const float* scale, rmm_bf16* Y, int64_t ldy, double rho, int32_t* idx_out,

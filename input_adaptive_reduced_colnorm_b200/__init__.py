@@ -323,7 +323,7 @@ def attention(Q, K, V, rho: float, *, causal: bool = True, scale: float = 1.0, o
 
 
 def linear_int8(A, Wq, scale, rho: float, *, out=None, return_idx: bool = False, workspace=None):
-    """Y = (A[:, I] Wq[I, :]) * scale with I chosen on A (decode, n <= 8 rows).
+    """Y = (A[:, I] Wq[I, :]) * scale with I chosen on A (decode, n <= 32 rows).
     A [n, d] bf16, Wq [d, m] int8, scale [m] float32, all CUDA."""
     import torch
     _require(A, "A", torch.bfloat16, 2)

@@ -335,50 +335,61 @@ namespace rmm {
 // order.  Non-causal only.
 constexpr int kColsqShortMaxRows = 32;
 
-// Sums of squares of columns [col0, col0 + 8) of an n-row matrix (n may be
-// anything; used for n <= 32): rows summed 4 at a time in fp32 (exact bf16
-// squares) and folded into fp64, in row order.  Columns at or past d read as 0.
-// The decode selection kernel computes its scores with this same function, so
-// its keys are bit-identical to colsq_short_kernel's.
-__device__ __forceinline__ void colsq_short_cols8(const uint16_t* A, int64_t lda, int64_t n, int64_t col0, int64_t d,
-                                                  double (&acc)[8]) {
-  const bool full = col0 + 8 <= d;
+// Sums of squares of columns [col0, col0 + CPT) (CPT = 4 or 8) of an n-row
+// matrix (n may be anything; used for n <= 32): rows summed 4 at a time in fp32
+// (exact bf16 squares) and folded into fp64, in row order.  Columns at or past d
+// read as 0.  Each column's arithmetic does not depend on CPT, and the decode
+// selection kernel computes its scores with this same function, so its keys are
+// bit-identical to colsq_short_kernel's.
+template <int CPT>
+__device__ __forceinline__ void colsq_short_cols(const uint16_t* A, int64_t lda, int64_t n, int64_t col0, int64_t d,
+                                                 double (&acc)[CPT]) {
+  static_assert(CPT == 4 || CPT == 8, "four or eight columns per thread");
+  constexpr int WPR = CPT / 2;  // 32-bit words per row chunk
+  const bool full = col0 + CPT <= d;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  for (int e = 0; e < CPT; ++e) acc[e] = 0.0;
   for (int64_t r0 = 0; r0 < n; r0 += 8) {
-    uint32_t w[8][4];
+    uint32_t w[8][WPR];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      w[u][0] = w[u][1] = w[u][2] = w[u][3] = 0u;
+#pragma unroll
+      for (int q = 0; q < WPR; ++q) w[u][q] = 0u;
       if (r0 + u < n) {
         const uint16_t* src = A + (r0 + u) * lda + col0;
         if (full) {
-          const uint4 v = ldg_nc_v4(src);
-          w[u][0] = v.x;
-          w[u][1] = v.y;
-          w[u][2] = v.z;
-          w[u][3] = v.w;
+          if constexpr (CPT == 8) {
+            const uint4 v = ldg_nc_v4(src);
+            w[u][0] = v.x;
+            w[u][1] = v.y;
+            w[u][2] = v.z;
+            w[u][3] = v.w;
+          } else {
+            const uint2 v = ldg_nc_v2(src);
+            w[u][0] = v.x;
+            w[u][1] = v.y;
+          }
         } else {
-          for (int e = 0; e < 8; ++e)
+          for (int e = 0; e < CPT; ++e)
             if (col0 + e < d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
         }
       }
     }
 #pragma unroll
     for (int g = 0; g < 8; g += 4) {
-      float a32[8];
+      float a32[CPT];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a32[e] = 0.f;
+      for (int e = 0; e < CPT; ++e) a32[e] = 0.f;
 #pragma unroll
       for (int u = g; u < g + 4; ++u) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < CPT; ++e) {
           const float x = (e & 1) ? bf16hi(w[u][e >> 1]) : bf16lo(w[u][e >> 1]);
           a32[e] = fmaf(x, x, a32[e]);
         }
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += static_cast<double>(a32[e]);
+      for (int e = 0; e < CPT; ++e) acc[e] += static_cast<double>(a32[e]);
     }
   }
 }
@@ -389,7 +400,7 @@ __global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {
   const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
   if (col0 >= p.d) return;
   double acc[8];
-  colsq_short_cols8(p.A + b * p.batch_stride, p.lda, p.n, col0, p.d, acc);
+  colsq_short_cols<8>(p.A + b * p.batch_stride, p.lda, p.n, col0, p.d, acc);
   double* out = p.colsq + b * p.d + col0;
 #pragma unroll
   for (int e = 0; e < 8; ++e)

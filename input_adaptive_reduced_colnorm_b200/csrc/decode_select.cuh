@@ -6,10 +6,11 @@
 //
 // At decode sizes each of the three steps is a latency-bound launch of a few
 // microseconds, and one CTA selecting over d = 8192 keys is issue-bound, so the
-// work is spread over one cluster of C = ceil(d / 2048) CTAs (C <= 8):
-//   * CTA r owns columns [2048 r, 2048 (r + 1)); each of its 256 threads owns 8
-//     consecutive columns and computes their fp64 scores with the arithmetic of
-//     the short-matrix column-score kernel (bit-identical keys);
+// work is spread over one cluster of C CTAs of 256 threads (C <= 8):
+//   * each thread owns KPT consecutive columns (4 while 8 CTAs of 1024 columns
+//     cover d, i.e. d <= 8192; else 8, d <= 16384) and computes their fp64 scores
+//     with the arithmetic of the short-matrix column-score kernel (bit-identical
+//     keys); CTA r owns columns [256 KPT r, 256 KPT (r + 1));
 //   * the k-th largest key is found by an MSB-first radix select over the
 //     64-bit key patterns (non-negative doubles order like their bits): leading
 //     bits shared by every key are skipped (cluster-wide AND / OR), each pass
@@ -43,9 +44,11 @@ struct DecodeSelParams {
 };
 
 constexpr int kDecSelThreads = 256;
-constexpr int kDecSelCols = kDecSelThreads * 8;  // columns per CTA
 constexpr int kDecSelMaxCtas = 8;                // portable cluster size
-constexpr int kDecSelMaxD = kDecSelCols * kDecSelMaxCtas;
+// KPT columns per thread: 4 for d <= 8192 (clusters of up to 8 CTAs of 1024
+// columns: half the per-thread work of 8), 8 up to d = 16384
+constexpr int kDecSelMaxD = kDecSelThreads * 8 * kDecSelMaxCtas;
+__host__ __device__ constexpr int decsel_cols_per_cta(int kpt) { return kDecSelThreads * kpt; }
 constexpr int kDecSelMaxRows = 32;
 
 // The two halves of a cluster barrier, for work that can overlap its latency.
@@ -112,6 +115,7 @@ __device__ __forceinline__ void decsel_cluster_andor(uint64_t& a, uint64_t& o, u
   o = res[1];
 }
 
+template <int KPT>
 __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const DecodeSelParams p) {
   __shared__ uint32_t whist[kDecSelThreads / 32][256];
   __shared__ uint32_t hist[2][256];
@@ -128,21 +132,21 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   const int C = static_cast<int>(gridDim.x);  // the grid is one cluster
   const int rank = static_cast<int>(cluster_ctarank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t col0 = static_cast<int64_t>(rank) * kDecSelCols + tid * 8;
+  const int64_t col0 = static_cast<int64_t>(rank) * decsel_cols_per_cta(KPT) + tid * KPT;
 
   // ---- scores (fp64, bit-identical to colsq_short_kernel) and their key patterns
-  uint64_t key[8];
+  uint64_t key[KPT];
   uint32_t valid = 0;
   {
-    double acc[8];
+    double acc[KPT];
     if (col0 < p.d) {
-      colsq_short_cols8(p.x, p.ldx, p.n, col0, p.d, acc);
+      colsq_short_cols<KPT>(p.x, p.ldx, p.n, col0, p.d, acc);
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+      for (int e = 0; e < KPT; ++e) acc[e] = 0.0;
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < KPT; ++e) {
       key[e] = static_cast<uint64_t>(__double_as_longlong(acc[e]));
       if (col0 + e < p.d) valid |= 1u << e;
     }
@@ -156,7 +160,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   {
     uint64_t a = ~0ull, o = 0ull;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < KPT; ++e)
       if ((valid >> e) & 1u) {
         a &= key[e];
         o |= key[e];
@@ -185,7 +189,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
     // the bucket's histogram of the next digit, and the AND / OR of its members
     uint64_t ba = ~0ull, bo = 0ull;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < KPT; ++e)
       if (((valid >> e) & 1u) && (key[e] & msk) == pre) {
         ba &= key[e];
         bo |= key[e];
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   // ---- classify: above the threshold, or equal to it
   uint32_t gt = 0, eq = 0;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
+  for (int e = 0; e < KPT; ++e) {
     if (!((valid >> e) & 1u)) continue;
     const uint64_t km = key[e] & msk;
     if (km > pre) gt |= 1u << e;
@@ -327,7 +331,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   {
     int r = s_eq_before + eq_rank;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < KPT; ++e)
       if ((eq >> e) & 1u) {
         if (take || r < need) sel |= 1u << e;
         ++r;
@@ -337,29 +341,37 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   {
     int pos = pos0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < KPT; ++e)
       if ((sel >> e) & 1u) p.idx[pos++] = static_cast<int32_t>(col0 + e);
   }
   if (p.xpack != nullptr) {
     if (sel != 0u) {
       // eight rows' loads are issued before any of their stores, so each batch
       // costs one round trip instead of eight
-      const bool full = col0 + 8 <= p.d;
+      const bool full = col0 + KPT <= p.d;
+      constexpr int WPR = KPT / 2;  // 32-bit words per row chunk
       for (int r0 = 0; r0 < p.n; r0 += 8) {
-        uint32_t w[8][4];
+        uint32_t w[8][WPR];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          w[u][0] = w[u][1] = w[u][2] = w[u][3] = 0u;
+#pragma unroll
+          for (int q = 0; q < WPR; ++q) w[u][q] = 0u;
           if (r0 + u < p.n) {
             const uint16_t* src = p.x + static_cast<int64_t>(r0 + u) * p.ldx + col0;
             if (full) {
-              const uint4 v = ldg_nc_v4(src);
-              w[u][0] = v.x;
-              w[u][1] = v.y;
-              w[u][2] = v.z;
-              w[u][3] = v.w;
+              if constexpr (KPT == 8) {
+                const uint4 v = ldg_nc_v4(src);
+                w[u][0] = v.x;
+                w[u][1] = v.y;
+                w[u][2] = v.z;
+                w[u][3] = v.w;
+              } else {
+                const uint2 v = ldg_nc_v2(src);
+                w[u][0] = v.x;
+                w[u][1] = v.y;
+              }
             } else {
-              for (int e = 0; e < 8; ++e)
+              for (int e = 0; e < KPT; ++e)
                 if (col0 + e < p.d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
             }
           }
@@ -370,7 +382,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
           uint16_t* dst = p.xpack + static_cast<int64_t>(r0 + u) * p.ld_pack;
           int pos = pos0;
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
+          for (int e = 0; e < KPT; ++e)
             if ((sel >> e) & 1u) dst[pos++] = static_cast<uint16_t>(w[u][e >> 1] >> (16 * (e & 1)));
         }
       }

@@ -351,8 +351,9 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
 // super tile, 4 rows): thread 0 lists the owning CTAs in shared memory once (at
 // most grid + 1 of them: dynamic shared memory of (grid + 1) ints), then each
 // thread adds the float4 partials of 4 columns of one row over the list
-// (independent loads, summed in CTA order).
-__global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy) {
+// (independent loads, summed in CTA order), times scale[col] when scale is given.
+__global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int grid, uint16_t* Y, int64_t ldy,
+                                                         const float* scale) {
   extern __shared__ int s_own[];
   __shared__ int s_count;
   const int sup = blockIdx.x / kGemvTiles;
@@ -394,7 +395,12 @@ __global__ void __launch_bounds__(128) gemv_fixup_kernel(const GemvParams p, int
     aw += v.w;
   }
   const int col = sup * kGemvCols + tl * 128 + i4;
-  const float a[4] = {ax, ay, az, aw};
+  float a[4] = {ax, ay, az, aw};
+  if (scale != nullptr) {  // int8 weights: one fp32 scale per output column
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (col + e < p.m) a[e] *= __ldg(scale + col + e);
+  }
   uint16_t* y = Y + static_cast<int64_t>(r) * ldy + col;
 #pragma unroll
   for (int e = 0; e < 4; ++e)

@@ -363,9 +363,12 @@ rmm_status launch_decode_select(const uint16_t* x, int64_t n, int64_t d, int64_t
   p.idx = idx;
   p.xpack = xpack;
   p.ld_pack = ld_pack;
-  const int C = static_cast<int>(ceil_div(d, kDecSelCols));
-  const cudaError_t e = launch_cluster(decode_select_kernel, dim3(static_cast<unsigned>(C)), dim3(kDecSelThreads), 0, C,
-                                       s, p);
+  // four columns per thread while a cluster of at most 8 CTAs covers d, else eight
+  const bool four = d <= decsel_cols_per_cta(4) * kDecSelMaxCtas;
+  const int C = static_cast<int>(ceil_div(d, decsel_cols_per_cta(four ? 4 : 8)));
+  const cudaError_t e =
+      four ? launch_cluster(decode_select_kernel<4>, dim3(static_cast<unsigned>(C)), dim3(kDecSelThreads), 0, C, s, p)
+           : launch_cluster(decode_select_kernel<8>, dim3(static_cast<unsigned>(C)), dim3(kDecSelThreads), 0, C, s, p);
   if (e != cudaSuccess) return cuda_fail(e, "decode selection launch");
   return RMM_OK;
 }
@@ -628,6 +631,9 @@ rmm_status gemm_gathered(const uint16_t* A, int64_t n, int64_t k, int64_t lda, c
 
 // Decode path (n <= 32): Y = x[:, I] . W[I, :] streaming only the kept rows of W.
 constexpr int64_t kDecodeMaxRows = 32;
+// int8 weights: activation rows up to which the CUDA-core kernel runs; the tensor
+// cores take more
+constexpr int64_t kI8CudaCoreMaxRows = 2;
 
 int decode_grid(int64_t units) { return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, num_sms()))); }
 
@@ -666,7 +672,8 @@ rmm_status decode_product(const uint16_t* xp, int64_t n, int64_t ldx, const uint
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = launch_chained(gemv_fixup_kernel, dim3(static_cast<unsigned>(g.m_super * kGemvTiles), static_cast<unsigned>(ceil_div(n, 4))),
-                     dim3(128), static_cast<size_t>(grid + 1) * sizeof(int), s, g, grid, Y, ldy);
+                     dim3(128), static_cast<size_t>(grid + 1) * sizeof(int), s, g, grid, Y, ldy,
+                     static_cast<const float*>(nullptr));
   if (e != cudaSuccess) return cuda_fail(e, "decode fix-up launch");
   return RMM_OK;
 }
@@ -823,9 +830,63 @@ cudaError_t launch_gemv_i8_t(const GemvI8Params& p, cudaStream_t s) {
 
 extern "C" {
 
+// int8 weights on the tensor cores (n > kI8CudaCoreMaxRows): dequantised in the
+// producer into the bf16 UMMA stage; x[:, I] packed by the decode selection.
+rmm_status int8_tc_product(const uint16_t* xp, int64_t n, int64_t ldx, const int8_t* W, int64_t k, int64_t m,
+                           int64_t ldw, const int32_t* idx, const float* scale, float* partial, uint16_t* Y, int64_t ldy,
+                           cudaStream_t s) {
+  GemvI8TcParams g{};
+  g.W = W;
+  g.ldw = ldw;
+  g.idx = idx;
+  g.k = static_cast<int>(k);
+  g.m = static_cast<int>(m);
+  g.n = static_cast<int>(n);
+  g.m_super = static_cast<int>(ceil_div(m, kGemvCols));
+  g.kb_total = static_cast<int>(ceil_div(k, 64));
+  g.units = static_cast<int64_t>(g.m_super) * g.kb_total;
+  g.partial = partial;
+  const int grid = decode_grid(g.units);
+  const int N = (n <= 16) ? 16 : 32;
+  CUtensorMap tx;
+  if (rmm_status st = make_tmap(&tx, xp, k, n, ldx * 2, 64, static_cast<uint32_t>(N))) return st;
+  const int smem = 1024 + kGemvStages * (kGemvCols * 64 * 2 + N * 64 * 2) + 256;
+  cudaError_t e;
+  if (N == 16) {
+    e = cudaFuncSetAttribute(gemv_i8tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = launch_chained(gemv_i8tc_kernel<16>, dim3(grid), dim3(kI8TcThreads), smem, s, tx, g);
+  } else {
+    e = cudaFuncSetAttribute(gemv_i8tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = launch_chained(gemv_i8tc_kernel<32>, dim3(grid), dim3(kI8TcThreads), smem, s, tx, g);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "int8 tensor-core launch");
+  GemvParams f{};
+  f.k = g.k;
+  f.m = g.m;
+  f.n = g.n;
+  f.m_super = g.m_super;
+  f.kb_total = g.kb_total;
+  f.units = g.units;
+  f.partial = partial;
+  e = launch_chained(gemv_fixup_kernel, dim3(static_cast<unsigned>(f.m_super * kGemvTiles), static_cast<unsigned>(ceil_div(n, 4))),
+                     dim3(128), static_cast<size_t>(grid + 1) * sizeof(int), s, f, grid, Y, ldy, scale);
+  if (e != cudaSuccess) return cuda_fail(e, "int8 fix-up launch");
+  return RMM_OK;
+}
+
 size_t rmm_linear_int8_workspace_bytes(int64_t n, int64_t d, int64_t m, double rho) {
   const int64_t k = rmm_k(rho, d);
   if (k < 0 || n < 1 || m < 1) return 0;
+  if (n > kI8CudaCoreMaxRows) {
+    Carver c(nullptr);
+    if (k < d) {
+      c.take<double>(d);
+      c.take<int32_t>(k);
+      c.take<uint16_t>(n * round_up(k, 8));
+    }
+    c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
+    return c.bytes();
+  }
   int chunk = 0, chunks = 0;
   i8_plan(n, k, m, &chunk, &chunks);
   Carver c(nullptr);
@@ -846,7 +907,7 @@ rmm_status rmm_linear_int8(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda,
     return fail(RMM_ERR_INVALID_ARG, "A, Wq, scale and Y are required");
   if (n < 1 || d < 1 || m < 1) return fail(RMM_ERR_INVALID_ARG, "n, d and m must be >= 1");
   if (lda < d || ldw < m || ldy < m) return fail(RMM_ERR_INVALID_ARG, "leading dimension too small");
-  if (n > kI8MaxRows) return fail(RMM_ERR_UNSUPPORTED, "the int8 path takes at most 8 activation rows");
+  if (n > kDecodeMaxRows) return fail(RMM_ERR_UNSUPPORTED, "the int8 path takes at most 32 activation rows");
   if (!aligned16(A) || !aligned16(Wq) || !aligned16(Y) || (ws != nullptr && !aligned16(ws)) || (lda % 8) ||
       (ldw % 8) || (ldy % 8) || (m % 8))
     return fail(RMM_ERR_UNSUPPORTED, "pointers 16-byte aligned; lda, ldw, ldy and m multiples of 8");
@@ -857,6 +918,33 @@ rmm_status rmm_linear_int8(const rmm_bf16* A, int64_t n, int64_t d, int64_t lda,
     return fail(RMM_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t k = rmm_k(rho, d);
+  if (n > kI8CudaCoreMaxRows) {
+    // tensor cores: the decode selection (with x[:, I]), then the dequantising product
+    Carver c(ws);
+    if (k == d) {
+      float* partial = c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
+      if (idx_out != nullptr) {
+        const cudaError_t e = launch_chained(iota_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(d, 256), 1024))),
+                                             dim3(256), 0, s, idx_out, 1, d);
+        if (e != cudaSuccess) return cuda_fail(e, "iota launch");
+      }
+      return int8_tc_product(A, n, lda, Wq, d, m, ldw, nullptr, scale, partial, reinterpret_cast<uint16_t*>(Y), ldy, s);
+    }
+    const int64_t k_pad = round_up(k, 8);
+    double* colsq = c.take<double>(d);
+    int32_t* idx_ws = c.take<int32_t>(k);
+    uint16_t* xpack = c.take<uint16_t>(n * k_pad);
+    float* partial = c.take<float>(static_cast<int64_t>(decode_partial_floats(n, m, k)));
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    if (decode_select_fits(n, d)) {
+      if (rmm_status st = launch_decode_select(A, n, d, lda, k, idx, xpack, k_pad, s)) return st;
+    } else {
+      if (rmm_status st = launch_colsq(A, 1, 0, n, d, lda, false, 0, colsq, s)) return st;
+      if (rmm_status st = launch_select(colsq, 1, d, k, idx, nullptr, s)) return st;
+      if (rmm_status st = pack_columns(A, n, d, lda, idx, k, xpack, k_pad, s)) return st;
+    }
+    return int8_tc_product(xpack, n, k_pad, Wq, k, m, ldw, idx, scale, partial, reinterpret_cast<uint16_t*>(Y), ldy, s);
+  }
   int chunk = 0, chunks = 0;
   i8_plan(n, k, m, &chunk, &chunks);
   if (chunks > 65535) return fail(RMM_ERR_UNSUPPORTED, "too many row chunks");

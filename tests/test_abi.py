@@ -201,7 +201,7 @@ def test_int8_argument_errors(L):
         return L.rmm_linear_int8(A, n, d, lda, W, m, ldw, s, Y, ldy, rho, None, ws, wsb, None)
     assert li8(s=None) == INVALID
     assert li8(rho=0.0) == INVALID
-    assert li8(n=9) == UNSUPPORTED
+    assert li8(n=33) == UNSUPPORTED
     assert li8(m=1020, ldw=1024, ldy=1024) == UNSUPPORTED  # m not a multiple of 8
     assert li8(ldw=1028) == UNSUPPORTED                    # ldw not a multiple of 8
     assert li8() == WORKSPACE
@@ -223,14 +223,14 @@ def test_attention_argument_errors(L):
     assert L.rmm_attention_workspace_bytes(1, 4, 2, 256, 512, 128, 0.5) >= 4 * 256 * 128 * 2
 
 
-@pytest.mark.parametrize("n", [1, 2, 3, 8])
+@pytest.mark.parametrize("n", [1, 2])
 @pytest.mark.parametrize("rho", [1.0, 0.9, 0.5, 0.01])
 def test_int8_plan_fills_at_most_one_wave(L, n, rho):
-    """The int8 GEMV's row chunks, read back from the workspace size (scores, index
-    set and chunks x n x m fp32 partial sums): the grid of 2048-column blocks x
-    chunks fits in one wave of co-resident CTAs (4, 3 or 2 per SM by the row count;
-    148 SMs when no device is visible) while every chunk holds at most 512 kept rows
-    and a multiple of 16."""
+    """The CUDA-core int8 GEMV (one or two activation rows) splits the kept rows into
+    chunks, read back from the workspace size (scores, index set and chunks x n x m
+    fp32 partial sums): the grid of 2048-column blocks x chunks fits in one wave of
+    co-resident CTAs (4 or 3 per SM by the row count; 148 SMs when no device is
+    visible) while every chunk holds at most 512 kept rows and a multiple of 16."""
     d, m = 8192, 28672
     k = L.rmm_k(rho, d)
     ws = L.rmm_linear_int8_workspace_bytes(n, d, m, rho)
@@ -245,3 +245,13 @@ def test_int8_plan_fills_at_most_one_wave(L, n, rho):
     # the chunk length the plan picks is a multiple of 16 covering k in `chunks` pieces
     lens = [ln for ln in range(16, 513, 16) if -(-k // ln) == chunks]
     assert lens, (k, chunks)
+
+
+@pytest.mark.parametrize("n", [3, 8, 32])
+def test_int8_tensor_core_workspace(L, n):
+    """From three activation rows on, int8 weights run on the tensor cores: the
+    workspace holds the scores, the index set, x[:, I] and the fp32 partials of the
+    bf16 decode product's split (the same size as rmm_linear's decode workspace)."""
+    d, m = 8192, 28672
+    for rho in (0.5, 1.0):
+        assert L.rmm_linear_int8_workspace_bytes(n, d, m, rho) == L.rmm_linear_workspace_bytes(n, d, m, rho)

@@ -35,10 +35,12 @@ def int8_parity(A, Wq, s, rho):
     return Y, idx
 
 
-@pytest.mark.parametrize("n", [1, 2, 3, 8])
+@pytest.mark.parametrize("n", [1, 2, 3, 8, 16, 17, 32])
 @pytest.mark.parametrize("rho", [0.5, 0.7, 1.0])
 def test_int8_small_ragged(n, rho):
-    """d and m off the 2048-column block and the 16-row unroll (d = 1000, m = 2056)."""
+    """d and m off the 2048-column block, the 512-column super tile and the 16-row
+    unroll (d = 1000, m = 2056: the last 16-byte int8 chunk holds 8 columns); n = 1, 2
+    on the CUDA cores, n >= 3 on the tensor cores."""
     g = synthetic.rng(37)
     A = synthetic.to_bf16(synthetic.outlier_activations(g, n, 1000, 1.5))
     Wq, s = synthetic.int8_weight(g, 1000, 2056)
@@ -73,10 +75,26 @@ def test_int8_extreme_codes_and_scales_are_exact():
     assert torch.equal(Y.cpu()[0], expect)
 
 
-@pytest.mark.parametrize("n", [1, 8])
+@pytest.mark.parametrize("n", [1, 8, 32])
 def test_int8_70b_mlp_up(n):
     """Llama-3.1-70B MLP-up shape (d = 8192, m = 28672) with int8 weights."""
     g = synthetic.rng(39)
     A = synthetic.to_bf16(synthetic.outlier_activations(g, n, 8192, 1.5))
     Wq, s = synthetic.int8_weight(g, 8192, 28672)
     int8_parity(A, Wq, s, 0.5)
+
+
+def test_int8_tensor_cores_match_the_cuda_core_kernel_row_by_row():
+    """The same weights and rows through both kernels: the tensor-core product of 8
+    rows equals, row by row, the CUDA-core product of each row alone within the
+    parity tolerance (both accumulate in fp32 from exact int8 values)."""
+    g = synthetic.rng(47)
+    A = synthetic.to_bf16(synthetic.outlier_activations(g, 8, 2048, 1.5))
+    Wq, s = synthetic.int8_weight(g, 2048, 4096)
+    Ad, Wd, sd = A.cuda(), Wq.cuda(), s.cuda()
+    Y8 = rmm.linear_int8(Ad, Wd, sd, 1.0)
+    torch.cuda.synchronize()
+    for r in range(8):
+        Y1 = rmm.linear_int8(Ad[r:r + 1].contiguous(), Wd, sd, 1.0)
+        torch.cuda.synchronize()
+        check_close(synthetic.widen(Y8[r:r + 1].cpu()), synthetic.widen(Y1.cpu()), f"row {r}")
