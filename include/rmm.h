@@ -334,8 +334,10 @@ const char* rmm_version(void);
  * Two entry points that exist only so that tests can reach device code no
  * product call exposes on its own; neither is part of the method.
  *
- * rmm_debug_exp2_poly: y_poly[i] = the fused attention's FMA-pipe 2^x (a cubic
- * fitted to 2^f on [0, 1): relative error <= 7.7e-5 for x in [-125, 0], <= 1.6e-4
+ * rmm_debug_exp2_poly: y_poly[i] = the fused attention's FMA-pipe 2^x (x split
+ * into its nearest integer n and f in [-1/2, 1/2], a cubic fitted to 2^f, the
+ * packed-pair code the attention runs: relative error < 7.6e-5 for x in
+ * [-125, 0], <= 1.6e-4
  * on [-126, -125) where the result can fall into the subnormal range, about
  * 2^-126 below -126) and y_exp2f[i] = CUDA's exp2f(x[i]), i < n.  All three are
  * device fp32 buffers.

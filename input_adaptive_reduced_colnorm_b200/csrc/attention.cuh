@@ -52,23 +52,72 @@ __device__ __forceinline__ float attn_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for the half of the weights that do not go to the
-// special-function unit: x = n + f with n = floor(x) and f in [0, 1), 2^f from a
-// cubic fitted (relative-error minimax on [0, 1]) to max relative error 7.7e-5
-// (7.64e-5, at f = 0), far below the bf16 rounding of P; 2^n is added to the
-// exponent field.  That bound holds for x in [-125, 0].  On [-126, -125) the
-// result is a normal float with the same bound except where n = -126 and the
-// cubic is below 1 (f < 1.1e-4): the sum then lands in the subnormal range and
-// the relative error reaches 1.5e-4.  Arguments below -126 give about 2^-126.
-// (Weights that small are 2^-125 of the row's largest weight, 1, and vanish
-// next to it in every sum.)
-__device__ __forceinline__ float attn_exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float n = floorf(x);
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(0.0780965686f, f, 0.2259650975f), f, 0.6958683133f), f, 0.9999235868f);
-  return __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
+// Packed fp32 pairs (sm_100): two keys of a row per instruction.
+__device__ __forceinline__ uint64_t attn_f2(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
 }
+__device__ __forceinline__ float attn_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float attn_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t attn_fma2(uint64_t a, uint64_t b, uint64_t c) {  // a * b + c
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t attn_add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t attn_sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float attn_max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// bf16 pair (lo in the low half), round to nearest
+__device__ __forceinline__ uint32_t attn_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// 2^x on the FMA pipe for two arguments at once, for the share of the weights
+// that does not go to the special-function unit.  x = n + f with n the nearest
+// integer (x + 1.5 * 2^23 rounds it into the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f from a cubic fitted here (relative-error minimax on
+// [-1/2, 1/2], Remez exchange) with maximum relative error 7.49e-5, far below
+// the bf16 rounding of P; n is added to the exponent field (one shift-add per
+// value).  The bound holds for x in [-125, 0] (the fp32 evaluation adds a few
+// 1e-7).  On [-126, -125) the sum can land in the subnormal range where n = -126
+// and the cubic is below 1, and the relative error there reaches 1.5e-4.
+// Arguments are clamped at -126, so anything smaller gives about 2^-126 (weights
+// that small are 2^-125 of the row's largest weight, 1, and vanish next to it).
+constexpr float kAttnExp2C0 = 0.99992805719f;
+constexpr float kAttnExp2C1 = 0.69326096773f;
+constexpr float kAttnExp2C2 = 0.24261112511f;
+constexpr float kAttnExp2C3 = 0.05517166853f;
+
+__device__ __forceinline__ uint64_t attn_exp2_poly2(uint64_t x) {
+  const uint64_t xc = attn_f2(fmaxf(attn_lo(x), -126.f), fmaxf(attn_hi(x), -126.f));
+  const uint64_t magic = attn_f2(12582912.f, 12582912.f);
+  const uint64_t r = attn_add2(xc, magic);              // 1.5 * 2^23 + n
+  const uint64_t f = attn_sub2(xc, attn_sub2(r, magic));  // x - n, exact
+  uint64_t q = attn_fma2(attn_f2(kAttnExp2C3, kAttnExp2C3), f, attn_f2(kAttnExp2C2, kAttnExp2C2));
+  q = attn_fma2(q, f, attn_f2(kAttnExp2C1, kAttnExp2C1));
+  q = attn_fma2(q, f, attn_f2(kAttnExp2C0, kAttnExp2C0));
+  // the low 9 bits of r hold n (two's complement): shifted into the exponent field
+  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(r) << 23);
+  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(r >> 32) << 23);
+  return static_cast<uint64_t>(lo) | (static_cast<uint64_t>(hi) << 32);
+}
+
+// one argument (the masked blocks): the same arithmetic, the same result
+__device__ __forceinline__ float attn_exp2_poly(float x) { return attn_lo(attn_exp2_poly2(attn_f2(x, x))); }
 
 // Elementwise attn_exp2_poly and CUDA's exp2f, for the unit test of the fit
 // (rmm_debug_exp2_poly).
@@ -336,7 +385,8 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait();
         if (fast) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e >> 5][e & 31]));
+          for (int e = 0; e < 32; ++e)
+            mx8[e & 7] = attn_max3(mx8[e & 7], __uint_as_float(v[0][e]), __uint_as_float(v[1][e]));
         } else {
 #pragma unroll
           for (int e = 0; e < 64; ++e) {
@@ -358,9 +408,10 @@ __global__ void __launch_bounds__(320, 1)
       const float corr = grow ? attn_exp2(m_run - m_use) : 1.f;  // 0 for the first block
       // pass 2: P = exp2(s * scale_log2 - m) packed as bf16 pairs into the first 64
       // columns of S (keys 64h .. 64h+63 become columns 32h .. 32h+31, already read)
-      float sum8[8];
+      uint64_t sum2[4];  // fp32 pairs: eight independent partial sums
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
+      for (int i = 0; i < 4; ++i) sum2[i] = 0ull;
+      const uint64_t sc2 = attn_f2(p.scale_log2, p.scale_log2), nm2 = attn_f2(-m_use, -m_use);
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t pk[32];
         uint32_t vv[2][32];  // half a block per read: two loads, one wait
@@ -371,15 +422,20 @@ __global__ void __launch_bounds__(320, 1)
         for (int cc = 0; cc < 2; ++cc) {
           const int c = 2 * hh + cc;
           const uint32_t (&v)[32] = vv[cc];
-          // even keys on the FMA pipe, odd keys on the special-function unit
           if (full) {
+            // keys 4e, 4e+1 on the FMA pipe (packed pairs), 4e+2, 4e+3 on the
+            // special-function unit; scaling, sums and the polynomial two keys per
+            // instruction
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use));
-              const float x1 = attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use));
-              sum8[e & 7] += x0 + x1;
-              const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
-              pk[cc * 16 + e] = *reinterpret_cast<const uint32_t*>(&t2);
+            for (int e = 0; e < 8; ++e) {
+              const uint64_t xa = attn_fma2(attn_f2(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1])), sc2, nm2);
+              const uint64_t xb =
+                  attn_fma2(attn_f2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])), sc2, nm2);
+              const uint64_t ya = attn_exp2_poly2(xa);
+              const uint64_t yb = attn_f2(attn_exp2(attn_lo(xb)), attn_exp2(attn_hi(xb)));
+              sum2[e & 3] = attn_add2(sum2[e & 3], attn_add2(ya, yb));
+              pk[cc * 16 + 2 * e] = attn_bf16x2(attn_lo(ya), attn_hi(ya));
+              pk[cc * 16 + 2 * e + 1] = attn_bf16x2(attn_lo(yb), attn_hi(yb));
             }
           } else {
 #pragma unroll
@@ -391,15 +447,15 @@ __global__ void __launch_bounds__(320, 1)
               const float x1 = (ka + 1 < p.nk && ka + 1 <= last_key)
                                    ? attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use))
                                    : 0.f;
-              sum8[e & 7] += x0 + x1;
-              const __nv_bfloat162 t2 = __floats2bfloat162_rn(x0, x1);
-              pk[cc * 16 + e] = *reinterpret_cast<const uint32_t*>(&t2);
+              sum2[e & 3] = attn_add2(sum2[e & 3], attn_f2(x0, x1));
+              pk[cc * 16 + e] = attn_bf16x2(x0, x1);
             }
           }
         }
         tmem_st32(s_col + static_cast<uint32_t>(hh * 32), pk);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      const uint64_t s01 = attn_add2(attn_add2(sum2[0], sum2[1]), attn_add2(sum2[2], sum2[3]));
+      const float sum = attn_lo(s01) + attn_hi(s01);
       l_run = l_run * corr + sum;
       m_run = m_new;
       // O *= corr where some row's reference maximum moved; PV(j-1) is complete (it

@@ -14,7 +14,14 @@
 //              MN-major operand layout (a TMA row gather stages only ~7 B/clk/SM
 //              on B200, 16-byte cp.async ~35 B/clk/SM); two threads per kept
 //              row, the next row number prefetched one stage ahead; thread 0
-//              also brings the packed activations x_I with a TMA tile.
+//              also brings the packed activations x_I with a TMA tile.  A
+//              producer never waits for its own copies: cp.async.mbarrier.arrive
+//              counts the thread on the stage's full barrier once its copies have
+//              landed, so all three 64 KB stages can be in flight, and the MMA
+//              thread fences the async proxy after its wait.  (The first version
+//              waited for its copies two stages back and fenced in the producers;
+//              the fence also waits for the copies still in flight, and the
+//              kernel streamed 0.79 of the copy bandwidth instead of 0.92.)
 //   warp 4     allocates TMEM; one thread issues tcgen05.mma (M=128, N, K=16).
 //   warps 5-8  epilogue: tcgen05.ld -> fp32 partial sums in global memory.
 // Work split (stream-K): the (super tile, 64-row k-block) units are cut into
@@ -78,7 +85,6 @@ __device__ __forceinline__ void gemv_for_each_owner(const GemvParams& p, int64_t
 constexpr int kGemvTiles = 4;                  // 128-column MMA tiles per super tile
 constexpr int kGemvCols = 128 * kGemvTiles;    // 512 columns = 1 KB of each kept row per stage
 constexpr int kGemvStages = 3;
-constexpr int kGemvLag = 2;  // cp.async groups a producer keeps in flight before signalling
 
 __device__ __forceinline__ int64_t gemv_unit_begin(int64_t c, int64_t units, int64_t G) { return (c * units) / G; }
 
@@ -86,11 +92,12 @@ __device__ __forceinline__ void cp_async16_z(void* dst, const void* src, uint32_
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// arrive on `bar` once every cp.async this thread issued so far has landed (the
+// arrival is one of the barrier's expected count)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // 32 lanes x 16 consecutive 32-bit columns (thread t: row lane_base + t).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -183,7 +190,6 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
     const int tid = threadIdx.x;
     int stage = 0;
     uint32_t phase = 0;
-    int64_t issued = 0;
     bool ok = true;
     int rows_next[16];
     if (u_begin < u_end) {
@@ -233,27 +239,15 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
         }
         cp_async16_z(dstA + tile * 16384 + a * 8192 + r * 128 + ((cw ^ (r & 7)) << 4), src, bytes);
       }
-      cp_async_commit_group();
-      ++issued;
-      if (issued > kGemvLag) {
-        // the copies of the stage issued kGemvLag groups ago have landed
-        cp_async_wait_group<kGemvLag>();
-        fence_proxy_async_smem();
-        const int s_old = static_cast<int>((issued - 1 - kGemvLag) % kGemvStages);
-        mbar_arrive(&full[s_old]);
-      }
+      cp_async_arrive_noinc(&full[stage]);
       if (++stage == kGemvStages) {
         stage = 0;
         phase ^= 1u;
       }
     }
-    // signal the stages still in flight (also on the abort path, so nothing lands late)
-    cp_async_wait_group<0>();
-    fence_proxy_async_smem();
-    if (ok) {
-      const int64_t first = issued > kGemvLag ? issued - kGemvLag : 0;
-      for (int64_t g = first; g < issued; ++g) mbar_arrive(&full[static_cast<int>(g % kGemvStages)]);
-    }
+    // nothing may land after exit (the abort path leaves copies in flight)
+    cp_async_wait_all();
+    (void)ok;
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -275,6 +269,9 @@ __global__ void __launch_bounds__(288, 1) gemv_kernel(const __grid_constant__ CU
             ok = false;
             break;
           }
+          // the stage's cp.async writes (acquired through the barrier) are ordered
+          // before the MMA's async-proxy reads
+          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
           const uint32_t x0 = smem_u32(sX + stage * X_BYTES);

@@ -240,13 +240,14 @@ __global__ void __launch_bounds__(kI8TcThreads, 1)
   if (warp < PW) {
     // ------------------------------------------------------------ producers
     // lane l covers columns [16 l, 16 l + 16) of the super tile: MMA tile l / 8,
-    // 64-column atom (l / 4) % 2, 16-byte chunks 2 (l % 4) and 2 (l % 4) + 1
+    // 64-column atom (l / 4) % 2, 16-byte bf16 chunks 2 (l % 4) and 2 (l % 4) + 1.
+    // Lanes of the odd atom store their two chunks in the other order, so each
+    // group of 8 lanes writes 8 different 16-byte bank groups per store.
     const int c16 = lane * 16;
     const int tile = lane >> 3, atom = (lane >> 2) & 1, cw = (lane & 3) * 2;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    // kept-row numbers two units ahead, data loads one unit ahead (registers)
     auto rows_of = [&](int64_t u, int (&dst)[RPW]) {
       const int kb = static_cast<int>(u % p.kb_total);
 #pragma unroll
@@ -258,68 +259,75 @@ __global__ void __launch_bounds__(kI8TcThreads, 1)
     // a row starts 16-byte aligned only when the row stride is a multiple of 16
     // bytes (the interface promises 8): otherwise two 8-byte loads per chunk
     const bool rows16 = (p.ldw & 15) == 0;
-    auto load_unit = [&](int64_t u, const int (&rows)[RPW], uint4 (&dst)[RPW]) {
-      const int sup = static_cast<int>(u / p.kb_total);
-      const int col = sup * kGemvCols + c16;
-#pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        dst[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (u < u_end && rows[j] >= 0 && col < p.m) {
-          const int8_t* src = p.W + static_cast<int64_t>(rows[j]) * p.ldw + col;
-          if (col + 16 <= p.m) {
-            if (rows16) {
-              dst[j] = ldg_nc_v4(src);
-            } else {
-              const uint2 a = ldg_nc_u2(src), b = ldg_nc_u2(src + 8);
-              dst[j] = make_uint4(a.x, a.y, b.x, b.y);
-            }
-          } else {  // m is a multiple of 8: the last chunk may hold 8 columns
-            const uint2 h = ldg_nc_u2(src);
-            dst[j] = make_uint4(h.x, h.y, 0u, 0u);
+    auto load_row = [&](int64_t u, int row) -> uint4 {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      const int col = static_cast<int>(u / p.kb_total) * kGemvCols + c16;
+      if (u < u_end && row >= 0 && col < p.m) {
+        const int8_t* src = p.W + static_cast<int64_t>(row) * p.ldw + col;
+        if (col + 16 <= p.m) {
+          if (rows16) {
+            v = ldg_nc_v4(src);
+          } else {
+            const uint2 a = ldg_nc_u2(src), b = ldg_nc_u2(src + 8);
+            v = make_uint4(a.x, a.y, b.x, b.y);
           }
+        } else {  // m is a multiple of 8: the last chunk may hold 8 columns
+          const uint2 h = ldg_nc_u2(src);
+          v = make_uint4(h.x, h.y, 0u, 0u);
         }
       }
+      return v;
     };
-    int rows_n1[RPW], rows_n2[RPW];
-    uint4 next[RPW];
-    rows_of(u_begin, rows_n1);
-    rows_of(u_begin + 1, rows_n2);
-    load_unit(u_begin, rows_n1, next);
-    for (int64_t u = u_begin; u < u_end; ++u) {
-      const int kb = static_cast<int>(u % p.kb_total);
-      uint4 cur[RPW];
+    // Two units of kept rows in flight per thread (buf[0] and buf[1], 64 KB of
+    // int8 per CTA): a row is converted and stored, then its register is
+    // reloaded at once with the same row of the unit two ahead.  Row numbers are
+    // loaded one unit before their data.
+    uint4 buf[2][RPW];
+    int rows_next[RPW];
+    rows_of(u_begin, rows_next);
 #pragma unroll
-      for (int j = 0; j < RPW; ++j) cur[j] = next[j];
+    for (int j = 0; j < RPW; ++j) buf[0][j] = load_row(u_begin, rows_next[j]);
+    rows_of(u_begin + 1, rows_next);
 #pragma unroll
-      for (int j = 0; j < RPW; ++j) rows_n1[j] = rows_n2[j];
-      rows_of(u + 2, rows_n2);
-      load_unit(u + 1, rows_n1, next);
-      int go = 1;
-      if (lane == 0) go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
-      go = __shfl_sync(0xffffffffu, go, 0);
-      if (!go) {
-        ok = false;
-        break;
-      }
-      if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&full[stage], X_BYTES);
-        tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * 64, 0);
-      }
-      uint8_t* dst = sA + stage * A_BYTES + tile * 16384 + atom * 8192;
+    for (int j = 0; j < RPW; ++j) buf[1][j] = load_row(u_begin + 1, rows_next[j]);
+    rows_of(u_begin + 2, rows_next);
+    for (int64_t u0 = u_begin; u0 < u_end && ok; u0 += 2) {
 #pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const int r = warp * RPW + j;  // kept row within the k-block
-        uint4 lo, hi;
-        i8x16_to_bf16(cur[j], lo, hi);
-        *reinterpret_cast<uint4*>(dst + r * 128 + ((cw ^ (r & 7)) << 4)) = lo;
-        *reinterpret_cast<uint4*>(dst + r * 128 + (((cw + 1) ^ (r & 7)) << 4)) = hi;
-      }
-      fence_proxy_async_smem();  // the generic-proxy stores are ordered before the MMA's reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[stage]);
-      if (++stage == kGemvStages) {
-        stage = 0;
-        phase ^= 1u;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int64_t u = u0 + hh;
+        if (u >= u_end) break;
+        const int kb = static_cast<int>(u % p.kb_total);
+        int go = 1;
+        if (lane == 0) go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kDevErrTimeoutProducer) ? 1 : 0;
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        if (threadIdx.x == 0) {
+          mbar_arrive_expect_tx(&full[stage], X_BYTES);
+          tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * 64, 0);
+        }
+        uint8_t* dst = sA + stage * A_BYTES + tile * 16384 + atom * 8192;
+#pragma unroll
+        for (int j = 0; j < RPW; ++j) {
+          const int r = warp * RPW + j;  // kept row within the k-block
+          uint4 lo, hi;
+          i8x16_to_bf16(buf[hh][j], lo, hi);
+          buf[hh][j] = load_row(u + 2, rows_next[j]);
+          const uint4 first = atom ? hi : lo, second = atom ? lo : hi;
+          *reinterpret_cast<uint4*>(dst + r * 128 + (((cw + atom) ^ (r & 7)) << 4)) = first;
+          *reinterpret_cast<uint4*>(dst + r * 128 + (((cw + 1 - atom) ^ (r & 7)) << 4)) = second;
+        }
+        rows_of(u + 3, rows_next);
+        // no proxy fence here: it would wait for this thread's loads still in flight
+        // (two units ahead); the MMA thread fences after its wait instead
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);  // release: the warp's stores, ordered by the syncwarp
+        if (++stage == kGemvStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
     }
     (void)ok;
@@ -344,6 +352,9 @@ __global__ void __launch_bounds__(kI8TcThreads, 1)
             ok = false;
             break;
           }
+          // the producers' generic-proxy stores (acquired through the barrier) are
+          // ordered before the MMA's async-proxy reads of the stage
+          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
           const uint32_t x0 = smem_u32(sX + stage * X_BYTES);
