@@ -218,9 +218,10 @@ rmm_status rmm_pv(const rmm_bf16* P, const rmm_bf16* V, rmm_bf16* O, int64_t bat
  * kernel, S and P kept on chip ("Algorithm Deep-Dive: RMM", Component mapping:
  * QK^T selects head dims by the Q column norm, K gathers them under GQA; Attention
  * vs MLP, Table 16: attention-internal reduction).  I_h is chosen exactly as in
- * rmm_qk; the softmax and the value product are the ordinary ones.  The score
- * product reads Q with the dropped dims of each head zeroed (workspace) and K as
- * it is.
+ * rmm_qk; the softmax and the value product are the ordinary ones.  For
+ * k <= 64 the score product runs over 64 dims: Q[:, I_h] and K_g(h)[:, I_h] are
+ * packed per query head into the workspace (zero past k); for 64 < k < dh it reads
+ * Q with the dropped dims of each head zeroed (workspace) and K as it is.
  *   Q  device bf16 [batch][hq][nq][dh], K / V [batch][hkv][nk][dh], contiguous.
  *   O  device bf16 [batch][hq][nq][dh].
  *   causal = 1: bottom-right aligned (key j visible to query i iff j <= i + nk - nq),

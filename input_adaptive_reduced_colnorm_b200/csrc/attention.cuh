@@ -4,10 +4,12 @@
 // GQA; Attention vs MLP, Table 16: attention-internal reduction):
 //   S_h = scale * Q_h[:, I_h] K_g(h)[:, I_h]^T   (-inf above the causal diagonal)
 //   O_h = softmax_rows(S_h) V_g(h)
-// The index sets come from the column-norm and selection kernels; the score
-// product reads Q with the dropped dims of its head zeroed and K as it is, so it
-// is exactly sum_{t in I_h} Q_h[:, t] K_g(h)[:, t]^T.  The value product is the
-// ordinary one (selecting P's columns would need all of P first).
+// The index sets come from the column-norm and selection kernels.  For k <= 64
+// the score product runs over 64 dims on Q[:, I_h] and K_g(h)[:, I_h] packed per
+// query head (zero past k, kp = 64); otherwise it reads Q with the dropped dims of
+// its head zeroed and K as it is (kp = 128).  Either way it is exactly
+// sum_{t in I_h} Q_h[:, t] K_g(h)[:, t]^T.  The value product is the ordinary one
+// (selecting P's columns would need all of P first).
 //
 // One CTA per (query head, pair of 128-row query tiles), see attn_pp_kernel:
 //   warp 0      TMA: both Q tiles once, then 128-key blocks of K (K-major, 128
@@ -30,7 +32,8 @@ namespace rmm {
 
 struct AttnParams {
   int nq, nk;          // query / key rows of one head
-  int kp;              // score dims staged per tile (the head dim, 128)
+  int kp;              // score dims staged per tile: 128 (Q with the dropped dims zeroed) or 64 (packed)
+  int k_per_item;      // 1: K holds one packed copy per query head (rows item * nk ..), 0: per key head
   int hq, hkv;         // heads (GQA: query head h reads key/value head h / (hq / hkv))
   int items;           // batch * hq
   int m_tiles;         // ceil(nq / 128)
@@ -163,9 +166,16 @@ namespace rmm {
 // one thread execute in issue order: S_X(j+1) is issued after PV_X(j), so it
 // cannot overwrite P_X(j) early, and the commit that signals S_X(j) also covers
 // PV_X(j-1), which makes O_X safe to rescale.
-constexpr int kAttnPPSmem = 2 * kAttnQBytes + 2 * kAttnKBytes + 2 * kAttnVBytes + 1024 + 256;
+constexpr int kAttnPPThreads = 18 * 32;  // TMA warp, MMA warp, 16 softmax warps
+// row-max / row-sum exchange [2 bufs][tile][quarter][half][lane] floats, then the
+// wait results [2 bufs][tile][quarter] ints (two per quarter, the first used)
+constexpr int kAttnXchBytes = 2 * 2 * 4 * 2 * 32 * 4 + 2 * 2 * 4 * 2 * 4;
+constexpr int kAttnPPSmem = 2 * kAttnQBytes + 2 * kAttnKBytes + 2 * kAttnVBytes + kAttnXchBytes + 1024 + 256;
 
-__global__ void __launch_bounds__(320, 1)
+// named barrier of the two warps that share a row quarter of a tile (64 threads)
+__device__ __forceinline__ void attn_pair_sync(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+
+__global__ void __launch_bounds__(kAttnPPThreads, 1)
     attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   extern __shared__ uint8_t app_smem_raw[];
@@ -173,7 +183,8 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sQ = smem;                    // [2 tiles][kAttnQBytes]
   uint8_t* sK = sQ + 2 * kAttnQBytes;    // [2 stages]
   uint8_t* sV = sK + 2 * kAttnKBytes;    // [2 stages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kAttnVBytes);
+  float* s_xch = reinterpret_cast<float*>(sV + 2 * kAttnVBytes);  // kAttnXchBytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kAttnVBytes + kAttnXchBytes);
   uint64_t* q_full = bars;        // 1
   uint64_t* k_full = bars + 1;    // 2 (stages)
   uint64_t* k_empty = bars + 3;   // 2
@@ -198,7 +209,7 @@ __global__ void __launch_bounds__(320, 1)
   nkb_t[1] = attn_key_blocks(p, m0 + kAttnTile < p.nq ? m0 + kAttnTile : m0);
   const int nkb = nkb_t[0] > nkb_t[1] ? nkb_t[0] : nkb_t[1];
   const int qrow0 = item * p.nq + m0;
-  const int krow0 = (b * p.hkv + g) * p.nk;
+  const int krow0 = (p.k_per_item ? item : b * p.hkv + g) * p.nk;
   const int vrow0 = (b * p.hkv + g) * p.nk;
   const uint32_t k_bytes = static_cast<uint32_t>(p.kp) * kAttnTile * 2;
 
@@ -210,7 +221,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 256);  // both softmax warpgroups of the tile
       mbar_init(&pv_done[s], 1);
     }
     mbar_init(drain, 1);
@@ -303,7 +314,7 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(&s_full[t]);
         return true;
       };
-      // O_t += P_t(j) V(j), P_t(j) in the first 64 columns of S_t
+      // O_t += P_t(j) V(j), P_t(j) in columns [0, 32) (keys 0-63) and [64, 96) (keys 64-127) of S_t
       auto issue_pv = [&](int t, int j) -> bool {
         const int s = j & 1;
         const uint32_t use = static_cast<uint32_t>(j >> 1);
@@ -315,11 +326,12 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t boff = static_cast<uint32_t>((kk >> 2) * 16384 + (kk & 3) * 2048);
           umma_bf16_ts(tmem_base + 256u + static_cast<uint32_t>(t * 128),
-                       tmem_base + static_cast<uint32_t>(t * 128 + kk * 8), make_sw128_desc(v0 + boff, 8192, 1024),
+                       tmem_base + static_cast<uint32_t>(t * 128 + (kk >> 2) * 64 + (kk & 3) * 8),
+                       make_sw128_desc(v0 + boff, 8192, 1024),
                        idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
         if (t == 1) umma_commit(&v_empty[s]);
-        if (j == nkb_t[t] - 1) umma_commit(&pv_done[t]);
+        if (j == (t ? nkb_t[1] : nkb_t[0]) - 1) umma_commit(&pv_done[t]);
         return true;
       };
       if (ok && nkb_t[0] > 0) ok = issue_s(0, 0);
@@ -344,44 +356,67 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (tile X) + epilogue
+    // Two threads per query row: warps 2-9 serve tile A, 10-17 tile B; within a
+    // tile the first four warps take keys 0-63 of every block (hw = 0), the next
+    // four keys 64-127 (hw = 1).  Warp w reads tensor-memory lanes 32 (w % 4) ..
+    // 32 (w % 4) + 31, so the two warps of a row quarter share their rows; they
+    // exchange the block's row maximum (and at the end the row sum) through
+    // shared memory at a 64-thread named barrier.
     auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
       int got = 1;
       if (lane == 0) got = mbar_wait(bar, parity, abort_flag, kDevErrTimeoutEpilogue, 32) ? 1 : 0;
       return __shfl_sync(0xffffffffu, got, 0) != 0;
     };
-    const int X = (warp - 2) >> 2;  // 0: tile A (warps 2-5), 1: tile B (warps 6-9)
+    const int w = warp - 2;
+    const int X = w >> 3;         // tile
+    const int hw = (w >> 2) & 1;  // key half of each block
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    const int pair_bar = 1 + X * 4 + quarter;  // named barrier 1..8
+    float* xch = s_xch + (X * 4 + quarter) * 64 + lane;  // + buf * 512 + half * 32
+    volatile int* got_flag = reinterpret_cast<volatile int*>(s_xch + 1024) + (X * 4 + quarter) * 2;  // + buf * 16 + half
     const int64_t qi = static_cast<int64_t>(m0) + X * kAttnTile + r;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t s_col = lane_base + static_cast<uint32_t>(X * 128);
-    const uint32_t o_col = lane_base + 256u + static_cast<uint32_t>(X * 128);
-    const int64_t last_key = p.causal ? qi + p.causal_off : static_cast<int64_t>(p.nk) - 1;
-    const int my_nkb = nkb_t[X];
-    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t s_col = lane_base + static_cast<uint32_t>(X * 128 + hw * 64);  // this thread's 64 scores
+    const uint32_t o_col = lane_base + 256u + static_cast<uint32_t>(X * 128 + hw * 64);  // its 64 columns of O
+    // the row's last visible key, clamped to [-1, nk - 1] (32-bit from here on)
+    int64_t last64 = p.causal ? qi + p.causal_off : static_cast<int64_t>(p.nk) - 1;
+    last64 = last64 < -1 ? -1 : (last64 > p.nk - 1 ? p.nk - 1 : last64);
+    const int last_key = static_cast<int>(last64);
+    const int my_nkb = X ? nkb_t[1] : nkb_t[0];
+    float m_run = -INFINITY, l_half = 0.f;
     bool ok = true;
     for (int j = 0; j < my_nkb && ok; ++j) {
-      if (!warp_wait(&s_full[X], static_cast<uint32_t>(j) & 1u)) {
+      // The hw = 0 warp waits (bounded) for S(j) and passes the outcome to its
+      // partner at a named barrier, so both warps of the pair take the same path
+      // and meet at every named barrier the same number of times (a bar.sync has
+      // no time limit).  The flag of a block is rewritten only two blocks later,
+      // after barriers the partner passes only once it has read it.
+      volatile int* gf = got_flag + (j & 1) * 16;
+      if (hw == 0) {
+        const bool got = warp_wait(&s_full[X], static_cast<uint32_t>(j) & 1u);
+        if (lane == 0) gf[0] = got ? 1 : 0;
+      }
+      attn_pair_sync(pair_bar);
+      if (gf[0] == 0) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int64_t key0 = static_cast<int64_t>(j) * kAttnTile;
-      // every key of the block visible to this row: no masking work
-      const bool full = (key0 + kAttnTile - 1 <= last_key) && (key0 + kAttnTile <= p.nk);
-      // pass 1: the row maximum of the block (scaled, masked), eight independent
-      // chains.  tcgen05.ld is warp-collective (.sync.aligned): every lane
-      // executes the same loads, outside any branch on row-dependent values; only
-      // the arithmetic on the loaded values depends on whether this row sees the
-      // whole block
+      const int key0 = j * kAttnTile + hw * 64;  // this thread's first key of the block
+      // every one of this thread's keys visible to the row: no masking work
+      const bool full = key0 + 63 <= last_key;
+      // pass 1: the maximum of this thread's 64 scores (scaled, masked), eight
+      // independent chains.  tcgen05.ld is warp-collective (.sync.aligned): every
+      // lane executes the same loads, outside any branch on row-dependent values.
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
       const bool fast = full && p.scale_log2 > 0.f;
-      for (int hh = 0; hh < 2; ++hh) {  // half a block per read: two loads, one wait
+      {
         uint32_t v[2][32];
-        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64), v[0]);
-        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64 + 32), v[1]);
+        tmem_ld32(s_col, v[0]);
+        tmem_ld32(s_col + 32u, v[1]);
         tmem_ld_wait();
         if (fast) {
 #pragma unroll
@@ -389,79 +424,79 @@ __global__ void __launch_bounds__(320, 1)
             mx8[e & 7] = attn_max3(mx8[e & 7], __uint_as_float(v[0][e]), __uint_as_float(v[1][e]));
         } else {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const int64_t key = key0 + hh * 64 + e;
-            if (key < p.nk && key <= last_key)
+          for (int e = 0; e < 64; ++e)
+            if (key0 + e <= last_key)
               mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e >> 5][e & 31]) * p.scale_log2);
-          }
         }
       }
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       if (fast) mx *= p.scale_log2;
+      // the row maximum: exchange with the other half (double-buffered by block
+      // parity, so a value is never overwritten before the partner has read it).
+      // The barrier also orders the partner's score loads before this thread's
+      // stores of P below.
+      float* xb = xch + (j & 1) * 512;
+      xb[hw * 32] = mx;
+      tc_fence_before();
+      attn_pair_sync(pair_bar);
+      tc_fence_after();
+      mx = fmaxf(mx, xb[(hw ^ 1) * 32]);
       // the reference maximum moves only when the row's maximum grows by more than
       // kAttnRescaleLog2 (log2 units): the weights exp2(s - m) then stay below 2^8,
-      // and O and l are rescaled rarely instead of at almost every block
+      // and O and l are rescaled rarely instead of at almost every block.  Both
+      // halves of a row compute the same m and corr.
       const bool grow = (m_run == -INFINITY) || (mx > m_run + kAttnRescaleLog2);
       const float m_new = grow ? fmaxf(m_run, mx) : m_run;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float corr = grow ? attn_exp2(m_run - m_use) : 1.f;  // 0 for the first block
-      // pass 2: P = exp2(s * scale_log2 - m) packed as bf16 pairs into the first 64
-      // columns of S (keys 64h .. 64h+63 become columns 32h .. 32h+31, already read)
-      uint64_t sum2[4];  // fp32 pairs: eight independent partial sums
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sum2[i] = 0ull;
+      // pass 2: P = exp2(s * scale_log2 - m) as bf16 pairs; keys 64 hw .. 64 hw + 63
+      // go to columns 64 hw .. 64 hw + 31 of S (this thread's own scores, read)
+      uint64_t sum2[2];  // fp32 pairs: four independent partial sums
+      sum2[0] = sum2[1] = 0ull;
       const uint64_t sc2 = attn_f2(p.scale_log2, p.scale_log2), nm2 = attn_f2(-m_use, -m_use);
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t pk[32];
-        uint32_t vv[2][32];  // half a block per read: two loads, one wait
-        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64), vv[0]);
-        tmem_ld32(s_col + static_cast<uint32_t>(hh * 64 + 32), vv[1]);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t vc[32];
+        tmem_ld32(s_col + static_cast<uint32_t>(h * 32), vc);
         tmem_ld_wait();
+        uint32_t pk[16];
+        if (full) {
+          // keys 4e, 4e+1 on the FMA pipe (packed pairs), 4e+2, 4e+3 on the
+          // special-function unit; scaling, sums and the polynomial two keys per
+          // instruction
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * hh + cc;
-          const uint32_t (&v)[32] = vv[cc];
-          if (full) {
-            // keys 4e, 4e+1 on the FMA pipe (packed pairs), 4e+2, 4e+3 on the
-            // special-function unit; scaling, sums and the polynomial two keys per
-            // instruction
+          for (int e = 0; e < 8; ++e) {
+            const uint64_t xa =
+                attn_fma2(attn_f2(__uint_as_float(vc[4 * e]), __uint_as_float(vc[4 * e + 1])), sc2, nm2);
+            const uint64_t xb2 =
+                attn_fma2(attn_f2(__uint_as_float(vc[4 * e + 2]), __uint_as_float(vc[4 * e + 3])), sc2, nm2);
+            const uint64_t ya = attn_exp2_poly2(xa);
+            const uint64_t yb = attn_f2(attn_exp2(attn_lo(xb2)), attn_exp2(attn_hi(xb2)));
+            sum2[e & 1] = attn_add2(sum2[e & 1], attn_add2(ya, yb));
+            pk[2 * e] = attn_bf16x2(attn_lo(ya), attn_hi(ya));
+            pk[2 * e + 1] = attn_bf16x2(attn_lo(yb), attn_hi(yb));
+          }
+        } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint64_t xa = attn_fma2(attn_f2(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1])), sc2, nm2);
-              const uint64_t xb =
-                  attn_fma2(attn_f2(__uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])), sc2, nm2);
-              const uint64_t ya = attn_exp2_poly2(xa);
-              const uint64_t yb = attn_f2(attn_exp2(attn_lo(xb)), attn_exp2(attn_hi(xb)));
-              sum2[e & 3] = attn_add2(sum2[e & 3], attn_add2(ya, yb));
-              pk[cc * 16 + 2 * e] = attn_bf16x2(attn_lo(ya), attn_hi(ya));
-              pk[cc * 16 + 2 * e + 1] = attn_bf16x2(attn_lo(yb), attn_hi(yb));
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int64_t ka = key0 + c * 32 + 2 * e;
-              const float x0 = (ka < p.nk && ka <= last_key)
-                                   ? attn_exp2_poly(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use))
-                                   : 0.f;
-              const float x1 = (ka + 1 < p.nk && ka + 1 <= last_key)
-                                   ? attn_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use))
-                                   : 0.f;
-              sum2[e & 3] = attn_add2(sum2[e & 3], attn_f2(x0, x1));
-              pk[cc * 16 + e] = attn_bf16x2(x0, x1);
-            }
+          for (int e = 0; e < 16; ++e) {
+            const int ka = key0 + h * 32 + 2 * e;
+            const float x0 =
+                (ka <= last_key) ? attn_exp2_poly(fmaf(__uint_as_float(vc[2 * e]), p.scale_log2, -m_use)) : 0.f;
+            const float x1 =
+                (ka + 1 <= last_key) ? attn_exp2(fmaf(__uint_as_float(vc[2 * e + 1]), p.scale_log2, -m_use)) : 0.f;
+            sum2[e & 1] = attn_add2(sum2[e & 1], attn_f2(x0, x1));
+            pk[e] = attn_bf16x2(x0, x1);
           }
         }
-        tmem_st32(s_col + static_cast<uint32_t>(hh * 32), pk);
+        tmem_st16(s_col + static_cast<uint32_t>(h * 16), pk);
       }
-      const uint64_t s01 = attn_add2(attn_add2(sum2[0], sum2[1]), attn_add2(sum2[2], sum2[3]));
-      const float sum = attn_lo(s01) + attn_hi(s01);
-      l_run = l_run * corr + sum;
+      const uint64_t s01 = attn_add2(sum2[0], sum2[1]);
+      l_half = l_half * corr + (attn_lo(s01) + attn_hi(s01));
       m_run = m_new;
-      // O *= corr where some row's reference maximum moved; PV(j-1) is complete (it
-      // was issued before S(j))
+      // O *= corr where some row's reference maximum moved (this thread's 64
+      // columns); PV(j-1) is complete (it was issued before S(j))
       if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
           tmem_ld32(o_col + static_cast<uint32_t>(c * 32), o);
           tmem_ld_wait();
@@ -474,12 +509,16 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(&p_full[X]);
     }
-    // epilogue: O / l as bf16
+    // epilogue: O / l as bf16, l = the sum of both halves of the row (both warps of
+    // the pair leave the loop after the same block, see the wait flag)
+    xch[(my_nkb & 1) * 512 + hw * 32] = l_half;
+    attn_pair_sync(pair_bar);
+    const float l_row = l_half + xch[(my_nkb & 1) * 512 + (hw ^ 1) * 32];
     if (ok && my_nkb > 0 && warp_wait(&pv_done[X], 0u)) {
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint16_t* orow = p.O + (static_cast<int64_t>(item) * p.nq + qi) * 128;
-      for (int c = 0; c < 4; ++c) {
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+      uint16_t* orow = p.O + (static_cast<int64_t>(item) * p.nq + qi) * 128 + hw * 64;
+      for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
         tmem_ld32(o_col + static_cast<uint32_t>(c * 32), v);
         tmem_ld_wait();

@@ -36,12 +36,17 @@
 // 16-byte cp.async straight into the 128-byte-swizzled MN-major stage (a TMA
 // copy per row or per four rows stages only ~7-8 B/clk/SM on B200, 16-byte
 // cp.async ~35, and the pair needs ~22 B/clk/SM of B at full tensor rate).
-// Each warp keeps two k-blocks of copies in flight; when a k-block has landed
-// its lanes fence the async proxy and lane 0 arrives, with cluster-scope
-// release, on the even CTA's full barrier, which then counts the A bytes of
-// both CTAs (TMA) and the eight B warps of the pair.  The MMA thread waits on
-// it with cluster-scope acquire.  Kept indices t >= k and columns past N read
-// as zeros.
+// A B thread never waits for its own copies: cp.async.mbarrier.arrive counts
+// it on a barrier once they have landed, so every stage of the ring can be in
+// flight.  On the even CTA that barrier is the MMA's full barrier itself (it
+// counts the A bytes of both CTAs, this CTA's 128 B threads and one forwarder);
+// on the odd CTA it is a local one (bfull), and one thread (warp 1, idle there
+// otherwise) waits on it, fences the async proxy and arrives on the even CTA's
+// full barrier with cluster-scope release.  The MMA thread waits with
+// cluster-scope acquire and fences the async proxy for its own CTA's copies.
+// (A proxy fence in the copying threads themselves waits for their copies still
+// in flight: the first version fenced there and kept about one stage in
+// flight.)  Kept indices t >= k and columns past N read as zeros.
 // Work split as in the one-CTA kernel, with pairs as the workers: whole tiles
 // round-robin, then the tiles of a partial last wave cut into two 256 x 128
 // pieces.  Every wait is bounded; the CTAs meet at a cluster barrier before
@@ -59,20 +64,20 @@ struct PairCfg {
   static constexpr int EPI_BYTES = 4 * 2 * 4096;
   static constexpr int TMEM_COLS = 512;          // two 256-column accumulators
   static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + EPI_BYTES + 1024 + 256;
-  static_assert(8 * (2 * STAGES + 5) + 8 <= 256, "barrier area");
+  static_assert(8 * (3 * STAGES + 5) + 8 <= 256, "barrier area");
 };
 
 constexpr int kPairGatherWarps = 4;  // B producer warps per CTA with GATHER (warps 6-9)
-constexpr int kPairGatherLag = 2;    // k-blocks of copies a B warp keeps in flight before arriving
 
 __device__ __forceinline__ void pair_cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void pair_cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void pair_cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// arrive on `bar` once every cp.async this thread issued so far has landed (the
+// arrival is one of the barrier's expected count)
+__device__ __forceinline__ void pair_cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void pair_cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Pair tile order: batch item, then N tile, then 256-row M tile fastest.
 __device__ __forceinline__ void pair_tile_coords(const GemmParams& p, int tile, int& b, int& m0, int& nt) {
@@ -100,7 +105,8 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;  // used in the even CTA
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* bfull = drain + 1;  // GATHER, odd CTA: its B threads' copies of a stage have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bfull + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,9 +115,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
   const int npairs = static_cast<int>(gridDim.x >> 1);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // GATHER: the A bytes of both CTAs (one expect_tx arrival) and the B warps of both CTAs
-      mbar_init(&full[s], GATHER ? 1 + 2 * kPairGatherWarps : 1);
+      // GATHER: the A bytes of both CTAs (one expect_tx arrival), every B thread of
+      // this CTA (its copies landed) and the odd CTA's forwarding thread
+      mbar_init(&full[s], GATHER ? 1 + 32 * kPairGatherWarps + 1 : 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&bfull[s], 32 * kPairGatherWarps);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -212,6 +220,9 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             ok = false;
             break;
           }
+          // GATHER: this CTA's cp.async writes of the stage (acquired through the
+          // barrier) are ordered before the MMA's async-proxy reads
+          if (GATHER) fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
@@ -237,6 +248,30 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
+    } else if (GATHER && rank == 1 && lane == 0) {
+      // ------------------------------------------------------------ forwarder (odd CTA)
+      // The B threads of this CTA count their copies on the local bfull barrier
+      // (cp.async.mbarrier.arrive reaches this CTA's barriers only); once a
+      // stage's copies have all landed this thread fences the async proxy and
+      // passes the stage on to the even CTA's full barrier (cluster release).
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      GemmWork wk;
+      for (int it = 0; ok && gemm_work<256>(p, total_tiles, it, wk, npairs, pair); ++it) {
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&bfull[stage], phase, abort_flag, kDevErrTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive_cluster(full_even + 8u * static_cast<uint32_t>(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
     }
     __syncwarp();
   } else if (GATHER && warp >= 6) {
@@ -244,11 +279,11 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
     // warp g copies kept rows 16g .. 16g+15 of each k-block: a row's run is cpr
     // 16-byte chunks (cpr = 16, or 8 for a 64-column half), rpi = 32 / cpr rows
     // per warp instruction; each lane holds the row numbers of its rows for the
-    // current and the next k-block (loaded one k-block ahead, no shuffles).
+    // current and the next k-block (loaded one k-block ahead, no shuffles; four
+    // k-blocks ahead measured no faster).
     const int g = warp - 6;
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t issued = 0;
     bool ok = true;
     int rows_next[8];
     auto load_rows = [&](int kb, int rpi, int (&dst)[8]) {
@@ -305,31 +340,19 @@ __global__ void __launch_bounds__(GATHER ? 320 : 192, 1)
             pair_cp_async16(dst, src, bytes);
           }
         }
-        pair_cp_async_commit();
-        ++issued;
-        if (issued > kPairGatherLag) {
-          // the copies of the k-block issued kPairGatherLag groups ago have landed
-          pair_cp_async_wait<kPairGatherLag>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          const uint32_t s_old = (issued - 1 - kPairGatherLag) % STAGES;
-          if (lane == 0) mbar_arrive_cluster(full_even + 8u * s_old);
-        }
+        // this thread is counted on the stage once its copies have landed: on the
+        // even CTA straight on the MMA's full barrier, on the odd CTA on bfull (the
+        // forwarder passes it on); no waits here, so every stage can be in flight
+        pair_cp_async_arrive_noinc(rank == 0 ? &full[stage] : &bfull[stage]);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    // the k-blocks still in flight: land them (also on the abort path, so nothing
-    // lands after exit) and, unless aborting, signal them
-    pair_cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (ok && lane == 0) {
-      const uint32_t first = issued > kPairGatherLag ? issued - kPairGatherLag : 0u;
-      for (uint32_t q = first; q < issued; ++q) mbar_arrive_cluster(full_even + 8u * (q % STAGES));
-    }
+    // nothing may land after exit (the abort path leaves copies in flight)
+    pair_cp_async_wait_all();
+    (void)ok;
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;

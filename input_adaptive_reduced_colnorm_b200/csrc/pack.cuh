@@ -32,11 +32,23 @@ struct PackParams {
   int64_t causal_off;
 };
 
+// first element of batch item b's source matrix (32-bit division when it fits)
+__device__ __forceinline__ const uint16_t* pack_item_base(const PackParams& p, int64_t b) {
+  if (b < (1LL << 31) && p.g_outer < (1LL << 31) && p.g_inner < (1LL << 31)) {
+    const uint32_t b32 = static_cast<uint32_t>(b), go = static_cast<uint32_t>(p.g_outer);
+    const uint32_t outer = b32 / go, inner = (b32 - outer * go) / static_cast<uint32_t>(p.g_inner);
+    return p.src + static_cast<int64_t>(outer) * p.s_outer + static_cast<int64_t>(inner) * p.s_inner;
+  }
+  return p.src + (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
+}
+
 __device__ __forceinline__ const uint16_t* pack_src_row(const PackParams& p, int64_t r, int64_t& b, int64_t& i) {
-  b = r / p.rows;
+  if (r < (1LL << 31) && p.rows < (1LL << 31))
+    b = static_cast<uint32_t>(r) / static_cast<uint32_t>(p.rows);
+  else
+    b = r / p.rows;
   i = r - b * p.rows;
-  const int64_t item = (b / p.g_outer) * p.s_outer + ((b % p.g_outer) / p.g_inner) * p.s_inner;
-  return p.src + item + i * p.src_ld;
+  return pack_item_base(p, b) + i * p.src_ld;
 }
 
 __device__ __forceinline__ uint4 pack_gather8(const PackParams& p, const uint16_t* row, const int32_t* idx, int64_t t0,
@@ -249,14 +261,29 @@ __global__ void __launch_bounds__(256) pack_short_rows_kernel(const PackParams p
   for (int64_t r0 = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * R; r0 < total;
        r0 += warps * R) {
     uint32_t out[R][PG];
+    // batch item and row of r0 (the divisions once per R rows, 32-bit when the
+    // sizes allow); the next rows step through them
+    int64_t b, i;
+    if (total < (1LL << 31)) {
+      b = static_cast<uint32_t>(r0) / static_cast<uint32_t>(p.rows);
+      i = r0 - b * p.rows;
+    } else {
+      b = r0 / p.rows;
+      i = r0 - b * p.rows;
+    }
+    const uint16_t* item_base = pack_item_base(p, b);
 #pragma unroll
     for (int u = 0; u < R; ++u) {
       const int64_t row = r0 + u;
 #pragma unroll
       for (int q = 0; q < PG; ++q) out[u][q] = 0u;
       if (row >= total) continue;
-      int64_t b, i;
-      const uint16_t* src = pack_src_row(p, row, b, i);
+      if (u > 0 && ++i == p.rows) {
+        ++b;
+        i = 0;
+        item_base = pack_item_base(p, b);
+      }
+      const uint16_t* src = item_base + i * p.src_ld;
       if (b != cur_b) {  // this batch item's kept columns (0xFFFF past k: padding)
 #pragma unroll
         for (int q = 0; q < PG; ++q) {
@@ -283,6 +310,70 @@ __global__ void __launch_bounds__(256) pack_short_rows_kernel(const PackParams p
       for (int q = 0; q < PG; ++q) {
         const int t2 = q * 32 + lane;
         if (t2 < pairs) dst[t2] = out[u][q];
+      }
+    }
+  }
+}
+
+// Narrow rows (d a power of two from 64 to 256, no causal mask, rows per batch
+// item a multiple of 8): each warp stages 8 consecutive rows with 16-byte loads,
+// all in flight at once, into its shared-memory slice, then lane l writes the
+// column pairs l, l + 32, ... of each packed row from there.  (One row in flight
+// per warp left the 131072-row packs of the attention's 64-dim score product
+// latency-bound.)  The kept-index pairs of the current batch item stay in
+// registers (k_pad <= 256).
+template <int D>
+__global__ void __launch_bounds__(256) pack_narrow_rows_kernel(const PackParams p) {
+  wait_prior_kernels();
+  constexpr int RW = 8;            // rows per warp step
+  constexpr int VPR = D / 8;       // 16-byte vectors per row
+  constexpr int VPL = RW * VPR / 32;  // vectors per lane per step
+  constexpr int PG = 4;            // pair groups per lane: k_pad <= 256
+  __shared__ __align__(16) uint16_t pn_buf[8][RW][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint16_t (*buf)[D] = pn_buf[warp];
+  const int64_t steps = p.batch * p.rows / RW;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * 8;
+  const int pairs = static_cast<int>(p.k_pad / 2);
+  int64_t cur_b = -1;
+  uint32_t j0[PG], j1[PG];
+  for (int64_t st = static_cast<int64_t>(blockIdx.x) * 8 + warp; st < steps; st += wstride) {
+    const int64_t r0 = st * RW;
+    int64_t b, i;
+    const uint16_t* src = pack_src_row(p, r0, b, i);  // the step's 8 rows share their batch item
+    uint4 v[VPL];
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      const int vi = q * 32 + lane;
+      v[q] = ldg_nc_v4(src + static_cast<int64_t>(vi / VPR) * p.src_ld + (vi % VPR) * 8);
+    }
+    if (b != cur_b) {  // this batch item's kept columns (0xFFFF past k: padding)
+#pragma unroll
+      for (int q = 0; q < PG; ++q) {
+        const int t = 2 * (q * 32 + lane);
+        j0[q] = (t < p.k) ? static_cast<uint32_t>(__ldg(p.idx + b * p.k + t)) : 0xFFFFu;
+        j1[q] = (t + 1 < p.k) ? static_cast<uint32_t>(__ldg(p.idx + b * p.k + t + 1)) : 0xFFFFu;
+      }
+      cur_b = b;
+    }
+    __syncwarp();  // the previous step's gathers from buf are done
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      const int vi = q * 32 + lane;
+      *reinterpret_cast<uint4*>(&buf[vi / VPR][(vi % VPR) * 8]) = v[q];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < RW; ++u) {
+      uint32_t* dst = reinterpret_cast<uint32_t*>(p.dst + (r0 + u) * p.k_pad);
+#pragma unroll
+      for (int q = 0; q < PG; ++q) {
+        const int t2 = q * 32 + lane;
+        if (t2 < pairs) {
+          const uint32_t a = (j0[q] < static_cast<uint32_t>(D)) ? buf[u][j0[q]] : 0u;
+          const uint32_t c = (j1[q] < static_cast<uint32_t>(D)) ? buf[u][j1[q]] : 0u;
+          dst[t2] = a | (c << 16);
+        }
       }
     }
   }

@@ -377,7 +377,16 @@ rmm_status launch_pack(const PackParams& p, cudaStream_t s) {
   const int64_t rows = p.batch * p.rows;
   const int64_t d_round = round_up(p.d, 8);
   cudaError_t e;
-  if (p.d <= 512 && p.k_pad <= 256 && p.k_pad % 2 == 0) {
+  const bool narrow = (p.d == 64 || p.d == 128 || p.d == 256) && p.src_ld % 8 == 0 && p.k_pad <= 256 &&
+                      p.k_pad % 2 == 0 && !p.causal && p.rows % 8 == 0 && p.d <= p.src_ld &&
+                      (p.batch == 1 || (p.s_outer % 8 == 0 && p.s_inner % 8 == 0));
+  if (narrow && rows >= 8192) {
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(rows / 8, 8), 6LL * num_sms()));
+    auto kern = (p.d == 64) ? pack_narrow_rows_kernel<64> : (p.d == 128) ? pack_narrow_rows_kernel<128>
+                                                                         : pack_narrow_rows_kernel<256>;
+    e = launch_chained(kern, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p);
+    if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  } else if (p.d <= 512 && p.k_pad <= 256 && p.k_pad % 2 == 0) {
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(ceil_div(rows, 8 * 4), 8LL * num_sms()));
     e = launch_chained(pack_short_rows_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, s, p);
     if (e != cudaSuccess) return cuda_fail(e, "pack launch");
@@ -697,17 +706,23 @@ int64_t rmm_k(double rho, int64_t d) {
 
 namespace {
 // Workspace of rmm_attention (rho < 1): scores, index sets, keep bytes and Q with
-// the dropped dims zeroed.  (Packing Q[:, I] and K[:, I] per query head to 64 dims
-// halves the score MMA, but while the fused kernel is bound by its softmax the
-// two packs cost more than they save, so K is read as is.)
+// the dropped dims zeroed for 64 < k < 128; for k <= 64, Q[:, I_h] and
+// K_g(h)[:, I_h] packed to 64 dims per query head, so the score MMA runs over 64
+// dims instead of 128 (the kernel's MMAs are bound by their shared-memory operand
+// reads, so halving the score product's K shortens it).
+constexpr int64_t kAttnPackedDims = 64;
 size_t attention_bytes(int64_t items, int64_t nq, int64_t nk, int64_t dh, int64_t k) {
-  (void)nk;
   if (k == dh) return 0;
   Carver c(nullptr);
   c.take<double>(items * dh);
   c.take<int32_t>(items * k);
-  c.take<uint8_t>(items * dh);
-  c.take<uint16_t>(items * nq * dh);
+  if (k <= kAttnPackedDims) {
+    c.take<uint16_t>(items * nq * kAttnPackedDims);
+    c.take<uint16_t>(items * nk * kAttnPackedDims);
+  } else {
+    c.take<uint8_t>(items * dh);
+    c.take<uint16_t>(items * nq * dh);
+  }
   return c.bytes();
 }
 }  // namespace
@@ -761,7 +776,47 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
   const uint16_t* qsrc = Q;
   const uint16_t* ksrc = K;
   ap.kp = 128;
-  if (k < dh) {
+  ap.k_per_item = 0;
+  if (k < dh && k <= kAttnPackedDims) {
+    // scores and selection on Q, then Q[:, I_h] and K_g(h)[:, I_h] packed to 64
+    // dims (zero past k) for every query head
+    Carver c(ws);
+    double* colsq = c.take<double>(items * dh);
+    int32_t* idx_ws = c.take<int32_t>(items * k);
+    int32_t* idx = idx_out ? idx_out : idx_ws;
+    uint16_t* qp = c.take<uint16_t>(items * nq * kAttnPackedDims);
+    uint16_t* kpk = c.take<uint16_t>(items * nk * kAttnPackedDims);
+    if (rmm_status st = launch_colsq(Q, items, nq * dh, nq, dh, dh, false, 0, colsq, s)) return st;
+    if (rmm_status st = launch_select(colsq, items, dh, k, idx, nullptr, s)) return st;
+    PackParams pq{};
+    pq.src = Q;
+    pq.src_ld = dh;
+    pq.rows = nq;
+    pq.d = dh;
+    pq.g_outer = 1;
+    pq.g_inner = 1;
+    pq.s_outer = nq * dh;
+    pq.s_inner = 0;
+    pq.idx = idx;
+    pq.k = k;
+    pq.k_pad = kAttnPackedDims;
+    pq.dst = qp;
+    pq.batch = items;
+    if (rmm_status st = launch_pack(pq, s)) return st;
+    PackParams pk = pq;  // query head b * hq + h reads key head b * hkv + h / (hq / hkv)
+    pk.src = K;
+    pk.rows = nk;
+    pk.g_outer = hq;
+    pk.s_outer = hkv * nk * dh;
+    pk.g_inner = hq / hkv;
+    pk.s_inner = nk * dh;
+    pk.dst = kpk;
+    if (rmm_status st = launch_pack(pk, s)) return st;
+    qsrc = qp;
+    ksrc = kpk;
+    ap.kp = static_cast<int>(kAttnPackedDims);
+    ap.k_per_item = 1;
+  } else if (k < dh) {
     Carver c(ws);
     double* colsq = c.take<double>(items * dh);
     int32_t* idx_ws = c.take<int32_t>(items * k);
@@ -790,11 +845,12 @@ rmm_status rmm_attention(const rmm_bf16* Q, const rmm_bf16* K, const rmm_bf16* V
   }
   CUtensorMap tq, tk, tv;
   if (rmm_status st = make_tmap(&tq, qsrc, ap.kp, items * nq, ap.kp * 2, 64, 128)) return st;
-  if (rmm_status st = make_tmap(&tk, ksrc, ap.kp, batch * hkv * nk, ap.kp * 2, 64, 128)) return st;
+  if (rmm_status st = make_tmap(&tk, ksrc, ap.kp, (ap.k_per_item ? items : batch * hkv) * nk, ap.kp * 2, 64, 128))
+    return st;
   if (rmm_status st = make_tmap(&tv, V, dh, batch * hkv * nk, dh * 2, 64, 64)) return st;
   cudaError_t e = cudaFuncSetAttribute(attn_pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnPPSmem);
   if (e != cudaSuccess) return cuda_fail(e, "attention attribute");
-  e = launch_chained(attn_pp_kernel, dim3(static_cast<unsigned>(items * ceil_div(m_tiles, 2))), dim3(320), kAttnPPSmem, s,
+  e = launch_chained(attn_pp_kernel, dim3(static_cast<unsigned>(items * ceil_div(m_tiles, 2))), dim3(kAttnPPThreads), kAttnPPSmem, s,
                      tq, tk, tv, ap);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return RMM_OK;

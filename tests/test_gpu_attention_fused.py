@@ -54,7 +54,7 @@ def qkv(hq, hkv, nq, nk, seed=40):
     return Q, K, V
 
 
-@pytest.mark.parametrize("rho", [0.5, 0.7, 1.0])
+@pytest.mark.parametrize("rho", [0.3, 0.5, 0.7, 1.0])
 @pytest.mark.parametrize("causal", [True, False])
 def test_fused_attention_small_gqa(rho, causal):
     """4 query / 2 key-value heads, 300 rows (ragged last query tile and key block)."""

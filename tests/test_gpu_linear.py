@@ -232,6 +232,21 @@ def test_gather_columns_short_rows(d, k, ld):
     assert not ap[:, k:].any()
 
 
+@pytest.mark.parametrize("d,k,ld,lda", [(128, 64, 64, 128), (128, 39, 64, 136), (64, 17, 24, 64), (256, 200, 256, 264)])
+def test_gather_columns_narrow_rows(d, k, ld, lda):
+    """Many rows of 64, 128 or 256 columns (the attention's packed score operands):
+    the 8-rows-per-warp staged gather; strided rows, kept columns in any order,
+    zero padding past k."""
+    g = synthetic.rng(45)
+    full = synthetic.to_bf16(g.standard_normal((16384, lda), dtype=np.float32)).cuda()
+    A = full[:, :d]
+    idx = torch.as_tensor(g.permutation(d)[:k], dtype=torch.int32).cuda()
+    ap = rmm.gather_columns(A, idx, ld_pack=ld)
+    torch.cuda.synchronize()
+    assert torch.equal(ap[:, :k], A[:, idx.long()])
+    assert not ap[:, k:].any()
+
+
 _DECODE_W = {}
 
 
