@@ -167,7 +167,7 @@ struct GemvI8TcParams {
   float* partial;      // [m_super + gridDim.x][4][n][128]
 };
 
-constexpr int kI8TcProducerWarps = 8;
+constexpr int kI8TcProducerWarps = 16;
 constexpr int kI8TcThreads = (kI8TcProducerWarps + 5) * 32;
 
 // sixteen int8 (one 16-byte load) -> sixteen bf16 (two 16-byte words)

@@ -460,7 +460,12 @@ __global__ void __launch_bounds__(256) pack_rows_bulk_kernel(const PackParams p,
     const bool got = mbar_wait(&full[q % NBUF], (q / NBUF) & 1, abort_flag, kDevErrTimeoutProducer);
     // row q has landed everywhere and every thread is done with row q - 1
     if (!__syncthreads_and(got)) break;
-    if (threadIdx.x == 0 && issued < static_cast<uint32_t>(nrows)) issue_next();  // into row q - 1's buffer
+    if (threadIdx.x == 0 && issued < static_cast<uint32_t>(nrows)) {
+      // every thread's reads of row q - 1's buffer (ordered before this point by
+      // the barrier) before the bulk copy into it: the issuing thread fences
+      fence_proxy_async_smem();
+      issue_next();  // into row q - 1's buffer
+    }
 
     const uint16_t* row = reinterpret_cast<const uint16_t*>(bufs + (q % NBUF) * buf_bytes);
     const uint32_t lim = static_cast<uint32_t>(pack_visible(p, gather_at.i));
@@ -473,7 +478,6 @@ __global__ void __launch_bounds__(256) pack_rows_bulk_kernel(const PackParams p,
       const uint32_t v1 = (j1 < lim) ? row[j1] : 0u;
       dst[t] = v0 | (v1 << 16);
     }
-    fence_proxy_async_smem();  // this row's reads are ordered before the next bulk copy into its buffer
     gather_at.next(p);
   }
   if (threadIdx.x == 0 && *abort_flag) {
