@@ -192,6 +192,9 @@ rmm_status launch_colsq_tma(const uint16_t* A, int64_t batch, int64_t bstride, i
   int W = 0, C = 0;
   int64_t best = 0;
   for (int w = 256; w >= 64; w /= 2) {
+    // a strip twice as wide as the matrix stages (and sums) as many zero columns
+    // as real ones: the narrower strip holds twice the rows per tile
+    if (w > 64 && w >= 2 * d) continue;
     const int64_t R = kColsqTileBytes / (2 * w);
     for (int c = 1; c <= 8; c *= 2) {
       if (c > 1 && n < c * 2 * R) break;
