@@ -12,16 +12,18 @@
 // (selecting P's columns would need all of P first).
 //
 // One CTA per (query head, pair of 128-row query tiles), see attn_pp_kernel:
-//   warp 0      TMA: both Q tiles once, then 128-key blocks of K (K-major, 128
-//               dims) and V (MN-major, 128 dims) into two-stage rings.
-//   warp 1      tensor memory (512 columns: S_A, S_B, O_A, O_B); lane 0 issues
-//               S_t(j) = Q_t K(j)^T (M = N = 128, K = 128) and O_t += P_t(j) V(j)
-//               (A = P_t from tensor memory, K = 128), alternating the tiles.
-//   warps 2..9  two softmax warpgroups (tile A: warps 2-5, tile B: 6-9), one
-//               query row per thread: running max m and sum l in log2 units,
-//               weights half by ex2.approx, half by a fitted polynomial on the
-//               FMA pipe, P written back as bf16 pairs into tensor memory, rows of
-//               O rescaled there when their maximum grew; at the end O / l.
+//   warp 0       TMA: both Q tiles once, then 128-key blocks of K (K-major) and V
+//                (MN-major, 128 dims) into two-stage rings.
+//   warp 1       tensor memory (512 columns: S_A, S_B, O_A, O_B); lane 0 issues
+//                S_t(j) = Q_t K(j)^T (M = N = 128, K = kp) and O_t += P_t(j) V(j)
+//                (A = P_t from tensor memory, K = 128), alternating the tiles.
+//   warps 2..17  softmax, two threads per query row (warps 2-9 tile A, 10-17
+//                tile B; in each tile the first four warps take keys 0-63 of a
+//                block, the next four keys 64-127): running max m and sum l in
+//                log2 units, weights by ex2.approx (in the masked diagonal
+//                blocks half of them by a fitted polynomial on the FMA pipe), P
+//                written back as bf16 pairs into tensor memory, O rescaled there
+//                when a row's maximum jumped; at the end O / l.
 // Every wait is bounded (about one second); on a timeout the CTA records an
 // error code, drains its copies, lets the MMA finish and returns.
 #pragma once
@@ -461,20 +463,14 @@ __global__ void __launch_bounds__(kAttnPPThreads, 1)
         tmem_ld_wait();
         uint32_t pk[16];
         if (full) {
-          // keys 4e, 4e+1 on the FMA pipe (packed pairs), 4e+2, 4e+3 on the
-          // special-function unit; scaling, sums and the polynomial two keys per
-          // instruction
+          // every key on the special-function unit (one instruction per key; the
+          // packed cubic takes ~2.5, and the unit has room at this rate)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint64_t xa =
-                attn_fma2(attn_f2(__uint_as_float(vc[4 * e]), __uint_as_float(vc[4 * e + 1])), sc2, nm2);
-            const uint64_t xb2 =
-                attn_fma2(attn_f2(__uint_as_float(vc[4 * e + 2]), __uint_as_float(vc[4 * e + 3])), sc2, nm2);
-            const uint64_t ya = attn_exp2_poly2(xa);
-            const uint64_t yb = attn_f2(attn_exp2(attn_lo(xb2)), attn_exp2(attn_hi(xb2)));
-            sum2[e & 1] = attn_add2(sum2[e & 1], attn_add2(ya, yb));
-            pk[2 * e] = attn_bf16x2(attn_lo(ya), attn_hi(ya));
-            pk[2 * e + 1] = attn_bf16x2(attn_lo(yb), attn_hi(yb));
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t xq = attn_fma2(attn_f2(__uint_as_float(vc[2 * e]), __uint_as_float(vc[2 * e + 1])), sc2, nm2);
+            const float y0 = attn_exp2(attn_lo(xq)), y1 = attn_exp2(attn_hi(xq));
+            sum2[e & 1] = attn_add2(sum2[e & 1], attn_f2(y0, y1));
+            pk[e] = attn_bf16x2(y0, y1);
           }
         } else {
 #pragma unroll
