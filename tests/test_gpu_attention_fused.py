@@ -46,11 +46,11 @@ def fused_parity(Q, K, V, rho, causal, scale, rows=None):
     return O, idx
 
 
-def qkv(hq, hkv, nq, nk, seed=40):
+def qkv(hq, hkv, nq, nk, seed=40, batch=1):
     g = synthetic.rng(seed)
-    Q = synthetic.to_bf16(g.standard_normal((1, hq, nq, 128), dtype=np.float32) * np.exp(g.standard_normal(128)).astype(np.float32))
-    K = synthetic.to_bf16(g.standard_normal((1, hkv, nk, 128), dtype=np.float32))
-    V = synthetic.to_bf16(g.standard_normal((1, hkv, nk, 128), dtype=np.float32))
+    Q = synthetic.to_bf16(g.standard_normal((batch, hq, nq, 128), dtype=np.float32) * np.exp(g.standard_normal(128)).astype(np.float32))
+    K = synthetic.to_bf16(g.standard_normal((batch, hkv, nk, 128), dtype=np.float32))
+    V = synthetic.to_bf16(g.standard_normal((batch, hkv, nk, 128), dtype=np.float32))
     return Q, K, V
 
 
@@ -60,6 +60,15 @@ def test_fused_attention_small_gqa(rho, causal):
     """4 query / 2 key-value heads, 300 rows (ragged last query tile and key block)."""
     Q, K, V = qkv(4, 2, 300, 300)
     fused_parity(Q, K, V, rho, causal, 0.088)
+
+
+@pytest.mark.parametrize("rho", [0.4, 0.8, 1.0])
+def test_fused_attention_batch_of_two(rho):
+    """Two batch items of 4 query / 2 key-value heads (different data per item):
+    the item index of Q, K, V and O, the packed operands (rho 0.4) and the zeroed
+    Q (rho 0.8) per item."""
+    Q, K, V = qkv(4, 2, 260, 260, seed=47, batch=2)
+    fused_parity(Q, K, V, rho, True, 0.09)
 
 
 def test_fused_attention_rectangular_causal():
