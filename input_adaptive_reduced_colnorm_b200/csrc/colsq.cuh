@@ -339,14 +339,17 @@ constexpr int kColsqShortMaxRows = 32;
 // matrix (n may be anything; used for n <= 32): rows summed 4 at a time in fp32
 // (exact bf16 squares) and folded into fp64, in row order.  Columns at or past d
 // read as 0.  Each column's arithmetic does not depend on CPT, and the decode
-// selection kernel computes its scores with this same function, so its keys are
-// bit-identical to colsq_short_kernel's.
-template <int CPT>
-__device__ __forceinline__ void colsq_short_cols(const uint16_t* A, int64_t lda, int64_t n, int64_t col0, int64_t d,
-                                                 double (&acc)[CPT]) {
+// selection kernel computes its scores with this same summation (reading its
+// rows from shared memory), so its keys are bit-identical to colsq_short_kernel's.
+//
+// The summation itself, over row chunks that ``row_words(r, w)`` supplies (the
+// CPT bf16 values of row r as CPT / 2 packed words): rows in batches of eight
+// (all eight fetched before any is used), four squares added in fp32, then each
+// group of four added to the fp64 total in row order.
+template <int CPT, typename RowWords>
+__device__ __forceinline__ void colsq_short_sum(int64_t n, RowWords&& row_words, double (&acc)[CPT]) {
   static_assert(CPT == 4 || CPT == 8, "four or eight columns per thread");
   constexpr int WPR = CPT / 2;  // 32-bit words per row chunk
-  const bool full = col0 + CPT <= d;
 #pragma unroll
   for (int e = 0; e < CPT; ++e) acc[e] = 0.0;
   for (int64_t r0 = 0; r0 < n; r0 += 8) {
@@ -355,25 +358,7 @@ __device__ __forceinline__ void colsq_short_cols(const uint16_t* A, int64_t lda,
     for (int u = 0; u < 8; ++u) {
 #pragma unroll
       for (int q = 0; q < WPR; ++q) w[u][q] = 0u;
-      if (r0 + u < n) {
-        const uint16_t* src = A + (r0 + u) * lda + col0;
-        if (full) {
-          if constexpr (CPT == 8) {
-            const uint4 v = ldg_nc_v4(src);
-            w[u][0] = v.x;
-            w[u][1] = v.y;
-            w[u][2] = v.z;
-            w[u][3] = v.w;
-          } else {
-            const uint2 v = ldg_nc_v2(src);
-            w[u][0] = v.x;
-            w[u][1] = v.y;
-          }
-        } else {
-          for (int e = 0; e < CPT; ++e)
-            if (col0 + e < d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
-        }
-      }
+      if (r0 + u < n) row_words(r0 + u, w[u]);
     }
 #pragma unroll
     for (int g = 0; g < 8; g += 4) {
@@ -392,6 +377,36 @@ __device__ __forceinline__ void colsq_short_cols(const uint16_t* A, int64_t lda,
       for (int e = 0; e < CPT; ++e) acc[e] += static_cast<double>(a32[e]);
     }
   }
+}
+
+// Columns col0 .. col0 + CPT - 1 of A read from global memory.
+template <int CPT>
+__device__ __forceinline__ void colsq_short_cols(const uint16_t* A, int64_t lda, int64_t n, int64_t col0, int64_t d,
+                                                 double (&acc)[CPT]) {
+  constexpr int WPR = CPT / 2;
+  const bool full = col0 + CPT <= d;
+  colsq_short_sum<CPT>(
+      n,
+      [&](int64_t r, uint32_t(&w)[WPR]) {
+        const uint16_t* src = A + r * lda + col0;
+        if (full) {
+          if constexpr (CPT == 8) {
+            const uint4 v = ldg_nc_v4(src);
+            w[0] = v.x;
+            w[1] = v.y;
+            w[2] = v.z;
+            w[3] = v.w;
+          } else {
+            const uint2 v = ldg_nc_v2(src);
+            w[0] = v.x;
+            w[1] = v.y;
+          }
+        } else {
+          for (int e = 0; e < CPT; ++e)
+            if (col0 + e < d) w[e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
+        }
+      },
+      acc);
 }
 
 __global__ void __launch_bounds__(128) colsq_short_kernel(const ColsqParams p) {

@@ -8,20 +8,25 @@
 // microseconds, and one CTA selecting over d = 8192 keys is issue-bound, so the
 // work is spread over one cluster of C CTAs of 256 threads (C <= 8):
 //   * each thread owns KPT consecutive columns (4 while 8 CTAs of 1024 columns
-//     cover d, i.e. d <= 8192; else 8, d <= 16384) and computes their fp64 scores
-//     with the arithmetic of the short-matrix column-score kernel (bit-identical
-//     keys); CTA r owns columns [256 KPT r, 256 KPT (r + 1));
+//     cover d, i.e. d <= 8192; else 8, d <= 16384); CTA r owns columns
+//     [256 KPT r, 256 KPT (r + 1)).  The thread copies its chunk of every row
+//     into shared memory with cp.async (all rows in flight at once, where
+//     batches of eight register loads cost one round trip each), computes the
+//     fp64 scores from there with the arithmetic of the short-matrix
+//     column-score kernel (bit-identical keys), and packs x[:, I] from the same
+//     copy at the end;
 //   * the k-th largest key is found by an MSB-first radix select over the
 //     64-bit key patterns (non-negative doubles order like their bits): leading
 //     bits shared by every key are skipped (cluster-wide AND / OR), each pass
 //     resolves 8 bits with per-warp histograms merged per CTA and then across
-//     the cluster through distributed shared memory, one cluster barrier per
-//     pass; the same barrier carries each pass's AND / OR of the bucket's
+//     the cluster through distributed shared memory (each thread reads its bin
+//     from every CTA with independent loads), one cluster barrier per pass; the same barrier carries each pass's AND / OR of the bucket's
 //     members, so bits the bucket shares are skipped and a bucket of identical
 //     keys (squares of a single bf16 row) ends the passes at once;
 //   * the compaction takes every key above the threshold and the lowest-index
 //     keys equal to it, in index order: counts are exchanged once across the
-//     cluster (CTA order is column order), then two block scans give each
+//     cluster (CTA order is column order; warp 0 reads the lower CTAs' counts
+//     in parallel and scans them), then two block scans give each
 //     thread its positions; the thread writes I and, for its kept columns,
 //     x[:, I] (zero-padded to the packed row length).
 // Every count is an integer, so the result does not depend on atomic order.
@@ -50,6 +55,8 @@ constexpr int kDecSelMaxCtas = 8;                // portable cluster size
 constexpr int kDecSelMaxD = kDecSelThreads * 8 * kDecSelMaxCtas;
 __host__ __device__ constexpr int decsel_cols_per_cta(int kpt) { return kDecSelThreads * kpt; }
 constexpr int kDecSelMaxRows = 32;
+// shared memory for the staged rows: n rows x 256 threads x KPT bf16
+__host__ __device__ constexpr int decsel_stage_bytes(int n, int kpt) { return n * kDecSelThreads * kpt * 2; }
 
 // The two halves of a cluster barrier, for work that can overlap its latency.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
@@ -127,6 +134,7 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   __shared__ int s_digit, s_above, s_cnt;
   __shared__ int s_counts[2];  // this CTA's keys above the threshold / equal to it (read by the cluster)
   __shared__ int s_sel_base, s_eq_before;
+  extern __shared__ __align__(16) uint8_t s_rows[];  // [n][kDecSelThreads][KPT] bf16
 
   wait_prior_kernels();
   const int C = static_cast<int>(gridDim.x);  // the grid is one cluster
@@ -134,13 +142,60 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t col0 = static_cast<int64_t>(rank) * decsel_cols_per_cta(KPT) + tid * KPT;
 
+  // ---- this thread's chunk of every row, staged in shared memory
+  constexpr int WPR = KPT / 2;  // 32-bit words per row chunk
+  const bool full = col0 + KPT <= p.d;
+  uint8_t* my_rows = s_rows + tid * (KPT * 2);
+  constexpr int kRowStride = kDecSelThreads * KPT * 2;
+  if (col0 < p.d) {
+    if (full) {
+      // x is 16-byte aligned with a row pitch of a multiple of 8 elements, so
+      // each chunk (8 or 16 bytes) is aligned
+      for (int r = 0; r < p.n; ++r) {
+        const uint16_t* src = p.x + static_cast<int64_t>(r) * p.ldx + col0;
+        const uint32_t dst = smem_u32(my_rows + r * kRowStride);
+        if constexpr (KPT == 8)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+        else
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else {
+      for (int r = 0; r < p.n; ++r) {
+        const uint16_t* src = p.x + static_cast<int64_t>(r) * p.ldx + col0;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(my_rows + r * kRowStride);
+        for (int q = 0; q < WPR; ++q) {
+          uint32_t v = 0u;
+          for (int e = 2 * q; e < 2 * q + 2; ++e)
+            if (col0 + e < p.d) v |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
+          dst[q] = v;
+        }
+      }
+    }
+  }
+  // each thread reads back only what it copied itself
+  auto row_words = [&](int64_t r, uint32_t(&w)[WPR]) {
+    const uint8_t* src = my_rows + r * kRowStride;
+    if constexpr (KPT == 8) {
+      const uint4 v = *reinterpret_cast<const uint4*>(src);
+      w[0] = v.x;
+      w[1] = v.y;
+      w[2] = v.z;
+      w[3] = v.w;
+    } else {
+      const uint2 v = *reinterpret_cast<const uint2*>(src);
+      w[0] = v.x;
+      w[1] = v.y;
+    }
+  };
+
   // ---- scores (fp64, bit-identical to colsq_short_kernel) and their key patterns
   uint64_t key[KPT];
   uint32_t valid = 0;
   {
     double acc[KPT];
     if (col0 < p.d) {
-      colsq_short_cols<KPT>(p.x, p.ldx, p.n, col0, p.d, acc);
+      colsq_short_sum<KPT>(p.n, row_words, acc);
     } else {
 #pragma unroll
       for (int e = 0; e < KPT; ++e) acc[e] = 0.0;
@@ -242,9 +297,14 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
     }
     // thread t takes digit 255 - t, so the exclusive scan in thread order counts the larger digits
     const int bin = 255 - tid;
-    uint32_t cnt = 0;
     const uint32_t haddr = smem_u32(hb + bin);
-    for (int q = 0; q < C; ++q) cnt += ld_shared_cluster_u32(map_shared_rank(haddr, static_cast<uint32_t>(q)));
+    uint32_t hv[kDecSelMaxCtas];
+#pragma unroll
+    for (int q = 0; q < kDecSelMaxCtas; ++q)
+      hv[q] = q < C ? ld_shared_cluster_u32(map_shared_rank(haddr, static_cast<uint32_t>(q))) : 0u;
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int q = 0; q < kDecSelMaxCtas; ++q) cnt += hv[q];
     const int above = block_exclusive_scan<kDecSelThreads>(static_cast<int>(cnt), s_warp, &s_total);
     if (bin <= static_cast<int>(dmask) && above < need && need <= above + static_cast<int>(cnt)) {
       s_digit = bin;
@@ -309,19 +369,31 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
     s_counts[1] = eq_cta;
   }
   cluster_sync();
-  if (tid == 0) {
-    int sel_before = 0, eq_before = 0;
-    const uint32_t base = smem_u32(s_counts);
-    for (int q = 0; q < rank; ++q) {
-      const int g = static_cast<int>(ld_shared_cluster_u32(map_shared_rank(base, static_cast<uint32_t>(q))));
-      const int e = static_cast<int>(ld_shared_cluster_u32(map_shared_rank(base + 4, static_cast<uint32_t>(q))));
-      int taken = take ? e : need - eq_before;
-      taken = taken < 0 ? 0 : (taken > e ? e : taken);
-      sel_before += g + taken;
-      eq_before += e;
+  if (warp == 0) {
+    // lane q < rank holds CTA q's counts; the keys equal to the threshold that
+    // CTA q takes depend on those of the CTAs before it (an exclusive scan)
+    int g = 0, e = 0;
+    if (lane < rank) {
+      const uint32_t base = smem_u32(s_counts);
+      g = static_cast<int>(ld_shared_cluster_u32(map_shared_rank(base, static_cast<uint32_t>(lane))));
+      e = static_cast<int>(ld_shared_cluster_u32(map_shared_rank(base + 4, static_cast<uint32_t>(lane))));
     }
-    s_sel_base = sel_before;
-    s_eq_before = eq_before;
+    int e_incl = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, e_incl, o);
+      if (lane >= o) e_incl += y;
+    }
+    int taken = take ? e : need - (e_incl - e);
+    taken = taken < 0 ? 0 : (taken > e ? e : taken);
+    int sel_before = g + taken;  // 0 for lanes at or past rank
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sel_before += __shfl_xor_sync(0xffffffffu, sel_before, o);
+    const int eq_before = __shfl_sync(0xffffffffu, e_incl, 31);
+    if (lane == 0) {
+      s_sel_base = sel_before;
+      s_eq_before = eq_before;
+    }
   }
   __syncthreads();
   // no CTA reads another's shared memory past this point: arrive now, and wait
@@ -346,45 +418,15 @@ __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(const Dec
   }
   if (p.xpack != nullptr) {
     if (sel != 0u) {
-      // eight rows' loads are issued before any of their stores, so each batch
-      // costs one round trip instead of eight
-      const bool full = col0 + KPT <= p.d;
-      constexpr int WPR = KPT / 2;  // 32-bit words per row chunk
-      for (int r0 = 0; r0 < p.n; r0 += 8) {
-        uint32_t w[8][WPR];
+      // from the staged copy of the thread's columns
+      for (int r = 0; r < p.n; ++r) {
+        uint32_t w[WPR];
+        row_words(r, w);
+        uint16_t* dst = p.xpack + static_cast<int64_t>(r) * p.ld_pack;
+        int pos = pos0;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-#pragma unroll
-          for (int q = 0; q < WPR; ++q) w[u][q] = 0u;
-          if (r0 + u < p.n) {
-            const uint16_t* src = p.x + static_cast<int64_t>(r0 + u) * p.ldx + col0;
-            if (full) {
-              if constexpr (KPT == 8) {
-                const uint4 v = ldg_nc_v4(src);
-                w[u][0] = v.x;
-                w[u][1] = v.y;
-                w[u][2] = v.z;
-                w[u][3] = v.w;
-              } else {
-                const uint2 v = ldg_nc_v2(src);
-                w[u][0] = v.x;
-                w[u][1] = v.y;
-              }
-            } else {
-              for (int e = 0; e < KPT; ++e)
-                if (col0 + e < p.d) w[u][e >> 1] |= static_cast<uint32_t>(__ldg(src + e)) << (16 * (e & 1));
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (r0 + u >= p.n) break;
-          uint16_t* dst = p.xpack + static_cast<int64_t>(r0 + u) * p.ld_pack;
-          int pos = pos0;
-#pragma unroll
-          for (int e = 0; e < KPT; ++e)
-            if ((sel >> e) & 1u) dst[pos++] = static_cast<uint16_t>(w[u][e >> 1] >> (16 * (e & 1)));
-        }
+        for (int e = 0; e < KPT; ++e)
+          if ((sel >> e) & 1u) dst[pos++] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
       }
     }
     if (rank == C - 1 && tid < p.n)

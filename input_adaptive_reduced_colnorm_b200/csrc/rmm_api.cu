@@ -369,9 +369,11 @@ rmm_status launch_decode_select(const uint16_t* x, int64_t n, int64_t d, int64_t
   // four columns per thread while a cluster of at most 8 CTAs covers d, else eight
   const bool four = d <= decsel_cols_per_cta(4) * kDecSelMaxCtas;
   const int C = static_cast<int>(ceil_div(d, decsel_cols_per_cta(four ? 4 : 8)));
-  const cudaError_t e =
-      four ? launch_cluster(decode_select_kernel<4>, dim3(static_cast<unsigned>(C)), dim3(kDecSelThreads), 0, C, s, p)
-           : launch_cluster(decode_select_kernel<8>, dim3(static_cast<unsigned>(C)), dim3(kDecSelThreads), 0, C, s, p);
+  auto kern = four ? decode_select_kernel<4> : decode_select_kernel<8>;
+  const int smem = decsel_stage_bytes(static_cast<int>(n), four ? 4 : 8);  // the staged rows
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "decode selection attribute");
+  e = launch_cluster(kern, dim3(static_cast<unsigned>(C)), dim3(kDecSelThreads), static_cast<size_t>(smem), C, s, p);
   if (e != cudaSuccess) return cuda_fail(e, "decode selection launch");
   return RMM_OK;
 }
