@@ -316,11 +316,48 @@ def bench_workloads(dev, stream, L, reps=10, warm=3):
         nbytes = kept_bytes(n, d, m, rho)
         return {"k": k, "ms": ms, "tflops": 2.0 * n * k * m / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9}
 
-    # single linear layer, 128 x 1024 x 1024, rho = 0.5 (latency-bound)
+    def graph_call_ms(call, calls=20, replays=5):
+        """Per-call time of ``call(stream)`` replayed from one CUDA graph that holds
+        ``calls`` back-to-back calls: the device time of a launch-bound call
+        without the per-kernel host work of an eager call."""
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                call(ctypes.c_void_p(side.cuda_stream))
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(calls):
+                call(ctypes.c_void_p(side.cuda_stream))
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(replays):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del g
+        return e0.elapsed_time(e1) / (calls * replays)
+
+    # single linear layer, 128 x 1024 x 1024, rho = 0.5 (latency-bound): eager
+    # calls, and the same call replayed from a CUDA graph
     A, B = synthetic.linear_small()
     A, B = A.to(dev), B.to(dev)
     r05, r1 = linear_case(A, B, 0.5), linear_case(A, B, 1.0)
-    out["linear_128x1024x1024"] = {"0.5": r05, "1.0": r1, "speedup_vs_rho1": r1["ms"] / r05["ms"]}
+    for r, row in ((0.5, r05), (1.0, r1)):
+        n_, d_ = A.shape
+        m_ = B.shape[1]
+        Yg = torch.empty((n_, m_), dtype=torch.bfloat16, device=dev)
+        wsg = torch.empty(max(L.rmm_linear_workspace_bytes(n_, d_, m_, r), 256), dtype=torch.uint8, device=dev)
+        row["graph_ms"] = graph_call_ms(lambda st: ok(L.rmm_linear(A.data_ptr(), n_, d_, d_, B.data_ptr(), m_, m_,
+                                                                   Yg.data_ptr(), m_, r, None, wsg.data_ptr(),
+                                                                   wsg.numel(), st)))
+    out["linear_128x1024x1024"] = {"0.5": r05, "1.0": r1, "speedup_vs_rho1": r1["ms"] / r05["ms"],
+                                   "graph_speedup_vs_rho1": r1["graph_ms"] / r05["graph_ms"]}
 
     # decode GEMV, Llama-3.1-70B MLP-up: x n x 8192, W 8192 x 28672 (HBM-bound on kept W rows)
     _, W = synthetic.decode_gemv(1)
